@@ -1,0 +1,330 @@
+"""Plain fp64 CPU oracle for RTPurbo-style head-wise hybrid attention.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg use this module. The CUDA library never imports
+it and it shares no code with the CUDA sources.
+
+What it computes, step by step (the sources, by page and paragraph):
+
+* Head-wise split: about 15% of heads are retrieval heads, the rest are
+  streaming heads that run sliding-window attention with a window of 8192
+  (RTPurboV2 article, th-motor.com: the paragraphs on retrieval vs streaming
+  heads and on the Qwen3-Coder-30B-A3B recipe). The split is an input here.
+* Indexer: a per-KV-head low-rank projector maps the head dimension D to
+  r = 16 (RTPurboV2 article, paragraph on the low-rank projector); it is a
+  cheap scout whose scores pick candidates, after which exact attention runs
+  at full dimension on the small selected set (RTPurbo digest, Telegram
+  channel "Data analysis", post 5185).
+* Block score for prefill: the maximum of the projected dot product over the
+  (query, key) pairs of a 64 x 64 block pair; each query block keeps its top-k
+  causal key blocks plus key block 0 (the sink) plus the window blocks (the
+  tiny 2K-token prefill workload statement).
+* Decode: token-level top-k over the whole cache by the projected score,
+  unioned with the last W tokens and token 0, then exact softmax attention
+  (the 128K-context decode workload statement).
+
+Readings taken where the sources are silent (each one is used identically by
+the CUDA path, which is written separately from the same text):
+
+* softmax scale ``1/sqrt(D)`` is passed explicitly as ``scale``;
+* query head ``h`` reads KV head ``h // (Hq/Hkv)``; its projector is that KV
+  head's;
+* inputs are taken as already position-encoded (no RoPE is applied);
+* prefill top-k ranks *every* causal key block ``j <= i`` (sink and window
+  blocks included), and only then is the union with sink and window taken;
+* the block score of the diagonal block uses causal pairs only (``u <= t``);
+* the retrieval heads' prefill window is block-granular: the ``W/64`` key
+  blocks ending at the diagonal block, with the causal mask inside the
+  diagonal block;
+* the SWA window holds ``W`` keys including the query itself,
+  ``t - W < u <= t``;
+* keys are a set: a key reached twice (selected and in the window) counts once;
+* exact score ties rank the smaller index first;
+* the stored key index and the prefill query index are rounded to bf16
+  (round-to-nearest-even of the exact sum); the decode query index stays
+  unrounded (fp32 on the GPU, fp64 here);
+* when fewer candidates than ``k`` exist, all are taken (``-1`` pads the rest).
+
+Parity pins live in ``tests/test_oracle_pins.py``; every function below is
+pinned there (no function here is parity unpinned).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+BLOCK = 64
+
+
+# ---------------------------------------------------------------------------
+# bf16 rounding
+# ---------------------------------------------------------------------------
+def bf16_round(x) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 value, ties to even.
+
+    bf16 keeps 8 significant bits and fp32's exponent range; below 2**-126 the
+    spacing is fixed at 2**-133 (subnormals). Returned as fp64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros_like(x)
+    nz = x != 0
+    _, e = np.frexp(x[nz])                       # x = m * 2**e, 0.5 <= |m| < 1
+    exp_unbiased = np.maximum(e - 1, -126)       # floor(log2|x|), clamped at the subnormal range
+    quantum = np.ldexp(1.0, exp_unbiased - 7)    # spacing of 8 significant bits
+    out[nz] = np.rint(x[nz] / quantum) * quantum  # np.rint: round half to even
+    return out
+
+
+def to_f64(t) -> np.ndarray:
+    """A torch tensor or array (any float dtype) as fp64 numpy (bf16 -> fp64 is exact)."""
+    try:
+        import torch
+        if isinstance(t, torch.Tensor):
+            return t.detach().to("cpu").to(torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(t, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Index projection (low-rank projector D -> r)
+# ---------------------------------------------------------------------------
+def project(x, P, round_to_bf16: bool = True) -> np.ndarray:
+    """x_tilde = x @ P for rows ``x[..., D]`` and one projector ``P[D, r]``.
+
+    The sum is taken in fp64 (every bf16 x bf16 product is exact there), then
+    rounded once to bf16 when the result is a stored index.
+    """
+    y = np.matmul(to_f64(x), to_f64(P))
+    return bf16_round(y) if round_to_bf16 else y
+
+
+# ---------------------------------------------------------------------------
+# Prefill selection
+# ---------------------------------------------------------------------------
+def block_scores(qt, kt, i: int, block: int = BLOCK, key_chunk_blocks: int = 4096) -> np.ndarray:
+    """s[j] for j = 0..i: max over causal pairs (t in query block i, u in key
+    block j, u <= t) of qt[t] . kt[u].
+
+    ``qt`` [N, r] and ``kt`` [N, r] are one head's projected queries and keys.
+    The keys are visited in chunks of ``key_chunk_blocks`` blocks only to bound
+    the temporary; a maximum does not depend on the order it is taken in.
+    """
+    qt = to_f64(qt)
+    kt = to_f64(kt)
+    qb = qt[i * block:(i + 1) * block]                       # [64, r]
+    t_pos = np.arange(i * block, (i + 1) * block)
+    out = np.empty(i + 1)
+    for j0 in range(0, i + 1, key_chunk_blocks):
+        j1 = min(i + 1, j0 + key_chunk_blocks)
+        kb = kt[j0 * block:j1 * block]                       # [(j1-j0)*64, r]
+        s = qb @ kb.T                                        # [64, (j1-j0)*64]
+        u_pos = np.arange(j0 * block, j1 * block)
+        s = np.where(u_pos[None, :] <= t_pos[:, None], s, -np.inf)
+        out[j0:j1] = s.reshape(block, j1 - j0, block).max(axis=(0, 2))
+    return out
+
+
+def topk_desc(scores, k: int) -> np.ndarray:
+    """Indices of the k largest scores (ties: smaller index first), ascending.
+
+    With ``len(scores) <= k`` every index is returned.
+    """
+    scores = np.asarray(scores, dtype=np.float64)
+    n = scores.shape[0]
+    if n <= k:
+        return np.arange(n, dtype=np.int64)
+    order = np.lexsort((np.arange(n), -scores))   # primary: score desc; secondary: index asc
+    return np.sort(order[:k])
+
+
+def select_prefill(qt, kt, topk: int, qblocks=None, block: int = BLOCK):
+    """Top-k causal key blocks for each query block of one head.
+
+    Returns ``(sel, scores)``: dicts keyed by query block i, ``sel[i]`` the
+    ascending selected block indices (min(k, i+1) of them), ``scores[i]`` the
+    block scores s[0..i] used for the ranking.
+    """
+    N = to_f64(qt).shape[0]
+    nb = N // block
+    qblocks = range(nb) if qblocks is None else qblocks
+    sel, scores = {}, {}
+    for i in qblocks:
+        s = block_scores(qt, kt, i, block)
+        scores[i] = s
+        sel[i] = topk_desc(s, topk)
+    return sel, scores
+
+
+def attended_blocks(sel_i, i: int, window_blocks: int, sink_blocks: int) -> np.ndarray:
+    """Key blocks attended by query block i: selected, sink blocks and the
+    window blocks ending at the diagonal, as an ascending set."""
+    win = np.arange(max(0, i - window_blocks + 1), i + 1)
+    sink = np.arange(0, min(sink_blocks, i + 1))
+    return np.unique(np.concatenate([np.asarray(sel_i, dtype=np.int64), sink, win]))
+
+
+# ---------------------------------------------------------------------------
+# Exact attention
+# ---------------------------------------------------------------------------
+def attend(q_rows, q_pos, keys, values, key_pos, scale: float, window=None) -> np.ndarray:
+    """Softmax attention of each query row over the given keys, keeping only
+    keys at positions <= the query's position (and, with ``window``, only keys
+    at positions > the query's position - window).
+
+    ``q_rows`` [m, D], ``q_pos`` [m], ``keys``/``values`` [n, D], ``key_pos`` [n].
+    fp64 throughout, max-subtracted exponentials.
+    """
+    q_rows, keys, values = to_f64(q_rows), to_f64(keys), to_f64(values)
+    logits = scale * (q_rows @ keys.T)                         # [m, n]
+    kp = np.asarray(key_pos)[None, :]
+    qp = np.asarray(q_pos)[:, None]
+    ok = kp <= qp
+    if window is not None:
+        ok &= kp > qp - window
+    logits = np.where(ok, logits, -np.inf)
+    m = logits.max(axis=1, keepdims=True)
+    p = np.exp(logits - m)
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ values
+
+
+def sparse_attn_prefill_block(q, k, v, i: int, attended, scale: float,
+                              block: int = BLOCK) -> np.ndarray:
+    """Output rows of query block i of one retrieval head.
+
+    ``q`` [N, D] (that head), ``k``/``v`` [N, D] (its KV head), ``attended``
+    the ascending key-block set.
+    """
+    rows = np.arange(i * block, (i + 1) * block)
+    key_pos = np.concatenate([np.arange(j * block, (j + 1) * block) for j in attended])
+    return attend(to_f64(q[rows]), rows, to_f64(k[key_pos]), to_f64(v[key_pos]), key_pos, scale)
+
+
+def swa_rows(q, k, v, rows, window: int, scale: float, q_pos0: int = 0) -> np.ndarray:
+    """Sliding-window attention for query rows ``rows`` of one head.
+
+    Query row t sits at position ``q_pos0 + t`` and attends the keys u with
+    ``pos - window < u <= pos`` (and u inside the key array).
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    pos = q_pos0 + rows
+    Nk = k.shape[0]
+    lo, hi = max(0, int(pos.min()) - window + 1), min(Nk, int(pos.max()) + 1)
+    kp = np.arange(lo, hi)
+    return attend(to_f64(q[rows]), pos, to_f64(k[lo:hi]), to_f64(v[lo:hi]), kp, scale, window)
+
+
+# ---------------------------------------------------------------------------
+# Decode
+# ---------------------------------------------------------------------------
+def decode_scores(qt, kt) -> np.ndarray:
+    """score_u = qt . kt[u] for every cached token u (qt [r], kt [L, r])."""
+    return to_f64(kt) @ to_f64(qt)
+
+
+def select_decode(qt, kt, topk: int) -> np.ndarray:
+    """Token-level top-k over the whole cache (ascending indices)."""
+    return topk_desc(decode_scores(qt, kt), topk)
+
+
+def decode_attended(sel, L: int, window: int, sink: int) -> np.ndarray:
+    """Selected tokens, tokens 0..sink-1 and the last ``window`` tokens, as a set."""
+    return np.unique(np.concatenate([np.asarray(sel, dtype=np.int64),
+                                     np.arange(0, min(sink, L)),
+                                     np.arange(max(0, L - window), L)]))
+
+
+def attend_decode(q, kc, vc, keys_idx, scale: float) -> np.ndarray:
+    """One query (at the last position) over the cache rows ``keys_idx``."""
+    keys_idx = np.asarray(keys_idx, dtype=np.int64)
+    L = kc.shape[0]
+    return attend(to_f64(q)[None, :], [L - 1], to_f64(kc[keys_idx]), to_f64(vc[keys_idx]),
+                  keys_idx, scale)[0]
+
+
+# ---------------------------------------------------------------------------
+# Whole-layer drivers
+# ---------------------------------------------------------------------------
+def kv_of(h: int, Hq: int, Hkv: int) -> int:
+    return h // (Hq // Hkv)
+
+
+def prefill_layer(q, k, v, P, ret_heads, window: int, ret_window: int, topk: int,
+                  scale: float, qblocks=None, sink_blocks: int = 1, heads=None,
+                  block: int = BLOCK):
+    """One prefill layer for batch element 0-sliced tensors.
+
+    ``q`` [N, Hq, D], ``k``/``v`` [N, Hkv, D], ``P`` [Hkv, D, r] (bf16 values).
+    Computes the output rows of the query blocks ``qblocks`` (default: all)
+    for ``heads`` (default: all). Returns a dict with ``out`` {(h, i): [64, D]},
+    ``sel``/``scores`` {(h, i): ...} for retrieval heads, and ``kt``/``qt``.
+    """
+    P = to_f64(P)
+    N, Hq, D = q.shape
+    Hkv = k.shape[1]
+    nb = N // block
+    qblocks = list(range(nb)) if qblocks is None else list(qblocks)
+    heads = list(range(Hq)) if heads is None else list(heads)
+    ret = set(ret_heads)
+    wb = ret_window // block
+    kt_cache, res = {}, dict(out={}, sel={}, scores={}, kt={}, qt={})
+    for h in heads:
+        g = kv_of(h, Hq, Hkv)
+        if h in ret:
+            if g not in kt_cache:
+                kt_cache[g] = project(k[:, g, :], P[g])
+            kt = kt_cache[g]
+            qt = project(q[:, h, :], P[g])
+            res["kt"][g], res["qt"][h] = kt, qt
+            sel, sc = select_prefill(qt, kt, topk, qblocks, block)
+            for i in qblocks:
+                att = attended_blocks(sel[i], i, wb, sink_blocks)
+                res["sel"][(h, i)] = sel[i]
+                res["scores"][(h, i)] = sc[i]
+                res["out"][(h, i)] = sparse_attn_prefill_block(q[:, h, :], k[:, g, :], v[:, g, :],
+                                                               i, att, scale, block)
+        else:
+            for i in qblocks:
+                rows = np.arange(i * block, (i + 1) * block)
+                res["out"][(h, i)] = swa_rows(q[:, h, :], k[:, g, :], v[:, g, :], rows,
+                                              window, scale)
+    return res
+
+
+def decode_layer(q, kc, vc, P, ret_heads, window: int, ret_window: int, topk: int,
+                 scale: float, sink: int = 1, heads=None):
+    """One decode step for one sequence.
+
+    ``q`` [Hq, D], ``kc``/``vc`` [L, Hkv, D], ``P`` [Hkv, D, r]. The key index
+    is the bf16-rounded projection of the cache; the query index is unrounded.
+    Returns ``out`` {h: [D]}, ``sel``/``scores`` {h: ...}.
+    """
+    q, P = to_f64(q), to_f64(P)
+    Hq, D = q.shape
+    L, Hkv, _ = kc.shape
+    heads = list(range(Hq)) if heads is None else list(heads)
+    ret = set(ret_heads)
+    res = dict(out={}, sel={}, scores={}, kt={})
+    for h in heads:
+        g = kv_of(h, Hq, Hkv)
+        if h in ret:
+            if g not in res["kt"]:
+                res["kt"][g] = project(kc[:, g, :], P[g])
+            kt = res["kt"][g]
+            qt = project(q[h], P[g], round_to_bf16=False)
+            sc = decode_scores(qt, kt)
+            sel = topk_desc(sc, topk)
+            res["sel"][h], res["scores"][h] = sel, sc
+            idx = decode_attended(sel, L, ret_window, sink)
+        else:
+            idx = np.arange(max(0, L - window), L)
+        res["out"][h] = attend_decode(q[h], kc[:, g, :], vc[:, g, :], idx, scale)
+    return res
+
+
+__all__ = [
+    "BLOCK", "bf16_round", "to_f64", "project", "block_scores", "topk_desc", "select_prefill",
+    "attended_blocks", "attend", "sparse_attn_prefill_block", "swa_rows", "decode_scores",
+    "select_decode", "decode_attended", "attend_decode", "kv_of", "prefill_layer",
+    "decode_layer",
+]

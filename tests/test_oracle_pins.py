@@ -1,0 +1,429 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself.
+
+Kinds of pin used here:
+  * hand-worked examples (``tests/golden/*.json``, each with its derivation);
+  * special cases that reduce to a library routine (torch's float64
+    ``scaled_dot_product_attention`` with an explicit mask, torch's bf16 cast);
+  * closed forms (window 1 returns the query's own value row; two keys with a
+    known logit gap);
+  * brute force on tiny inputs (pure-Python loops over every pair and a full
+    sort, ``tests/brute.py``);
+  * invariants (convex hull, key permutation, counts, causal-only blocks).
+
+The last section plants plausible mistakes in copies of the oracle's
+functions and checks that a pin above catches each one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import brute
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(12345)
+
+
+def _bf16_arr(shape, scale=1.0, rs=rng):
+    return O.bf16_round(rs.standard_normal(shape) * scale)
+
+
+def _sdpa_masked(q, k, v, mask, scale):
+    """torch float64 SDPA for one head: q [m,D], k/v [n,D], mask [m,n] bool (True = attend)."""
+    qt = torch.from_numpy(q)[None, None]
+    kt = torch.from_numpy(k)[None, None]
+    vt = torch.from_numpy(v)[None, None]
+    mt = torch.from_numpy(mask)[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mt,
+                                                            scale=scale)[0, 0].numpy()
+
+
+# ---------------------------------------------------------------------------
+# bf16 rounding
+# ---------------------------------------------------------------------------
+def test_bf16_round_known_values():
+    one = 1.0
+    cases = {
+        one: one,
+        one + 2.0 ** -8: one,                           # midpoint, ties to even (mantissa 0)
+        one + 3 * 2.0 ** -8: one + 2.0 ** -6,           # midpoint between m=1 and m=2 -> even m=2
+        one + 2.0 ** -8 + 2.0 ** -20: one + 2.0 ** -7,  # just above the midpoint
+        -(one + 3 * 2.0 ** -8): -(one + 2.0 ** -6),
+        3.0 * 2.0 ** -134: 2.0 ** -132,                 # subnormal: 1.5 quanta of 2**-133 -> 2 quanta
+        2.0 ** -135: 0.0,                               # quarter quantum -> 0
+        0.0: 0.0,
+    }
+    for x, want in cases.items():
+        assert O.bf16_round(np.array([x]))[0] == want, x
+
+
+def test_bf16_round_matches_torch_cast_on_fp32_values():
+    x = (rng.standard_normal(200000) * np.exp(rng.uniform(-20, 20, 200000))).astype(np.float32)
+    x = np.concatenate([x, np.float32([1e-39, -3e-40, 65504.0, 3.3895e38])])
+    want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    got = O.bf16_round(x.astype(np.float64))
+    np.testing.assert_array_equal(got, want)
+
+
+# ---------------------------------------------------------------------------
+# Projection
+# ---------------------------------------------------------------------------
+def test_project_identity_columns_exact():
+    x = _bf16_arr((300, 128), 3.0)
+    P = np.zeros((128, 16))
+    P[np.arange(16), np.arange(16)] = 1.0
+    np.testing.assert_array_equal(O.project(x, P), x[:, :16])
+
+
+def test_project_single_entries_closed_form():
+    # column c picks 2**-c times component (5c mod 128): every result is exact.
+    x = _bf16_arr((64, 128))
+    P = np.zeros((128, 16))
+    for c in range(16):
+        P[(5 * c) % 128, c] = 2.0 ** -c
+    want = np.stack([x[:, (5 * c) % 128] * 2.0 ** -c for c in range(16)], axis=1)
+    np.testing.assert_array_equal(O.project(x, P), want)
+
+
+def test_project_rounds_once_to_bf16():
+    x = np.zeros((1, 128))
+    x[0, 0] = 1.0
+    x[0, 1] = 2.0 ** -8          # 1 + 2**-8 is a bf16 tie -> 1.0
+    x[0, 2] = 2.0 ** -30         # pushes it above the tie -> 1 + 2**-7
+    P = np.zeros((128, 16))
+    P[0, 0] = P[1, 0] = 1.0
+    P[0, 1] = P[1, 1] = P[2, 1] = 1.0
+    y = O.project(x, P)
+    assert y[0, 0] == 1.0 and y[0, 1] == 1.0 + 2.0 ** -7
+    assert O.project(x, P, round_to_bf16=False)[0, 1] == 1.0 + 2.0 ** -8 + 2.0 ** -30
+
+
+# ---------------------------------------------------------------------------
+# Selection: hand-worked golden examples
+# ---------------------------------------------------------------------------
+def test_golden_block_selection():
+    g = json.load(open(os.path.join(GOLDEN, "block_select_hand.json")))
+    qt, kt = np.array(g["qt"], float), np.array(g["kt"], float)
+    b = g["block"]
+    sel, scores = O.select_prefill(qt, kt, g["topk"], block=b)
+    for i in range(len(qt) // b):
+        assert list(scores[i]) == g["scores"][str(i)]
+        assert list(sel[i]) == g["selected"][str(i)]
+        att = O.attended_blocks(sel[i], i, g["window_blocks"], g["sink_blocks"])
+        assert list(att) == g["attended"][str(i)]
+
+
+def test_golden_decode_selection():
+    g = json.load(open(os.path.join(GOLDEN, "decode_select_hand.json")))
+    qt, kt = np.array(g["qt"], float), np.array(g["kt"], float)
+    assert list(O.decode_scores(qt, kt)) == g["scores"]
+    sel = O.select_decode(qt, kt, g["topk"])
+    assert list(sel) == g["selected"]
+    assert list(O.decode_attended(sel, len(kt), g["window"], g["sink"])) == g["attended"]
+
+
+# ---------------------------------------------------------------------------
+# Selection: brute force and the r = D reduction
+# ---------------------------------------------------------------------------
+def _clustered(n, D, centres, rs):
+    c = rs.standard_normal((centres, D))
+    c = 3 * c / np.linalg.norm(c, axis=1, keepdims=True)
+    return O.bf16_round(c[rs.integers(0, centres, n)] + rs.standard_normal((n, D)))
+
+
+@pytest.mark.parametrize("N,block,topk", [(64, 8, 3), (96, 16, 2), (128, 32, 1)])
+def test_block_scores_brute_force(N, block, topk):
+    rs = np.random.default_rng(N)
+    qt = O.bf16_round(rs.standard_normal((N, 4)))
+    kt = O.bf16_round(rs.standard_normal((N, 4)))
+    bs = brute.block_scores_bf(qt.tolist(), kt.tolist(), block)
+    sel, scores = O.select_prefill(qt, kt, topk, block=block)
+    for i in range(N // block):
+        for j in range(i + 1):
+            assert scores[i][j] == pytest.approx(bs[(i, j)], abs=1e-12)
+        assert list(sel[i]) == brute.topk_bf({j: bs[(i, j)] for j in range(i + 1)}, topk)
+
+
+def test_selection_with_identity_projector_is_exact_qk_topk():
+    """r = D, P = I: the projected score is the exact q.k, so the selection is
+    the top-k of the exact max-over-pairs q.k, found here by brute force."""
+    rs = np.random.default_rng(7)
+    N, D, block, topk = 256, 128, 64, 2
+    q = _clustered(N, D, 8, rs)
+    k = _clustered(N, D, 8, rs)
+    P = np.eye(D)
+    qt, kt = O.project(q, P), O.project(k, P)
+    np.testing.assert_array_equal(qt, q)
+    sel, _ = O.select_prefill(qt, kt, topk, block=block)
+    bs = brute.block_scores_bf(q.tolist(), k.tolist(), block)
+    for i in range(N // block):
+        assert list(sel[i]) == brute.topk_bf({j: bs[(i, j)] for j in range(i + 1)}, topk)
+
+
+def test_topk_ties_and_short_lists():
+    s = np.array([1.0, 3.0, 3.0, 2.0, 3.0])
+    assert list(O.topk_desc(s, 2)) == [1, 2]
+    assert list(O.topk_desc(s, 4)) == [1, 2, 3, 4]
+    assert list(O.topk_desc(s, 5)) == [0, 1, 2, 3, 4]
+    assert list(O.topk_desc(s, 9)) == [0, 1, 2, 3, 4]
+    rs = np.random.default_rng(3)
+    for _ in range(50):
+        s = rs.integers(0, 6, 40).astype(float)   # many ties
+        k = int(rs.integers(1, 40))
+        assert list(O.topk_desc(s, k)) == brute.topk_bf(dict(enumerate(s)), k)
+
+
+def test_prefill_selection_invariants():
+    rs = np.random.default_rng(11)
+    N, block, topk = 1024, 64, 4
+    qt = O.bf16_round(rs.standard_normal((N, 16)))
+    kt = O.bf16_round(rs.standard_normal((N, 16)))
+    sel, _ = O.select_prefill(qt, kt, topk, block=block)
+    for i, s in sel.items():
+        assert len(s) == min(topk, i + 1)
+        assert np.all(np.diff(s) > 0) and s.min() >= 0 and s.max() <= i
+        att = O.attended_blocks(s, i, 3, 1)
+        assert 0 in att and i in att and max(0, i - 2) in att
+        assert np.all(np.diff(att) > 0)
+
+
+# ---------------------------------------------------------------------------
+# Attention: library-routine reductions, closed forms, invariants
+# ---------------------------------------------------------------------------
+def test_attend_two_keys_closed_form():
+    q = np.array([[1.0, 0.0]])
+    k = np.array([[0.0, 0.0], [math.log(3.0), 5.0]])
+    v = np.array([[4.0, -8.0], [0.0, 8.0]])
+    o = O.attend(q, [1], k, v, [0, 1], 1.0)
+    np.testing.assert_allclose(o[0], [1.0, 4.0], rtol=0, atol=1e-14)   # weights 1/4, 3/4
+
+
+def test_sparse_prefill_with_all_blocks_is_dense_causal():
+    """k >= number of blocks: every query attends every earlier key, i.e.
+    dense causal attention (torch float64 SDPA, is_causal)."""
+    rs = np.random.default_rng(5)
+    N, D, block = 320, 128, 64
+    q, k, v = _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs)
+    scale = 1 / math.sqrt(D)
+    qt = O.bf16_round(rs.standard_normal((N, 16)))
+    kt = O.bf16_round(rs.standard_normal((N, 16)))
+    sel, _ = O.select_prefill(qt, kt, N // block, block=block)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, None], torch.from_numpy(k)[None, None],
+        torch.from_numpy(v)[None, None], is_causal=True, scale=scale)[0, 0].numpy()
+    for i in range(N // block):
+        att = O.attended_blocks(sel[i], i, 1, 1)
+        assert list(att) == list(range(i + 1))
+        o = O.sparse_attn_prefill_block(q, k, v, i, att, scale, block)
+        np.testing.assert_allclose(o, ref[i * block:(i + 1) * block], rtol=0, atol=1e-12)
+
+
+def test_sparse_prefill_matches_masked_sdpa():
+    """General sparse sets: the same attention as torch SDPA given the mask
+    'key block in the attended set and u <= t'."""
+    rs = np.random.default_rng(6)
+    N, D, block = 512, 64, 64
+    q, k, v = _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs)
+    scale = 0.125
+    for i, att in [(7, [0, 2, 5, 6, 7]), (3, [0, 3]), (5, [1, 4, 5])]:
+        rows = np.arange(i * block, (i + 1) * block)
+        mask = np.zeros((block, N), bool)
+        for j in att:
+            mask[:, j * block:(j + 1) * block] = True
+        mask &= np.arange(N)[None, :] <= rows[:, None]
+        ref = _sdpa_masked(q[rows], k, v, mask, scale)
+        o = O.sparse_attn_prefill_block(q, k, v, i, np.array(att), scale, block)
+        np.testing.assert_allclose(o, ref, rtol=0, atol=1e-12)
+
+
+def test_swa_wide_window_is_full_causal():
+    rs = np.random.default_rng(8)
+    N, D = 200, 128
+    q, k, v = _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs)
+    scale = 1 / math.sqrt(D)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, None], torch.from_numpy(k)[None, None],
+        torch.from_numpy(v)[None, None], is_causal=True, scale=scale)[0, 0].numpy()
+    for W in (N, N + 77):
+        np.testing.assert_allclose(O.swa_rows(q, k, v, np.arange(N), W, scale), ref,
+                                   rtol=0, atol=1e-12)
+
+
+def test_swa_window_one_returns_own_value():
+    rs = np.random.default_rng(9)
+    q, k, v = _bf16_arr((50, 32), 1, rs), _bf16_arr((50, 32), 1, rs), _bf16_arr((50, 32), 1, rs)
+    np.testing.assert_array_equal(O.swa_rows(q, k, v, np.arange(50), 1, 0.3), v)
+
+
+@pytest.mark.parametrize("W", [2, 17, 64])
+def test_swa_matches_band_masked_sdpa(W):
+    rs = np.random.default_rng(W)
+    N, D = 150, 64
+    q, k, v = _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs)
+    t = np.arange(N)
+    mask = (t[None, :] <= t[:, None]) & (t[None, :] > t[:, None] - W)
+    ref = _sdpa_masked(q, k, v, mask, 0.2)
+    np.testing.assert_allclose(O.swa_rows(q, k, v, t, W, 0.2), ref, rtol=0, atol=1e-12)
+
+
+def test_swa_decode_position_offset():
+    """A single query at position L-1 over an L-key cache: last W keys."""
+    rs = np.random.default_rng(10)
+    L, D, W = 300, 64, 40
+    q, k, v = _bf16_arr((1, D), 1, rs), _bf16_arr((L, D), 1, rs), _bf16_arr((L, D), 1, rs)
+    mask = np.zeros((1, L), bool)
+    mask[0, L - W:] = True
+    ref = _sdpa_masked(q, k, v, mask, 0.1)
+    np.testing.assert_allclose(O.swa_rows(q, k, v, [0], W, 0.1, q_pos0=L - 1), ref,
+                               rtol=0, atol=1e-12)
+
+
+def test_attention_invariants_hull_and_permutation():
+    rs = np.random.default_rng(12)
+    D = 128
+    q = _bf16_arr((4, D), 1, rs)
+    k, v = _bf16_arr((90, D), 1, rs), _bf16_arr((90, D), 1, rs)
+    pos = np.arange(90)
+    o = O.attend(q, [89] * 4, k, v, pos, 0.09)
+    assert np.all(o <= v.max(axis=0) + 1e-12) and np.all(o >= v.min(axis=0) - 1e-12)
+    perm = rs.permutation(90)
+    o2 = O.attend(q, [89] * 4, k[perm], v[perm], pos[perm], 0.09)
+    np.testing.assert_allclose(o, o2, rtol=0, atol=1e-13)
+
+
+def test_decode_all_tokens_is_dense_attention():
+    rs = np.random.default_rng(13)
+    L, D = 500, 128
+    q, kc, vc = _bf16_arr((D,), 1, rs), _bf16_arr((L, D), 1, rs), _bf16_arr((L, D), 1, rs)
+    qt, kt = rs.standard_normal(16), O.bf16_round(rs.standard_normal((L, 16)))
+    sel = O.select_decode(qt, kt, L)
+    att = O.decode_attended(sel, L, 8, 1)
+    assert list(att) == list(range(L))
+    o = O.attend_decode(q, kc, vc, att, 1 / math.sqrt(D))
+    ref = _sdpa_masked(q[None], kc, vc, np.ones((1, L), bool), 1 / math.sqrt(D))[0]
+    np.testing.assert_allclose(o, ref, rtol=0, atol=1e-12)
+
+
+def test_decode_identity_projector_selects_needles():
+    """With P = I the decode score is the exact q.k; keys planted as 8*unit(q)
+    (score 8|q|, far above the clustered background's q.k) are all selected."""
+    rs = np.random.default_rng(14)
+    L, D, n_needle = 4096, 128, 32
+    kc = _clustered(L, D, 64, rs)
+    q = _clustered(1, D, 64, rs)[0]
+    pos = np.sort(rs.choice(L, n_needle, replace=False))
+    kc[pos] = O.bf16_round(8 * q / np.linalg.norm(q))
+    sel = O.select_decode(O.project(q, np.eye(D), round_to_bf16=False), O.project(kc, np.eye(D)),
+                          n_needle)
+    assert list(sel) == list(pos)
+
+
+def test_decode_brute_force_pipeline():
+    rs = np.random.default_rng(15)
+    L, D, Hkv, Hq = 96, 16, 2, 4
+    kc = _bf16_arr((L, Hkv, D), 1, rs)
+    vc = _bf16_arr((L, Hkv, D), 1, rs)
+    q = _bf16_arr((Hq, D), 1, rs)
+    P = _bf16_arr((Hkv, D, 4), 0.25, rs)
+    res = O.decode_layer(q, kc, vc, P, ret_heads=[1, 2], window=10, ret_window=7, topk=5,
+                         scale=0.25, sink=1)
+    for h in range(Hq):
+        g = h // 2
+        if h in (1, 2):
+            qt = (q[h] @ P[g]).tolist()
+            kt = O.bf16_round(kc[:, g, :] @ P[g]).tolist()
+            sel, o = brute.decode_bf(q[h].tolist(), kc[:, g].tolist(), vc[:, g].tolist(), qt, kt,
+                                     5, 7, 1, 0.25)
+            assert list(res["sel"][h]) == sel
+        else:
+            o = brute.swa_bf([q[h].tolist()] * L, kc[:, g].tolist(), vc[:, g].tolist(), 10,
+                             0.25)[L - 1]
+        np.testing.assert_allclose(res["out"][h], o, rtol=0, atol=1e-12)
+
+
+def test_prefill_brute_force_pipeline():
+    """N = 256 prefill layer, every head, against the pure-Python definition."""
+    rs = np.random.default_rng(16)
+    N, D, Hq, Hkv, block = 256, 32, 4, 2, 64
+    q = _bf16_arr((N, Hq, D), 1, rs)
+    k = _bf16_arr((N, Hkv, D), 1, rs)
+    v = _bf16_arr((N, Hkv, D), 1, rs)
+    P = _bf16_arr((Hkv, D, 4), 0.3, rs)
+    res = O.prefill_layer(q, k, v, P, ret_heads=[0, 3], window=70, ret_window=64, topk=1,
+                          scale=0.2)
+    for h in range(Hq):
+        g = h // 2
+        if h in (0, 3):
+            qt = O.bf16_round(q[:, h] @ P[g]).tolist()
+            kt = O.bf16_round(k[:, g] @ P[g]).tolist()
+            sel, out = brute.prefill_head_bf(q[:, h].tolist(), k[:, g].tolist(), v[:, g].tolist(),
+                                             qt, kt, 1, 1, 1, block, 0.2)
+            for i in range(N // block):
+                assert list(res["sel"][(h, i)]) == sel[i]
+        else:
+            out = brute.swa_bf(q[:, h].tolist(), k[:, g].tolist(), v[:, g].tolist(), 70, 0.2)
+        for i in range(N // block):
+            np.testing.assert_allclose(res["out"][(h, i)], np.array(out[i * block:(i + 1) * block]),
+                                       rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Planted mistakes: each mutant of an oracle step must fail a pin above.
+# ---------------------------------------------------------------------------
+def _golden_selection_ok(block_scores_fn, topk_fn):
+    g = json.load(open(os.path.join(GOLDEN, "block_select_hand.json")))
+    qt, kt = np.array(g["qt"], float), np.array(g["kt"], float)
+    for i in range(4):
+        s = block_scores_fn(qt, kt, i, g["block"])
+        if list(topk_fn(s, g["topk"])) != g["selected"][str(i)]:
+            return False
+    return True
+
+
+def test_planted_mistakes_are_caught():
+    assert _golden_selection_ok(O.block_scores, O.topk_desc)
+
+    def non_causal_scores(qt, kt, i, block):       # diagonal block scored on every pair
+        qb = qt[i * block:(i + 1) * block]
+        s = qb @ kt[:(i + 1) * block].T
+        return s.reshape(block, i + 1, block).max(axis=(0, 2))
+
+    def ties_to_larger(scores, k):                  # reversed tie-break
+        n = len(scores)
+        if n <= k:
+            return np.arange(n)
+        order = np.lexsort((-np.arange(n), -np.asarray(scores)))
+        return np.sort(order[:k])
+
+    def sum_instead_of_max(qt, kt, i, block):       # block score as a mean, not a max
+        s = O.block_scores(qt, kt, i, block)
+        qb = qt[i * block:(i + 1) * block]
+        return np.array([(qb @ kt[j * block:(j + 1) * block].T).mean() for j in range(i + 1)])
+
+    assert not _golden_selection_ok(non_causal_scores, O.topk_desc)
+    assert not _golden_selection_ok(O.block_scores, ties_to_larger)
+    assert not _golden_selection_ok(sum_instead_of_max, O.topk_desc)
+
+    # SWA with the window off by one must fail the band-mask library check.
+    rs = np.random.default_rng(21)
+    N, D, W = 80, 32, 9
+    q, k, v = _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs)
+    t = np.arange(N)
+    mask = (t[None, :] <= t[:, None]) & (t[None, :] > t[:, None] - W)
+    ref = _sdpa_masked(q, k, v, mask, 0.2)
+    assert np.abs(O.swa_rows(q, k, v, t, W + 1, 0.2) - ref).max() > 1e-3
+
+    # Attention with a wrong scale must fail the two-key closed form.
+    qq = np.array([[1.0, 0.0]])
+    kk = np.array([[0.0, 0.0], [math.log(3.0), 5.0]])
+    vv = np.array([[4.0, -8.0], [0.0, 8.0]])
+    assert np.abs(O.attend(qq, [1], kk, vv, [0, 1], 0.5)[0] - [1.0, 4.0]).max() > 0.1
+
+    # Window blocks counted from the wrong end must fail the golden attended sets.
+    g = json.load(open(os.path.join(GOLDEN, "block_select_hand.json")))
+    wrong = np.unique(np.concatenate([np.array(g["selected"]["3"]), [0], np.arange(0, 1)]))
+    assert list(wrong) != g["attended"]["3"]

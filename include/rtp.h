@@ -1,0 +1,227 @@
+/*
+ * rtp.h - C ABI of the head-wise hybrid attention library (librtp.so).
+ *
+ * The method (RTPurbo / RTPurboV2): most attention heads of a long-context
+ * model are "streaming" heads that only need a local window and run causal
+ * sliding-window attention (SWA, window 8192 in the deployed recipe); about
+ * 15% are "retrieval" heads. For those, a cheap 16-dimensional indexer built
+ * from a per-KV-head low-rank projector P (D x 16) scores key blocks (prefill)
+ * or tokens (decode); the top-k are selected, and exact softmax attention is
+ * computed at the full head dimension over the sink, the local window and the
+ * selected keys.
+ *   Sources: RTPurboV2 article (th-motor.com), paragraphs on retrieval vs
+ *   streaming heads, on the low-rank projector (D -> r = 16) and on the
+ *   Qwen3-Coder-30B-A3B recipe (SWA window 8192); RTPurbo digest (Telegram
+ *   channel "Data analysis", post 5185): the 16-d indexer is a scout that
+ *   picks candidates, then honest attention runs at full dimension on them.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every call returns an rtp_status; nothing else crosses the ABI (no C++
+ *    exceptions). Arguments are validated on the host before any launch; a
+ *    rejected call launches nothing and leaves every output untouched.
+ *  - Device pointers: all tensor arguments are caller-owned device memory
+ *    (global memory of the current CUDA device). The library keeps no
+ *    pointer after a call returns and allocates no device memory itself:
+ *    scratch space is the caller's `ws` buffer, whose minimum size the
+ *    matching rtp_workspace_size_* call returns. `ws` must be 256-byte
+ *    aligned. Arguments documented as "host" are read during the call only.
+ *  - Asynchrony: work is enqueued on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream); results are ready when the stream reaches that
+ *    point. Launch failures return RTP_ERR_CUDA.
+ *  - bf16 tensors are IEEE bfloat16 (uint16 storage); rounding to bf16 is
+ *    round-to-nearest-even everywhere.
+ *  - Layouts: activations are [B, N, H, D] with element strides given by an
+ *    rtp_strides {b, n, h}; the last dimension (D) is contiguous. Every
+ *    stride must be a multiple of 8 elements and every base pointer 16-byte
+ *    aligned (tensor-memory-access tiles need 16-byte-aligned rows).
+ *  - Head mapping: query head h reads KV head h / (Hq / Hkv) (contiguous
+ *    grouped-query attention); Hq must be a multiple of Hkv.
+ *  - Sizes: D = 128 and block = 64 in this build; N (prefill) must be a
+ *    multiple of 64. Other values return RTP_ERR_UNSUPPORTED.
+ *  - Thread safety: calls are reentrant; concurrent calls on different
+ *    streams must use different workspaces.
+ */
+#ifndef RTP_H_
+#define RTP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RTP_VERSION 1
+
+#if defined(__GNUC__)
+#define RTP_API __attribute__((visibility("default")))
+#else
+#define RTP_API
+#endif
+
+typedef enum {
+  RTP_OK = 0,
+  RTP_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or index */
+  RTP_ERR_UNSUPPORTED = 2,   /* shape outside what this build implements, or no sm_100 device */
+  RTP_ERR_CUDA = 3,          /* a CUDA launch or runtime call failed */
+  RTP_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up */
+  RTP_ERR_WORKSPACE = 5      /* ws too small or misaligned */
+} rtp_status;
+
+typedef enum { RTP_BF16 = 0, RTP_F32 = 1 } rtp_dtype;
+
+/* Element strides of a [B, N, H, D] tensor (D contiguous). */
+typedef struct { int64_t b, n, h; } rtp_strides;
+
+struct CUstream_st;
+typedef struct CUstream_st* rtp_stream_t; /* same type as cudaStream_t */
+
+/* Human-readable name of a status (static storage, never NULL). */
+RTP_API const char* rtp_status_string(rtp_status s);
+/* RTP_VERSION of the loaded library. */
+RTP_API int rtp_version(void);
+
+/*
+ * rtp_index_project - the low-rank indexer projection x~ = x . P.
+ *   Source: RTPurboV2 article, paragraph on the low-rank projector (feature
+ *   dimension compressed from D to r = 16); the precomputed 16-d key index
+ *   of the 128K decode workload.
+ *
+ *   x        bf16 [B, N, Hx, D] device, strides xs.
+ *   P        bf16 [Hp, D, r] device, contiguous; one projector per KV head.
+ *   heads    host int32 [n_heads]: which heads of x to project (0 <= . < Hx).
+ *   proj_of  host int32 [n_heads]: which projector each listed head uses
+ *            (0 <= . < Hp; for a query head h this is h / (Hq/Hkv)).
+ *   out      device [B, n_heads, N, r], contiguous; out_dtype RTP_BF16 (the
+ *            stored index: fp32 accumulation, one RNE rounding) or RTP_F32
+ *            (the decode query index, unrounded fp32 accumulation).
+ *   r must be 16. n_heads >= 1. N >= 1 (no multiple-of-64 rule here).
+ */
+RTP_API rtp_status rtp_index_project(const void* x, rtp_strides xs, int B, int N, int Hx,
+                             const void* P, int Hp, int r,
+                             const int32_t* heads, const int32_t* proj_of, int n_heads,
+                             void* out, rtp_dtype out_dtype, rtp_stream_t stream);
+
+/*
+ * rtp_select_prefill - per query block, the top-k key blocks by block score.
+ *   Source: block score = max over the (query, key) pairs of a 64 x 64
+ *   block pair of q~ . k~, each query block keeping its top-k causal key
+ *   blocks (the tiny 2K prefill workload statement); the indexer as a scout
+ *   (RTPurbo digest). Only causal pairs (key position <= query position) are
+ *   scored; every causal key block j <= i is a candidate; exact ties rank
+ *   the smaller block first. The token score matrix is never materialised.
+ *
+ *   qt       bf16 [B, Hr, N, r] device, contiguous (projected retrieval-head queries).
+ *   kt       bf16 [B, Hkv, N, r] device, contiguous (projected keys).
+ *   kv_of    host int32 [Hr]: KV head of each retrieval head.
+ *   topk     k >= 1 selected blocks per query block.
+ *   blocks   int32 [B, Hr, N/64, topk] device out: ascending block indices,
+ *            min(k, i+1) of them, the rest -1.
+ *   counts   int32 [B, Hr, N/64] device out: min(k, i+1).
+ *   ws       workspace of rtp_workspace_size_select_prefill() bytes.
+ *   N must be a multiple of 64, r = 16.
+ */
+RTP_API size_t rtp_workspace_size_select_prefill(int B, int N, int Hr, int topk);
+RTP_API rtp_status rtp_select_prefill(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
+                              int r, const int32_t* kv_of, int topk,
+                              int32_t* blocks, int32_t* counts,
+                              void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * rtp_select_decode - token-level top-k over the whole cache.
+ *   Source: the 128K decode workload statement (retrieval heads take the
+ *   token-level top-2048 by q~ . k~ over the whole cache); RTPurbo digest.
+ *   Exact ties rank the smaller token first.
+ *
+ *   qt       fp32 [B, Hr, r] device (unrounded projected decode queries).
+ *   kindex   bf16 [B, Hkv, L, r] device, contiguous (the key index).
+ *   kv_of    host int32 [Hr].
+ *   idx      int32 [B, Hr, topk] device out: ascending token indices;
+ *            min(k, L) of them, the rest -1.
+ *   ws       workspace of rtp_workspace_size_select_decode() bytes.
+ *   r = 16, 1 <= topk <= 4096, L >= 1.
+ */
+RTP_API size_t rtp_workspace_size_select_decode(int B, int L, int Hr, int topk);
+RTP_API rtp_status rtp_select_decode(const float* qt, const void* kindex, int B, int L, int Hr, int Hkv,
+                             int r, const int32_t* kv_of, int topk, int32_t* idx,
+                             void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * rtp_sparse_attn_prefill - exact attention of retrieval heads over their
+ * selected key blocks, the sink blocks and the local window blocks.
+ *   Source: RTPurbo digest (honest attention at full dimension over the
+ *   small selected set); the tiny 2K prefill workload statement (top-k
+ *   blocks plus key block 0 plus the window blocks).
+ *   For query block i the attended key blocks are the set
+ *     blocks[i][0..count) U {0 .. sink_blocks-1} U {i-window_blocks+1 .. i},
+ *   each key once, with the causal mask (key position <= query position).
+ *
+ *   q, o     bf16 [B, N, Hq, D] device (strides qs, os); o is written only for
+ *            the listed heads.
+ *   k, v     bf16 [B, N, Hkv, D] device (strides ks, vs).
+ *   heads    host int32 [Hr]: the retrieval heads; row j of blocks/counts
+ *            belongs to heads[j].
+ *   blocks   int32 [B, Hr, N/64, topk], counts int32 [B, Hr, N/64] device, as
+ *            written by rtp_select_prefill (ascending; entries outside
+ *            [0, i] are ignored).
+ *   window_blocks >= 1, sink_blocks >= 0, scale > 0 (the softmax scale,
+ *   1/sqrt(D) in the method's usual form).
+ */
+RTP_API size_t rtp_workspace_size_sparse_attn_prefill(int B, int N, int Hr, int topk);
+RTP_API rtp_status rtp_sparse_attn_prefill(const void* q, rtp_strides qs, const void* k, rtp_strides ks,
+                                   const void* v, rtp_strides vs, void* o, rtp_strides os,
+                                   int B, int N, int Hq, int Hkv, const int32_t* heads, int Hr,
+                                   const int32_t* blocks, const int32_t* counts, int topk,
+                                   int window_blocks, int sink_blocks, float scale,
+                                   void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * rtp_sparse_attn_decode - one new query token per sequence attends, per
+ * retrieval head, the selected tokens, tokens 0..sink-1 and the last
+ * `window` tokens of the cache, each key once.
+ *   Source: the 128K decode workload statement (top-2048 unioned with the
+ *   last 8192 tokens and token 0, then exact softmax attention at D=128);
+ *   RTPurbo digest.
+ *
+ *   q        bf16 [B, Hq, D] device, contiguous; o likewise (written only for
+ *            the listed heads).
+ *   kc, vc   bf16 [B, L, Hkv, D] device (strides ks, vs): the cache, whose
+ *            last row (L-1) is the new token's own key/value.
+ *   heads    host int32 [Hr]; idx int32 [B, Hr, topk] device: distinct
+ *            token indices, -1 padded, as written by rtp_select_decode
+ *            (entries in the window or below `sink` are skipped there,
+ *            since those keys are attended anyway).
+ *   window >= 1, sink >= 0, scale > 0.
+ */
+RTP_API size_t rtp_workspace_size_sparse_attn_decode(int B, int L, int Hq, int Hr, int topk, int window);
+RTP_API rtp_status rtp_sparse_attn_decode(const void* q, const void* kc, rtp_strides ks,
+                                  const void* vc, rtp_strides vs, void* o,
+                                  int B, int L, int Hq, int Hkv, const int32_t* heads, int Hr,
+                                  const int32_t* idx, int topk, int window, int sink, float scale,
+                                  void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * rtp_swa - causal sliding-window attention of streaming heads.
+ *   Source: RTPurboV2 article (streaming heads use SWA, local window 8192).
+ *   Query row t sits at position q_pos0 + t and attends the keys u with
+ *   position - window < u <= position (u < Nk). Prefill: Nq = Nk = N,
+ *   q_pos0 = 0. Decode: Nq = 1, Nk = L, q_pos0 = L - 1.
+ *
+ *   q, o     bf16 [B, Nq, Hq, D] device (strides qs, os); o written only for
+ *            the listed heads.
+ *   k, v     bf16 [B, Nk, Hkv, D] device (strides ks, vs).
+ *   heads    host int32 [n_heads]: the streaming heads to compute.
+ *   window >= 1, scale > 0. Prefill (Nq > 1) needs Nq % 64 == 0.
+ */
+RTP_API size_t rtp_workspace_size_swa(int B, int Nq, int Nk, int n_heads, int window);
+RTP_API rtp_status rtp_swa(const void* q, rtp_strides qs, const void* k, rtp_strides ks,
+                   const void* v, rtp_strides vs, void* o, rtp_strides os,
+                   int B, int Nq, int Nk, int q_pos0, int Hq, int Hkv,
+                   const int32_t* heads, int n_heads, int window, float scale,
+                   void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RTP_H_ */

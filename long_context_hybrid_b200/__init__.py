@@ -1,0 +1,295 @@
+"""Python binding of librtp.so, the head-wise hybrid attention library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI (``include/rtp.h``). Tensors are torch CUDA tensors
+(PyTorch provides device memory and streams); each function passes raw
+pointers, element strides and the current stream to the matching C call and
+raises ``RtpError`` on any status other than RTP_OK. There is no fallback: if
+the library is missing, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librtp.so")
+
+RTP_OK, RTP_BF16, RTP_F32 = 0, 0, 1
+D_HEAD, R_INDEX, BLOCK = 128, 16, 64
+
+
+class RtpError(RuntimeError):
+    pass
+
+
+class Strides(ctypes.Structure):
+    _fields_ = [("b", ctypes.c_int64), ("n", ctypes.c_int64), ("h", ctypes.c_int64)]
+
+
+_lib = None
+_c_i32p = ctypes.POINTER(ctypes.c_int32)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+_SIGNATURES = {
+    "rtp_status_string": (ctypes.c_char_p, [_I]),
+    "rtp_version": (_I, []),
+    "rtp_index_project": (_I, [_P, Strides, _I, _I, _I, _P, _I, _I, _c_i32p, _c_i32p, _I, _P, _I, _P]),
+    "rtp_workspace_size_select_prefill": (_SZ, [_I, _I, _I, _I]),
+    "rtp_select_prefill": (_I, [_P, _P, _I, _I, _I, _I, _I, _c_i32p, _I, _P, _P, _P, _SZ, _P]),
+    "rtp_workspace_size_select_decode": (_SZ, [_I, _I, _I, _I]),
+    "rtp_select_decode": (_I, [_P, _P, _I, _I, _I, _I, _I, _c_i32p, _I, _P, _P, _SZ, _P]),
+    "rtp_workspace_size_sparse_attn_prefill": (_SZ, [_I, _I, _I, _I]),
+    "rtp_sparse_attn_prefill": (_I, [_P, Strides, _P, Strides, _P, Strides, _P, Strides, _I, _I, _I,
+                                     _I, _c_i32p, _I, _P, _P, _I, _I, _I, _F, _P, _SZ, _P]),
+    "rtp_workspace_size_sparse_attn_decode": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "rtp_sparse_attn_decode": (_I, [_P, _P, Strides, _P, Strides, _P, _I, _I, _I, _I, _c_i32p, _I,
+                                    _P, _I, _I, _I, _F, _P, _SZ, _P]),
+    "rtp_workspace_size_swa": (_SZ, [_I, _I, _I, _I, _I]),
+    "rtp_swa": (_I, [_P, Strides, _P, Strides, _P, Strides, _P, Strides, _I, _I, _I, _I, _I, _I,
+                     _c_i32p, _I, _I, _F, _P, _SZ, _P]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded librtp.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RtpError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m long_context_hybrid_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != RTP_OK:
+        raise RtpError(f"{what}: {lib().rtp_status_string(status).decode()}")
+
+
+def _i32(values: Sequence[int]):
+    arr = (ctypes.c_int32 * len(values))(*[int(v) for v in values])
+    return arr
+
+
+def _strides4(t: torch.Tensor) -> Strides:
+    assert t.dim() == 4 and t.stride(3) == 1, "expected [B, N, H, D] with contiguous D"
+    return Strides(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ws(nbytes: int, device, ws: Optional[torch.Tensor]):
+    if nbytes == 0:
+        return None, 0
+    if ws is not None and ws.numel() * ws.element_size() >= nbytes:
+        return ws.data_ptr(), ws.numel() * ws.element_size()
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return buf, nbytes
+
+
+def _wsptr(buf):
+    if buf is None:
+        return None
+    return buf if isinstance(buf, int) else buf.data_ptr()
+
+
+def kv_of(h: int, Hq: int, Hkv: int) -> int:
+    return h // (Hq // Hkv)
+
+
+# ---------------------------------------------------------------------------
+# The six calls
+# ---------------------------------------------------------------------------
+def index_project(x: torch.Tensor, P: torch.Tensor, heads: Sequence[int], proj_of: Sequence[int],
+                  out_dtype=torch.bfloat16, out: Optional[torch.Tensor] = None, stream=None):
+    """x [B,N,Hx,D] bf16, P [Hp,D,r] bf16 -> out [B, len(heads), N, r]."""
+    B, N, Hx, _ = x.shape
+    Hp, _, r = P.shape
+    if out is None:
+        out = torch.empty(B, len(heads), N, r, dtype=out_dtype, device=x.device)
+    dt = RTP_F32 if out.dtype == torch.float32 else RTP_BF16
+    _check(lib().rtp_index_project(x.data_ptr(), _strides4(x), B, N, Hx, P.data_ptr(), Hp, r,
+                                   _i32(heads), _i32(proj_of), len(heads), out.data_ptr(), dt,
+                                   _stream(stream)), "rtp_index_project")
+    return out
+
+
+def select_prefill(qt: torch.Tensor, kt: torch.Tensor, kv_of_ret: Sequence[int], topk: int,
+                   blocks: Optional[torch.Tensor] = None, counts: Optional[torch.Tensor] = None,
+                   ws: Optional[torch.Tensor] = None, stream=None):
+    """qt [B,Hr,N,r], kt [B,Hkv,N,r] bf16 -> (blocks [B,Hr,N/64,k], counts [B,Hr,N/64])."""
+    B, Hr, N, r = qt.shape
+    Hkv = kt.shape[1]
+    nb = N // BLOCK
+    if blocks is None:
+        blocks = torch.empty(B, Hr, nb, topk, dtype=torch.int32, device=qt.device)
+    if counts is None:
+        counts = torch.empty(B, Hr, nb, dtype=torch.int32, device=qt.device)
+    need = lib().rtp_workspace_size_select_prefill(B, N, Hr, topk)
+    buf, nbytes = _ws(need, qt.device, ws)
+    _check(lib().rtp_select_prefill(qt.data_ptr(), kt.data_ptr(), B, N, Hr, Hkv, r, _i32(kv_of_ret),
+                                    topk, blocks.data_ptr(), counts.data_ptr(), _wsptr(buf), nbytes,
+                                    _stream(stream)), "rtp_select_prefill")
+    return blocks, counts
+
+
+def select_decode(qt: torch.Tensor, kindex: torch.Tensor, kv_of_ret: Sequence[int], topk: int,
+                  idx: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """qt [B,Hr,r] fp32, kindex [B,Hkv,L,r] bf16 -> idx [B,Hr,k] int32 ascending."""
+    B, Hr, r = qt.shape
+    Hkv, L = kindex.shape[1], kindex.shape[2]
+    if idx is None:
+        idx = torch.empty(B, Hr, topk, dtype=torch.int32, device=qt.device)
+    need = lib().rtp_workspace_size_select_decode(B, L, Hr, topk)
+    buf, nbytes = _ws(need, qt.device, ws)
+    _check(lib().rtp_select_decode(qt.data_ptr(), kindex.data_ptr(), B, L, Hr, Hkv, r,
+                                   _i32(kv_of_ret), topk, idx.data_ptr(), _wsptr(buf), nbytes,
+                                   _stream(stream)), "rtp_select_decode")
+    return idx
+
+
+def sparse_attn_prefill(q, k, v, o, heads: Sequence[int], blocks, counts, window_blocks: int,
+                        sink_blocks: int = 1, scale: Optional[float] = None,
+                        ws: Optional[torch.Tensor] = None, stream=None):
+    """Retrieval-head prefill attention; writes o[:, :, heads, :]."""
+    B, N, Hq, D = q.shape
+    Hkv = k.shape[2]
+    topk = blocks.shape[-1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    need = lib().rtp_workspace_size_sparse_attn_prefill(B, N, len(heads), topk)
+    buf, nbytes = _ws(need, q.device, ws)
+    _check(lib().rtp_sparse_attn_prefill(q.data_ptr(), _strides4(q), k.data_ptr(), _strides4(k),
+                                         v.data_ptr(), _strides4(v), o.data_ptr(), _strides4(o),
+                                         B, N, Hq, Hkv, _i32(heads), len(heads), blocks.data_ptr(),
+                                         counts.data_ptr(), topk, window_blocks, sink_blocks, scale,
+                                         _wsptr(buf), nbytes, _stream(stream)),
+           "rtp_sparse_attn_prefill")
+    return o
+
+
+def sparse_attn_decode(q, kc, vc, o, heads: Sequence[int], idx, window: int, sink: int = 1,
+                       scale: Optional[float] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """Retrieval-head decode attention. q/o [B,Hq,D], kc/vc [B,L,Hkv,D]."""
+    B, Hq, D = q.shape
+    L, Hkv = kc.shape[1], kc.shape[2]
+    topk = idx.shape[-1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    need = lib().rtp_workspace_size_sparse_attn_decode(B, L, Hq, len(heads), topk, window)
+    buf, nbytes = _ws(need, q.device, ws)
+    _check(lib().rtp_sparse_attn_decode(q.data_ptr(), kc.data_ptr(), _strides4(kc), vc.data_ptr(),
+                                        _strides4(vc), o.data_ptr(), B, L, Hq, Hkv, _i32(heads),
+                                        len(heads), idx.data_ptr(), topk, window, sink, scale,
+                                        _wsptr(buf), nbytes, _stream(stream)),
+           "rtp_sparse_attn_decode")
+    return o
+
+
+def swa(q, k, v, o, heads: Sequence[int], window: int, q_pos0: int = 0,
+        scale: Optional[float] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """Streaming-head sliding-window attention. q/o [B,Nq,Hq,D], k/v [B,Nk,Hkv,D]."""
+    B, Nq, Hq, D = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    need = lib().rtp_workspace_size_swa(B, Nq, Nk, len(heads), window)
+    buf, nbytes = _ws(need, q.device, ws)
+    _check(lib().rtp_swa(q.data_ptr(), _strides4(q), k.data_ptr(), _strides4(k), v.data_ptr(),
+                         _strides4(v), o.data_ptr(), _strides4(o), B, Nq, Nk, q_pos0, Hq, Hkv,
+                         _i32(heads), len(heads), window, scale, _wsptr(buf), nbytes,
+                         _stream(stream)), "rtp_swa")
+    return o
+
+
+# ---------------------------------------------------------------------------
+# One layer, composed from the six calls
+# ---------------------------------------------------------------------------
+class PrefillLayer:
+    """One prefill layer: indexer projection, block selection, sparse attention
+    on retrieval heads and SWA on streaming heads, with buffers kept across calls."""
+
+    def __init__(self, B, N, Hq, Hkv, ret_heads, window, ret_window, topk, device,
+                 sink_blocks=1, scale=None):
+        self.B, self.N, self.Hq, self.Hkv = B, N, Hq, Hkv
+        self.ret = list(ret_heads)
+        self.swa_heads = [h for h in range(Hq) if h not in set(self.ret)]
+        self.window, self.topk, self.sink_blocks = window, topk, sink_blocks
+        self.window_blocks = ret_window // BLOCK
+        self.scale = 1.0 / math.sqrt(D_HEAD) if scale is None else scale
+        self.kv_ret = [kv_of(h, Hq, Hkv) for h in self.ret]
+        self.kv_used = sorted(set(self.kv_ret))
+        self.kv_slot = [self.kv_used.index(g) for g in self.kv_ret]
+        nb = N // BLOCK
+        if self.ret:
+            self.kt = torch.empty(B, len(self.kv_used), N, R_INDEX, dtype=torch.bfloat16, device=device)
+            self.qt = torch.empty(B, len(self.ret), N, R_INDEX, dtype=torch.bfloat16, device=device)
+            self.blocks = torch.empty(B, len(self.ret), nb, topk, dtype=torch.int32, device=device)
+            self.counts = torch.empty(B, len(self.ret), nb, dtype=torch.int32, device=device)
+
+    def __call__(self, q, k, v, P, o, stream=None):
+        if self.ret:
+            index_project(k, P, self.kv_used, self.kv_used, out=self.kt, stream=stream)
+            index_project(q, P, self.ret, self.kv_ret, out=self.qt, stream=stream)
+            select_prefill(self.qt, self.kt, self.kv_slot, self.topk, self.blocks, self.counts,
+                           stream=stream)
+            sparse_attn_prefill(q, k, v, o, self.ret, self.blocks, self.counts, self.window_blocks,
+                                self.sink_blocks, self.scale, stream=stream)
+        if self.swa_heads:
+            swa(q, k, v, o, self.swa_heads, self.window, 0, self.scale, stream=stream)
+        return o
+
+
+class DecodeStep:
+    """One decode step over a cache with a precomputed key index: query
+    projection, token selection, sparse attention on retrieval heads and SWA
+    on streaming heads."""
+
+    def __init__(self, B, L, Hq, Hkv, ret_heads, window, ret_window, topk, device, sink=1,
+                 scale=None):
+        self.B, self.L, self.Hq, self.Hkv = B, L, Hq, Hkv
+        self.ret = list(ret_heads)
+        self.swa_heads = [h for h in range(Hq) if h not in set(self.ret)]
+        self.window, self.ret_window, self.topk, self.sink = window, ret_window, topk, sink
+        self.scale = 1.0 / math.sqrt(D_HEAD) if scale is None else scale
+        self.kv_ret = [kv_of(h, Hq, Hkv) for h in self.ret]
+        if self.ret:
+            self.qt = torch.empty(B, len(self.ret), R_INDEX, dtype=torch.float32, device=device)
+            self.idx = torch.empty(B, len(self.ret), topk, dtype=torch.int32, device=device)
+            self.ws_sel = torch.empty(lib().rtp_workspace_size_select_decode(B, L, len(self.ret), topk),
+                                      dtype=torch.uint8, device=device)
+            self.ws_att = torch.empty(lib().rtp_workspace_size_sparse_attn_decode(
+                B, L, Hq, len(self.ret), topk, ret_window), dtype=torch.uint8, device=device)
+        if self.swa_heads:
+            self.ws_swa = torch.empty(lib().rtp_workspace_size_swa(B, 1, L, len(self.swa_heads), window),
+                                      dtype=torch.uint8, device=device)
+
+    def __call__(self, q, kc, vc, kindex, P, o, stream=None):
+        """q/o [B,Hq,D]; kc/vc [B,L,Hkv,D]; kindex [B,Hkv,L,r]."""
+        if self.ret:
+            index_project(q.unsqueeze(1), P, self.ret, self.kv_ret, out=self.qt.view(self.B, len(self.ret), 1, R_INDEX),
+                          stream=stream)
+            select_decode(self.qt, kindex, self.kv_ret, self.topk, self.idx, self.ws_sel, stream=stream)
+            sparse_attn_decode(q, kc, vc, o, self.ret, self.idx, self.ret_window, self.sink,
+                               self.scale, self.ws_att, stream=stream)
+        if self.swa_heads:
+            swa(q.unsqueeze(1), kc, vc, o.unsqueeze(1), self.swa_heads, self.window, self.L - 1,
+                self.scale, self.ws_swa, stream=stream)
+        return o
+
+
+__all__ = ["lib", "RtpError", "index_project", "select_prefill", "select_decode",
+           "sparse_attn_prefill", "sparse_attn_decode", "swa", "PrefillLayer", "DecodeStep",
+           "kv_of", "LIB_PATH"]

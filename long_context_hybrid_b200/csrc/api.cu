@@ -1,0 +1,225 @@
+// C ABI of the head-wise hybrid attention library: argument validation on
+// the host, then dispatch to the kernels. See include/rtp.h for the contract.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/rtp.h"
+#include "attn_prefill_common.cuh"
+#include "rtp_common.cuh"
+#include "rtp_internal.h"
+
+using namespace rtp;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+bool stride_ok(rtp_strides s) { return s.b % 8 == 0 && s.n % 8 == 0 && s.h % 8 == 0 && s.b >= 0 && s.n >= 0 && s.h >= 0; }
+
+rtp_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RTP_OK : RTP_ERR_CUDA; }
+
+// The device must be a Blackwell datacenter part (compute capability 10.x).
+rtp_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RTP_ERR_CUDA;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return RTP_ERR_CUDA;
+  return major == 10 ? RTP_OK : RTP_ERR_UNSUPPORTED;
+}
+
+rtp_status check_heads(const int32_t* heads, int n, int H) {
+  if (!heads || n < 1 || n > kMaxHeads) return RTP_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i)
+    if (heads[i] < 0 || heads[i] >= H) return RTP_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i)
+    for (int k = i + 1; k < n; ++k)
+      if (heads[i] == heads[k]) return RTP_ERR_INVALID_ARG;
+  return RTP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rtp_status_string(rtp_status s) {
+  switch (s) {
+    case RTP_OK: return "RTP_OK";
+    case RTP_ERR_INVALID_ARG: return "RTP_ERR_INVALID_ARG";
+    case RTP_ERR_UNSUPPORTED: return "RTP_ERR_UNSUPPORTED";
+    case RTP_ERR_CUDA: return "RTP_ERR_CUDA";
+    case RTP_ERR_TIMEOUT: return "RTP_ERR_TIMEOUT";
+    case RTP_ERR_WORKSPACE: return "RTP_ERR_WORKSPACE";
+  }
+  return "RTP_ERR_UNKNOWN";
+}
+
+int rtp_version(void) { return RTP_VERSION; }
+
+rtp_status rtp_index_project(const void* x, rtp_strides xs, int B, int N, int Hx,
+                             const void* P, int Hp, int r,
+                             const int32_t* heads, const int32_t* proj_of, int n_heads,
+                             void* out, rtp_dtype out_dtype, rtp_stream_t stream) {
+  if (!x || !P || !out || !proj_of) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || Hx < 1 || Hp < 1) return RTP_ERR_INVALID_ARG;
+  if (r != RTP_R) return RTP_ERR_UNSUPPORTED;
+  if (out_dtype != RTP_BF16 && out_dtype != RTP_F32) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out) || !aligned16(P) || !stride_ok(xs)) return RTP_ERR_INVALID_ARG;
+  rtp_status st = check_heads(heads, n_heads, Hx);
+  if (st != RTP_OK) return st;
+  for (int i = 0; i < n_heads; ++i)
+    if (proj_of[i] < 0 || proj_of[i] >= Hp) return RTP_ERR_INVALID_ARG;
+  if ((st = check_device()) != RTP_OK) return st;
+  return from_cuda(launch_project(x, xs.b, xs.n, xs.h, B, N, P, heads, proj_of, n_heads, out,
+                                  out_dtype == RTP_F32, (cudaStream_t)stream));
+}
+
+size_t rtp_workspace_size_select_prefill(int B, int N, int Hr, int topk) {
+  return select_prefill_ws_bytes(B, N, Hr, topk);
+}
+
+rtp_status rtp_select_prefill(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
+                              int r, const int32_t* kv_of, int topk,
+                              int32_t* blocks, int32_t* counts,
+                              void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  if (!qt || !kt || !blocks || !counts || !kv_of) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || N < RTP_BLOCK || Hr < 1 || Hr > kMaxHeads || Hkv < 1 || topk < 1) return RTP_ERR_INVALID_ARG;
+  if (N % RTP_BLOCK != 0 || r != RTP_R) return RTP_ERR_UNSUPPORTED;
+  if (N / RTP_BLOCK > 32768) return RTP_ERR_UNSUPPORTED;
+  if (!aligned16(qt) || !aligned16(kt) || !aligned16(blocks) || !aligned16(counts)) return RTP_ERR_INVALID_ARG;
+  for (int j = 0; j < Hr; ++j)
+    if (kv_of[j] < 0 || kv_of[j] >= Hkv) return RTP_ERR_INVALID_ARG;
+  const size_t need = select_prefill_ws_bytes(B, N, Hr, topk);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned256(ws))) return RTP_ERR_WORKSPACE;
+  rtp_status st = check_device();
+  if (st != RTP_OK) return st;
+  return from_cuda(launch_select_prefill(qt, kt, B, N, Hr, Hkv, kv_of, topk, blocks, counts, ws,
+                                         (cudaStream_t)stream));
+}
+
+size_t rtp_workspace_size_select_decode(int B, int L, int Hr, int topk) {
+  return select_decode_ws_bytes(B, L, Hr, topk);
+}
+
+rtp_status rtp_select_decode(const float* qt, const void* kindex, int B, int L, int Hr, int Hkv,
+                             int r, const int32_t* kv_of, int topk, int32_t* idx,
+                             void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  if (!qt || !kindex || !idx || !kv_of) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || Hr < 1 || Hr > kMaxHeads || Hkv < 1 || topk < 1) return RTP_ERR_INVALID_ARG;
+  if (r != RTP_R || topk > 4096) return RTP_ERR_UNSUPPORTED;
+  if (!aligned16(qt) || !aligned16(kindex) || !aligned16(idx)) return RTP_ERR_INVALID_ARG;
+  for (int j = 0; j < Hr; ++j)
+    if (kv_of[j] < 0 || kv_of[j] >= Hkv) return RTP_ERR_INVALID_ARG;
+  const size_t need = select_decode_ws_bytes(B, L, Hr, topk);
+  if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
+  rtp_status st = check_device();
+  if (st != RTP_OK) return st;
+  return from_cuda(launch_select_decode(qt, kindex, B, L, Hr, Hkv, kv_of, topk, idx, ws,
+                                        (cudaStream_t)stream));
+}
+
+size_t rtp_workspace_size_sparse_attn_prefill(int B, int N, int Hr, int topk) {
+  (void)B; (void)N; (void)Hr; (void)topk;
+  return 0;
+}
+
+rtp_status rtp_sparse_attn_prefill(const void* q, rtp_strides qs, const void* k, rtp_strides ks,
+                                   const void* v, rtp_strides vs, void* o, rtp_strides os,
+                                   int B, int N, int Hq, int Hkv, const int32_t* heads, int Hr,
+                                   const int32_t* blocks, const int32_t* counts, int topk,
+                                   int window_blocks, int sink_blocks, float scale,
+                                   void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  (void)ws; (void)ws_bytes;
+  if (!q || !k || !v || !o || !blocks || !counts) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || N < RTP_BLOCK || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || topk < 1) return RTP_ERR_INVALID_ARG;
+  if (window_blocks < 1 || sink_blocks < 0 || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
+  if (N % RTP_BLOCK != 0) return RTP_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
+  if (!stride_ok(qs) || !stride_ok(ks) || !stride_ok(vs) || !stride_ok(os)) return RTP_ERR_INVALID_ARG;
+  rtp_status st = check_heads(heads, Hr, Hq);
+  if (st != RTP_OK) return st;
+  if ((st = check_device()) != RTP_OK) return st;
+  PrefillAttnParams p{};
+  p.q = {q, qs.b, qs.n, qs.h}; p.k = {k, ks.b, ks.n, ks.h}; p.v = {v, vs.b, vs.n, vs.h};
+  p.o = o; p.o_sb = os.b; p.o_sn = os.n; p.o_sh = os.h;
+  p.Nq = N; p.Nk = N; p.q_pos0 = 0; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv;
+  p.sparse = 1; p.blocks = blocks; p.counts = counts; p.topk = topk;
+  p.window_tokens = window_blocks * RTP_BLOCK; p.window_blocks = window_blocks;
+  p.sink_blocks = sink_blocks;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_heads = Hr;
+  const int nb = N / RTP_BLOCK;
+  p.bitmap_words = (nb + 31) / 32;
+  const long cap = (long)topk + sink_blocks + window_blocks;
+  p.list_cap = (int)(cap < nb ? cap : nb);
+  for (int j = 0; j < Hr; ++j) p.head[j] = heads[j];
+  if (block_list_bytes(p) > 96 * 1024) return RTP_ERR_UNSUPPORTED;
+  return from_cuda(launch_prefill_attn_simt(p, nb, B, (cudaStream_t)stream));
+}
+
+size_t rtp_workspace_size_sparse_attn_decode(int B, int L, int Hq, int Hr, int topk, int window) {
+  (void)Hq;
+  return decode_attn_ws_bytes(B, L, Hr, topk, window);
+}
+
+rtp_status rtp_sparse_attn_decode(const void* q, const void* kc, rtp_strides ks,
+                                  const void* vc, rtp_strides vs, void* o,
+                                  int B, int L, int Hq, int Hkv, const int32_t* heads, int Hr,
+                                  const int32_t* idx, int topk, int window, int sink, float scale,
+                                  void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  if (!q || !kc || !vc || !o || !idx) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || topk < 1) return RTP_ERR_INVALID_ARG;
+  if (window < 1 || sink < 0 || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(o) || !aligned16(idx)) return RTP_ERR_INVALID_ARG;
+  if (!stride_ok(ks) || !stride_ok(vs)) return RTP_ERR_INVALID_ARG;
+  rtp_status st = check_heads(heads, Hr, Hq);
+  if (st != RTP_OK) return st;
+  const size_t need = decode_attn_ws_bytes(B, L, Hr, topk, window);
+  if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
+  if ((st = check_device()) != RTP_OK) return st;
+  return from_cuda(launch_decode_attn(q, (int64_t)Hq * RTP_D, RTP_D, kc, ks.b, ks.n, ks.h,
+                                      vc, vs.b, vs.n, vs.h, o, (int64_t)Hq * RTP_D, RTP_D,
+                                      B, L, L - 1, Hq, Hkv, heads, Hr, 1, idx, topk, window, sink,
+                                      scale, ws, (cudaStream_t)stream));
+}
+
+size_t rtp_workspace_size_swa(int B, int Nq, int Nk, int n_heads, int window) {
+  if (Nq != 1) return 0;
+  return decode_attn_ws_bytes(B, Nk, n_heads, 0, window);
+}
+
+rtp_status rtp_swa(const void* q, rtp_strides qs, const void* k, rtp_strides ks,
+                   const void* v, rtp_strides vs, void* o, rtp_strides os,
+                   int B, int Nq, int Nk, int q_pos0, int Hq, int Hkv,
+                   const int32_t* heads, int n_heads, int window, float scale,
+                   void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  if (!q || !k || !v || !o) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || Nq < 1 || Nk < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return RTP_ERR_INVALID_ARG;
+  if (q_pos0 < 0 || (int64_t)q_pos0 + Nq > Nk) return RTP_ERR_INVALID_ARG;
+  if (window < 1 || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
+  if (!stride_ok(qs) || !stride_ok(ks) || !stride_ok(vs) || !stride_ok(os)) return RTP_ERR_INVALID_ARG;
+  rtp_status st = check_heads(heads, n_heads, Hq);
+  if (st != RTP_OK) return st;
+  if (Nq == 1) {
+    const size_t need = decode_attn_ws_bytes(B, Nk, n_heads, 0, window);
+    if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
+    if ((st = check_device()) != RTP_OK) return st;
+    return from_cuda(launch_decode_attn(q, qs.b, qs.h, k, ks.b, ks.n, ks.h, v, vs.b, vs.n, vs.h,
+                                        o, os.b, os.h, B, Nk, q_pos0, Hq, Hkv, heads, n_heads, 0,
+                                        nullptr, 0, window, 0, scale, ws, (cudaStream_t)stream));
+  }
+  if (Nq % RTP_BLOCK != 0) return RTP_ERR_UNSUPPORTED;
+  if ((st = check_device()) != RTP_OK) return st;
+  PrefillAttnParams p{};
+  p.q = {q, qs.b, qs.n, qs.h}; p.k = {k, ks.b, ks.n, ks.h}; p.v = {v, vs.b, vs.n, vs.h};
+  p.o = o; p.o_sb = os.b; p.o_sn = os.n; p.o_sh = os.h;
+  p.Nq = Nq; p.Nk = Nk; p.q_pos0 = q_pos0; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv;
+  p.sparse = 0; p.window_tokens = window;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_heads = n_heads;
+  for (int j = 0; j < n_heads; ++j) p.head[j] = heads[j];
+  return from_cuda(launch_prefill_attn_simt(p, Nq / RTP_BLOCK, B, (cudaStream_t)stream));
+}
+
+}  // extern "C"

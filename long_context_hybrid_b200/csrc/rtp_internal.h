@@ -1,0 +1,50 @@
+// Internal launch entry points behind the C ABI (validated arguments only).
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace rtp {
+
+struct HeadList;
+
+cudaError_t launch_project(const void* x, int64_t sb, int64_t sn, int64_t sh, int B, int N,
+                           const void* P, const int32_t* heads, const int32_t* proj, int n_heads,
+                           void* out, int out_f32, cudaStream_t stream);
+
+size_t select_decode_ws_bytes(int B, int L, int Hr, int topk);
+cudaError_t launch_select_decode(const float* qt, const void* kindex, int B, int L, int Hr,
+                                 int Hkv, const int32_t* kv_of, int topk, int32_t* idx,
+                                 void* ws, cudaStream_t stream);
+
+size_t select_prefill_ws_bytes(int B, int N, int Hr, int topk);
+cudaError_t launch_select_prefill(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
+                                  const int32_t* kv_of, int topk, int32_t* blocks,
+                                  int32_t* counts, void* ws, cudaStream_t stream);
+
+// Decode attention (one query per sequence) for a list of heads; retrieval
+// heads (is_ret) add their selected tokens and the sink to the window.
+size_t decode_attn_ws_bytes(int B, int L, int n_heads, int topk, int window);
+cudaError_t launch_decode_attn(const void* q, int64_t q_sb, int64_t q_sh,
+                               const void* kc, int64_t k_sb, int64_t k_sn, int64_t k_sh,
+                               const void* vc, int64_t v_sb, int64_t v_sn, int64_t v_sh,
+                               void* o, int64_t o_sb, int64_t o_sh,
+                               int B, int L, int q_pos, int Hq, int Hkv,
+                               const int32_t* heads, int n_heads, int is_ret,
+                               const int32_t* idx, int topk, int window, int sink, float scale,
+                               void* ws, cudaStream_t stream);
+
+// Prefill attention over per-query-block key-block lists (SWA band or
+// selected/sink/window union).
+struct Tensor4 {
+  const void* p;
+  int64_t sb, sn, sh;
+};
+cudaError_t launch_prefill_attn(Tensor4 q, Tensor4 k, Tensor4 v, void* o, int64_t o_sb,
+                                int64_t o_sn, int64_t o_sh, int B, int Nq, int Nk, int q_pos0,
+                                int Hq, int Hkv, const int32_t* heads, int n_heads,
+                                int sparse, const int32_t* blocks, const int32_t* counts, int topk,
+                                int window_tokens, int window_blocks, int sink_blocks, float scale,
+                                cudaStream_t stream);
+
+}  // namespace rtp

@@ -251,13 +251,16 @@ def kv_of(h: int, Hq: int, Hkv: int) -> int:
 
 def prefill_layer(q, k, v, P, ret_heads, window: int, ret_window: int, topk: int,
                   scale: float, qblocks=None, sink_blocks: int = 1, heads=None,
-                  block: int = BLOCK):
+                  block: int = BLOCK, index=None):
     """One prefill layer for batch element 0-sliced tensors.
 
     ``q`` [N, Hq, D], ``k``/``v`` [N, Hkv, D], ``P`` [Hkv, D, r] (bf16 values).
     Computes the output rows of the query blocks ``qblocks`` (default: all)
     for ``heads`` (default: all). Returns a dict with ``out`` {(h, i): [64, D]},
     ``sel``/``scores`` {(h, i): ...} for retrieval heads, and ``kt``/``qt``.
+    ``index`` may carry already projected ``{"kt": {g: ...}, "qt": {h: ...}}``
+    (the output of ``project``) so that a caller sampling a few query blocks
+    projects the sequence once.
     """
     P = to_f64(P)
     N, Hq, D = q.shape
@@ -267,14 +270,16 @@ def prefill_layer(q, k, v, P, ret_heads, window: int, ret_window: int, topk: int
     heads = list(range(Hq)) if heads is None else list(heads)
     ret = set(ret_heads)
     wb = ret_window // block
-    kt_cache, res = {}, dict(out={}, sel={}, scores={}, kt={}, qt={})
+    kt_cache = dict(index["kt"]) if index else {}
+    qt_given = index["qt"] if index else {}
+    res = dict(out={}, sel={}, scores={}, kt={}, qt={})
     for h in heads:
         g = kv_of(h, Hq, Hkv)
         if h in ret:
             if g not in kt_cache:
                 kt_cache[g] = project(k[:, g, :], P[g])
             kt = kt_cache[g]
-            qt = project(q[:, h, :], P[g])
+            qt = qt_given[h] if h in qt_given else project(q[:, h, :], P[g])
             res["kt"][g], res["qt"][h] = kt, qt
             sel, sc = select_prefill(qt, kt, topk, qblocks, block)
             for i in qblocks:

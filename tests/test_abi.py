@@ -1,0 +1,109 @@
+"""CPU checks of the C ABI: the library builds, loads, exports every call the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rtp.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from long_context_hybrid_b200 import build
+    build.build()
+    import long_context_hybrid_b200 as rtp
+    return rtp.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"RTP_API\s+[\w\s\*]+?\b(rtp_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_six_calls():
+    syms = declared_symbols()
+    for name in ("rtp_index_project", "rtp_select_prefill", "rtp_select_decode",
+                 "rtp_sparse_attn_prefill", "rtp_sparse_attn_decode", "rtp_swa"):
+        assert name in syms
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_version_and_status_strings(L):
+    assert L.rtp_version() == 1
+    for s, name in enumerate(["RTP_OK", "RTP_ERR_INVALID_ARG", "RTP_ERR_UNSUPPORTED", "RTP_ERR_CUDA",
+                              "RTP_ERR_TIMEOUT", "RTP_ERR_WORKSPACE"]):
+        assert L.rtp_status_string(s).decode() == name
+    assert L.rtp_status_string(99).decode() == "RTP_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(L):
+    # Decode selection keeps one fp32 score per (sequence, retrieval head, token).
+    assert L.rtp_workspace_size_select_decode(8, 131072, 5, 2048) >= 8 * 5 * 131072 * 4
+    assert L.rtp_workspace_size_sparse_attn_decode(8, 131072, 32, 5, 2048, 8192) > 0
+    assert L.rtp_workspace_size_swa(8, 1, 131072, 27, 8192) > 0
+    assert L.rtp_workspace_size_swa(1, 4096, 4096, 27, 1024) == 0
+
+
+def _heads(vals):
+    return (ctypes.c_int32 * len(vals))(*vals)
+
+
+def test_rejects_bad_arguments_without_launching(L):
+    import long_context_hybrid_b200 as rtp
+    S = rtp.Strides
+    fake = 0x10000   # never dereferenced: validation fails first
+    INVALID, UNSUP, WS = 1, 2, 5
+    st = S(8192, 512, 128)
+    # null pointer
+    assert L.rtp_index_project(None, st, 1, 64, 4, fake, 1, 16, _heads([0]), _heads([0]), 1, fake, 0, None) == INVALID
+    # r != 16
+    assert L.rtp_index_project(fake, st, 1, 64, 4, fake, 1, 8, _heads([0]), _heads([0]), 1, fake, 0, None) == UNSUP
+    # head out of range, duplicate heads
+    assert L.rtp_index_project(fake, st, 1, 64, 4, fake, 1, 16, _heads([4]), _heads([0]), 1, fake, 0, None) == INVALID
+    assert L.rtp_index_project(fake, st, 1, 64, 4, fake, 1, 16, _heads([1, 1]), _heads([0, 0]), 2, fake, 0, None) == INVALID
+    # misaligned pointer / stride
+    assert L.rtp_index_project(fake + 2, st, 1, 64, 4, fake, 1, 16, _heads([0]), _heads([0]), 1, fake, 0, None) == INVALID
+    assert L.rtp_index_project(fake, S(8192, 516, 128), 1, 64, 4, fake, 1, 16, _heads([0]), _heads([0]), 1, fake, 0, None) == INVALID
+    # N not a multiple of 64 for prefill selection
+    assert L.rtp_select_prefill(fake, fake, 1, 100, 1, 1, 16, _heads([0]), 4, fake, fake, None, 0, None) == UNSUP
+    # kv head out of range
+    assert L.rtp_select_prefill(fake, fake, 1, 128, 1, 1, 16, _heads([1]), 4, fake, fake, None, 0, None) == INVALID
+    # decode selection without a workspace
+    assert L.rtp_select_decode(fake, fake, 1, 1000, 1, 1, 16, _heads([0]), 8, fake, None, 0, None) == WS
+    assert L.rtp_select_decode(fake, fake, 1, 1000, 1, 1, 16, _heads([0]), 8, fake, fake, 10, None) == WS
+    assert L.rtp_select_decode(fake, fake, 1, 1000, 1, 1, 16, _heads([0]), 5000, fake, fake, 1 << 30, None) == UNSUP
+    # sparse prefill: bad window / scale / GQA ratio
+    qs = S(64 * 8 * 128, 8 * 128, 128)
+    ks = S(64 * 2 * 128, 2 * 128, 128)
+    assert L.rtp_sparse_attn_prefill(fake, qs, fake, ks, fake, ks, fake, qs, 1, 64, 8, 2, _heads([0]), 1,
+                                     fake, fake, 4, 0, 1, ctypes.c_float(0.1), None, 0, None) == INVALID
+    assert L.rtp_sparse_attn_prefill(fake, qs, fake, ks, fake, ks, fake, qs, 1, 64, 8, 2, _heads([0]), 1,
+                                     fake, fake, 4, 1, 1, ctypes.c_float(-1.0), None, 0, None) == INVALID
+    assert L.rtp_sparse_attn_prefill(fake, qs, fake, ks, fake, ks, fake, qs, 1, 64, 8, 3, _heads([0]), 1,
+                                     fake, fake, 4, 1, 1, ctypes.c_float(0.1), None, 0, None) == INVALID
+    # SWA: query positions past the keys, prefill Nq not a multiple of 64
+    assert L.rtp_swa(fake, qs, fake, ks, fake, ks, fake, qs, 1, 64, 64, 1, 8, 2, _heads([1]), 1, 16,
+                     ctypes.c_float(0.1), None, 0, None) == INVALID
+    assert L.rtp_swa(fake, qs, fake, ks, fake, ks, fake, qs, 1, 65, 65, 0, 8, 2, _heads([1]), 1, 16,
+                     ctypes.c_float(0.1), None, 0, None) == UNSUP
+    # decode SWA needs a workspace
+    assert L.rtp_swa(fake, qs, fake, ks, fake, ks, fake, qs, 1, 1, 640, 639, 8, 2, _heads([1]), 1, 16,
+                     ctypes.c_float(0.1), None, 0, None) == WS
+    # decode sparse attention: idx null
+    assert L.rtp_sparse_attn_decode(fake, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, None,
+                                    16, 64, 1, ctypes.c_float(0.1), fake, 1 << 20, None) == INVALID
+
+
+def test_binding_raises_without_library(tmp_path, monkeypatch):
+    import long_context_hybrid_b200 as rtp
+    monkeypatch.setattr(rtp, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(rtp, "_lib", None)
+    with pytest.raises(rtp.RtpError):
+        rtp.lib()

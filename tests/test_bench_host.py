@@ -1,0 +1,75 @@
+"""Host-side logic of bench.py: the algorithmic work counts (checked against
+the oracle's own attended sets) and the multi-rank timing reduction (gloo,
+world size 2, on CPU)."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+import oracle as O
+
+
+def test_swa_pairs_brute():
+    for N, W in [(10, 3), (10, 10), (10, 50), (1000, 64), (4096, 4096)]:
+        want = sum(min(t + 1, W) for t in range(N))
+        assert bench.swa_pairs(N, W) == want
+
+
+def test_causal_pairs_brute():
+    for N in (64, 128, 640):
+        assert bench.causal_pairs(N) == N * (N + 1) // 2
+
+
+def test_sparse_pairs_matches_oracle_sets():
+    rs = np.random.default_rng(0)
+    nb, k, wb, sink = 40, 6, 5, 1
+    blocks = -np.ones((1, 2, nb, k), np.int32)
+    counts = np.zeros((1, 2, nb), np.int32)
+    want = 0
+    for j in range(2):
+        for i in range(nb):
+            n = min(k, i + 1)
+            sel = np.sort(rs.choice(i + 1, n, replace=False))
+            blocks[0, j, i, :n] = sel
+            counts[0, j, i] = n
+            att = O.attended_blocks(sel, i, wb, sink)
+            want += sum(64 * 64 if jb < i else 64 * 65 // 2 for jb in att)
+    got = bench.sparse_pairs(torch.from_numpy(blocks), torch.from_numpy(counts), wb, sink)
+    assert got == want
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    v = bench.max_over_ranks(float(10 + rank * 5), world)
+    bench.barrier(world)
+    out[rank] = v
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert out[0] == 15.0 and out[1] == 15.0

@@ -1,0 +1,130 @@
+"""Full-size parity: each seeded workload runs on the GPU at its full size, in
+the launch configuration the benchmark times; the oracle recomputes sampled
+outputs one by one (prefill: the first and last query blocks, the blocks at the
+window boundary and seeded random blocks, every head; decode: whole
+sequences). Selections follow the band rule; outputs the attention tolerance.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from helpers import assert_attn_close, assert_index_close, band_check
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+rtp = pytest.importorskip("long_context_hybrid_b200")
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from long_context_hybrid_b200 import build
+    build.build()
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    rtp.lib()
+
+
+def _f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def sample_blocks(cfg, n_random=3, seed=0):
+    nb = cfg.N // 64
+    wb = cfg.ret_window // 64
+    rs = np.random.default_rng(seed)
+    picks = {0, nb - 1, min(nb - 1, wb - 1), min(nb - 1, wb), min(nb - 1, cfg.topk), min(nb - 1, cfg.topk + 1)}
+    picks |= set(rs.choice(nb, n_random, replace=False).tolist())
+    return sorted(picks)
+
+
+def run_prefill_fullsize(cfg, n_random=3):
+    d = synth.make_prefill(cfg, device=DEV)
+    q, k, v, P = d["q"], d["k"], d["v"], d["P"]
+    layer = rtp.PrefillLayer(cfg.B, cfg.N, cfg.Hq, cfg.Hkv, cfg.ret_heads, cfg.window, cfg.ret_window,
+                             cfg.topk, DEV)
+    o = torch.zeros(cfg.B, cfg.N, cfg.Hq, 128, dtype=torch.bfloat16, device=DEV)
+    layer(q, k, v, P, o)
+    torch.cuda.synchronize()
+    qb = sample_blocks(cfg, n_random)
+    qc, kc, vc, Pc = q[0].cpu(), k[0].cpu(), v[0].cpu(), P.cpu()
+    G = cfg.Hq // cfg.Hkv
+    kt = {g: O.project(kc[:, g, :], Pc[g]) for g in layer.kv_used}
+    qt = {h: O.project(qc[:, h, :], Pc[h // G]) for h in cfg.ret_heads}
+    # the GPU's index: a sample of rows must satisfy the projection bound
+    rows = torch.arange(0, cfg.N, max(1, cfg.N // 4096))
+    for slot, g in enumerate(layer.kv_used):
+        assert_index_close(_f64(layer.kt[0, slot, rows]), kc[rows, g, :], Pc[g])
+    res = O.prefill_layer(qc, kc, vc, Pc, cfg.ret_heads, cfg.window, cfg.ret_window, cfg.topk,
+                          1 / math.sqrt(128), qblocks=qb, index={"kt": kt, "qt": qt})
+    blocks = layer.blocks.cpu().numpy() if layer.ret else None
+    outs, refs, n_tol = [], [], 0
+    for (h, i), ref in res["out"].items():
+        if h in cfg.ret_heads:
+            j = layer.ret.index(h)
+            n = min(cfg.topk, i + 1)
+            got = blocks[0, j, i, :n]
+            ok, amb, msg = band_check(got, res["sel"][(h, i)], res["scores"][(h, i)], cfg.topk)
+            assert ok, f"{cfg.name} selection h{h} i{i}: {msg}"
+            if not np.array_equal(np.sort(got), res["sel"][(h, i)]):
+                n_tol += 1
+                continue
+        outs.append(_f64(o[0, i * 64:(i + 1) * 64, h].cpu()))
+        refs.append(ref)
+    assert n_tol <= max(2, len(res["out"]) // 20)
+    return assert_attn_close(np.stack(outs), np.stack(refs), cfg.name)
+
+
+def run_decode_fullsize(cfg, seqs):
+    d = synth.make_decode(cfg, device=DEV)
+    q, kc, vc, P = d["q"], d["kc"], d["vc"], d["P"]
+    B, L = cfg.B, cfg.L
+    kindex = rtp.index_project(kc, P, list(range(cfg.Hkv)), list(range(cfg.Hkv)))
+    step = rtp.DecodeStep(B, L, cfg.Hq, cfg.Hkv, cfg.ret_heads, cfg.window, cfg.ret_window, cfg.topk, DEV,
+                          sink=cfg.sink)
+    o = torch.zeros(B, cfg.Hq, 128, dtype=torch.bfloat16, device=DEV)
+    step(q, kc, vc, kindex, P, o)
+    torch.cuda.synchronize()
+    idx = step.idx.cpu().numpy()
+    outs, refs, n_tol = [], [], 0
+    for b in seqs:
+        kcb, vcb = kc[b].cpu(), vc[b].cpu()
+        res = O.decode_layer(q[b].cpu(), kcb, vcb, P.cpu(), cfg.ret_heads, cfg.window, cfg.ret_window,
+                             cfg.topk, 1 / math.sqrt(128), sink=cfg.sink)
+        for g in res["kt"]:
+            assert_index_close(_f64(kindex[b, g]), kcb[:, g, :], P[g].cpu())
+        for h, ref in res["out"].items():
+            if h in cfg.ret_heads:
+                j = list(cfg.ret_heads).index(h)
+                ok, amb, msg = band_check(idx[b, j], res["sel"][h], res["scores"][h], cfg.topk)
+                assert ok, f"{cfg.name} b{b} h{h}: {msg}"
+                if not np.array_equal(np.sort(idx[b, j]), res["sel"][h]):
+                    n_tol += 1
+                    continue
+            outs.append(_f64(o[b, h].cpu()))
+            refs.append(ref)
+    return assert_attn_close(np.stack(outs), np.stack(refs), cfg.name)
+
+
+def test_prefill_32k_fullsize():
+    run_prefill_fullsize(synth.PREFILL_32K)
+
+
+def test_decode_128k_b8_fullsize():
+    run_decode_fullsize(synth.DECODE_128K, seqs=range(synth.DECODE_128K.B))
+
+
+def test_prefill_1m_fullsize():
+    run_prefill_fullsize(synth.PREFILL_1M, n_random=2)
+
+
+def test_prefill_128k_all_sparse_fullsize():
+    run_prefill_fullsize(synth.PREFILL_128K_ALL)
+
+
+def test_decode_64k_b32_all_sparse_fullsize():
+    run_decode_fullsize(synth.DECODE_64K_ALL, seqs=[0, 13, 31])

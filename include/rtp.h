@@ -83,6 +83,16 @@ RTP_API const char* rtp_status_string(rtp_status s);
 RTP_API int rtp_version(void);
 
 /*
+ * rtp_workspace_status - device-side status of the last call that used `ws`.
+ *   The prefill attention calls keep a status word in the first bytes of
+ *   their workspace: cleared on the stream before the launch, set to
+ *   RTP_ERR_TIMEOUT by a CTA whose bounded wait ran out (the kernel then
+ *   drains and returns instead of spinning). This call synchronises `stream`
+ *   and returns RTP_OK or the recorded status.
+ */
+RTP_API rtp_status rtp_workspace_status(const void* ws, rtp_stream_t stream);
+
+/*
  * rtp_index_project - the low-rank indexer projection x~ = x . P.
  *   Source: RTPurboV2 article, paragraph on the low-rank projector (feature
  *   dimension compressed from D to r = 16); the precomputed 16-d key index
@@ -119,8 +129,11 @@ RTP_API rtp_status rtp_index_project(const void* x, rtp_strides xs, int B, int N
  *   blocks   int32 [B, Hr, N/64, topk] device out: ascending block indices,
  *            min(k, i+1) of them, the rest -1.
  *   counts   int32 [B, Hr, N/64] device out: min(k, i+1).
- *   ws       workspace of rtp_workspace_size_select_prefill() bytes.
- *   N must be a multiple of 64, r = 16.
+ *   ws       workspace of rtp_workspace_size_select_prefill() bytes (the
+ *            status word, see rtp_workspace_status).
+ *   N must be a multiple of 64, r = 16; the block scores of a query-block
+ *   pair are kept on chip, which bounds N at about 1.4M tokens
+ *   (RTP_ERR_UNSUPPORTED beyond).
  */
 RTP_API size_t rtp_workspace_size_select_prefill(int B, int N, int Hr, int topk);
 RTP_API rtp_status rtp_select_prefill(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
@@ -167,6 +180,8 @@ RTP_API rtp_status rtp_select_decode(const float* qt, const void* kindex, int B,
  *            [0, i] are ignored).
  *   window_blocks >= 1, sink_blocks >= 0, scale > 0 (the softmax scale,
  *   1/sqrt(D) in the method's usual form).
+ *   ws       at least rtp_workspace_size_sparse_attn_prefill() bytes (the
+ *            status word, see rtp_workspace_status).
  */
 RTP_API size_t rtp_workspace_size_sparse_attn_prefill(int B, int N, int Hr, int topk);
 RTP_API rtp_status rtp_sparse_attn_prefill(const void* q, rtp_strides qs, const void* k, rtp_strides ks,
@@ -213,6 +228,8 @@ RTP_API rtp_status rtp_sparse_attn_decode(const void* q, const void* kc, rtp_str
  *   k, v     bf16 [B, Nk, Hkv, D] device (strides ks, vs).
  *   heads    host int32 [n_heads]: the streaming heads to compute.
  *   window >= 1, scale > 0. Prefill (Nq > 1) needs Nq % 64 == 0.
+ *   ws       at least rtp_workspace_size_swa() bytes: the split-K partials
+ *            for a single query (Nq == 1), the status word otherwise.
  */
 RTP_API size_t rtp_workspace_size_swa(int B, int Nq, int Nk, int n_heads, int window);
 RTP_API rtp_status rtp_swa(const void* q, rtp_strides qs, const void* k, rtp_strides ks,

@@ -41,6 +41,7 @@ _SZ = ctypes.c_size_t
 _SIGNATURES = {
     "rtp_status_string": (ctypes.c_char_p, [_I]),
     "rtp_version": (_I, []),
+    "rtp_workspace_status": (_I, [_P, _P]),
     "rtp_index_project": (_I, [_P, Strides, _I, _I, _I, _P, _I, _I, _c_i32p, _c_i32p, _I, _P, _I, _P]),
     "rtp_workspace_size_select_prefill": (_SZ, [_I, _I, _I, _I]),
     "rtp_select_prefill": (_I, [_P, _P, _I, _I, _I, _I, _I, _c_i32p, _I, _P, _P, _P, _SZ, _P]),
@@ -106,6 +107,12 @@ def _wsptr(buf):
     if buf is None:
         return None
     return buf if isinstance(buf, int) else buf.data_ptr()
+
+
+def workspace_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream and returns the status word a prefill attention
+    call left in ``ws`` (0 = RTP_OK, 4 = RTP_ERR_TIMEOUT)."""
+    return lib().rtp_workspace_status(ws.data_ptr(), _stream(stream))
 
 
 def kv_of(h: int, Hq: int, Hkv: int) -> int:
@@ -233,6 +240,10 @@ class PrefillLayer:
         self.kv_used = sorted(set(self.kv_ret))
         self.kv_slot = [self.kv_used.index(g) for g in self.kv_ret]
         nb = N // BLOCK
+        self.ws_sparse = torch.zeros(lib().rtp_workspace_size_sparse_attn_prefill(B, N, max(1, len(self.ret)), topk),
+                                     dtype=torch.uint8, device=device)
+        self.ws_swa = torch.zeros(lib().rtp_workspace_size_swa(B, N, N, max(1, len(self.swa_heads)), window),
+                                  dtype=torch.uint8, device=device)
         if self.ret:
             self.kt = torch.empty(B, len(self.kv_used), N, R_INDEX, dtype=torch.bfloat16, device=device)
             self.qt = torch.empty(B, len(self.ret), N, R_INDEX, dtype=torch.bfloat16, device=device)
@@ -246,10 +257,14 @@ class PrefillLayer:
             select_prefill(self.qt, self.kt, self.kv_slot, self.topk, self.blocks, self.counts,
                            stream=stream)
             sparse_attn_prefill(q, k, v, o, self.ret, self.blocks, self.counts, self.window_blocks,
-                                self.sink_blocks, self.scale, stream=stream)
+                                self.sink_blocks, self.scale, ws=self.ws_sparse, stream=stream)
         if self.swa_heads:
-            swa(q, k, v, o, self.swa_heads, self.window, 0, self.scale, stream=stream)
+            swa(q, k, v, o, self.swa_heads, self.window, 0, self.scale, ws=self.ws_swa, stream=stream)
         return o
+
+    def device_status(self, stream=None) -> int:
+        """Synchronises and returns the worst status word of the attention calls."""
+        return max(workspace_status(self.ws_sparse, stream), workspace_status(self.ws_swa, stream))
 
 
 class DecodeStep:

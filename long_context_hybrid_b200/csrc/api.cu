@@ -38,9 +38,32 @@ rtp_status check_heads(const int32_t* heads, int n, int H) {
   return RTP_OK;
 }
 
+// Tensor maps for q/k/v and the tcgen05 launch; the status word (first 4 bytes
+// of ws) is cleared on the stream first and set by a CTA whose wait ran out.
+rtp_status launch_tc(PrefillAttnParams& p, int B, void* ws, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_bnhd(&tq, p.q.p, B, p.Nq, p.Hq, p.q.sb, p.q.sn, p.q.sh, 128) ||
+      !make_tmap_bnhd(&tk, p.k.p, B, p.Nk, p.Hkv, p.k.sb, p.k.sn, p.k.sh, 64) ||
+      !make_tmap_bnhd(&tv, p.v.p, B, p.Nk, p.Hkv, p.v.sb, p.v.sn, p.v.sh, 64))
+    return RTP_ERR_CUDA;
+  if (prefill_attn_tc_smem_bytes(p) > 227 * 1024) return RTP_ERR_UNSUPPORTED;
+  int* status = static_cast<int*>(ws);
+  if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return RTP_ERR_CUDA;
+  const int n_tiles = (p.Nq + 127) / 128;
+  return from_cuda(launch_prefill_attn_tc(p, tq, tk, tv, n_tiles, B, status, stream));
+}
+
 }  // namespace
 
 extern "C" {
+
+rtp_status rtp_workspace_status(const void* ws, rtp_stream_t stream) {
+  if (!ws) return RTP_ERR_INVALID_ARG;
+  int v = 0;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RTP_ERR_CUDA;
+  if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return RTP_ERR_CUDA;
+  return v == 0 ? RTP_OK : (rtp_status)v;
+}
 
 const char* rtp_status_string(rtp_status s) {
   switch (s) {
@@ -85,12 +108,12 @@ rtp_status rtp_select_prefill(const void* qt, const void* kt, int B, int N, int 
   if (!qt || !kt || !blocks || !counts || !kv_of) return RTP_ERR_INVALID_ARG;
   if (B < 1 || N < RTP_BLOCK || Hr < 1 || Hr > kMaxHeads || Hkv < 1 || topk < 1) return RTP_ERR_INVALID_ARG;
   if (N % RTP_BLOCK != 0 || r != RTP_R) return RTP_ERR_UNSUPPORTED;
-  if (N / RTP_BLOCK > 32768) return RTP_ERR_UNSUPPORTED;
+  if (select_prefill_tc_smem(N / RTP_BLOCK) > 227 * 1024) return RTP_ERR_UNSUPPORTED;
   if (!aligned16(qt) || !aligned16(kt) || !aligned16(blocks) || !aligned16(counts)) return RTP_ERR_INVALID_ARG;
   for (int j = 0; j < Hr; ++j)
     if (kv_of[j] < 0 || kv_of[j] >= Hkv) return RTP_ERR_INVALID_ARG;
   const size_t need = select_prefill_ws_bytes(B, N, Hr, topk);
-  if (need > 0 && (!ws || ws_bytes < need || !aligned256(ws))) return RTP_ERR_WORKSPACE;
+  if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
   rtp_status st = check_device();
   if (st != RTP_OK) return st;
   return from_cuda(launch_select_prefill(qt, kt, B, N, Hr, Hkv, kv_of, topk, blocks, counts, ws,
@@ -120,7 +143,7 @@ rtp_status rtp_select_decode(const float* qt, const void* kindex, int B, int L, 
 
 size_t rtp_workspace_size_sparse_attn_prefill(int B, int N, int Hr, int topk) {
   (void)B; (void)N; (void)Hr; (void)topk;
-  return 0;
+  return kStatusBytes;
 }
 
 rtp_status rtp_sparse_attn_prefill(const void* q, rtp_strides qs, const void* k, rtp_strides ks,
@@ -129,7 +152,6 @@ rtp_status rtp_sparse_attn_prefill(const void* q, rtp_strides qs, const void* k,
                                    const int32_t* blocks, const int32_t* counts, int topk,
                                    int window_blocks, int sink_blocks, float scale,
                                    void* ws, size_t ws_bytes, rtp_stream_t stream) {
-  (void)ws; (void)ws_bytes;
   if (!q || !k || !v || !o || !blocks || !counts) return RTP_ERR_INVALID_ARG;
   if (B < 1 || N < RTP_BLOCK || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || topk < 1) return RTP_ERR_INVALID_ARG;
   if (window_blocks < 1 || sink_blocks < 0 || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
@@ -138,6 +160,7 @@ rtp_status rtp_sparse_attn_prefill(const void* q, rtp_strides qs, const void* k,
   if (!stride_ok(qs) || !stride_ok(ks) || !stride_ok(vs) || !stride_ok(os)) return RTP_ERR_INVALID_ARG;
   rtp_status st = check_heads(heads, Hr, Hq);
   if (st != RTP_OK) return st;
+  if (!ws || ws_bytes < kStatusBytes || !aligned256(ws)) return RTP_ERR_WORKSPACE;
   if ((st = check_device()) != RTP_OK) return st;
   PrefillAttnParams p{};
   p.q = {q, qs.b, qs.n, qs.h}; p.k = {k, ks.b, ks.n, ks.h}; p.v = {v, vs.b, vs.n, vs.h};
@@ -150,11 +173,12 @@ rtp_status rtp_sparse_attn_prefill(const void* q, rtp_strides qs, const void* k,
   p.n_heads = Hr;
   const int nb = N / RTP_BLOCK;
   p.bitmap_words = (nb + 31) / 32;
-  const long cap = (long)topk + sink_blocks + window_blocks;
+  // a CTA serves two query blocks: its list is the union of two attended sets
+  const long cap = 2L * ((long)topk + sink_blocks + window_blocks);
   p.list_cap = (int)(cap < nb ? cap : nb);
   for (int j = 0; j < Hr; ++j) p.head[j] = heads[j];
-  if (block_list_bytes(p) > 96 * 1024) return RTP_ERR_UNSUPPORTED;
-  return from_cuda(launch_prefill_attn_simt(p, nb, B, (cudaStream_t)stream));
+  if (nb > 32 * 4096) return RTP_ERR_UNSUPPORTED;
+  return launch_tc(p, B, ws, (cudaStream_t)stream);
 }
 
 size_t rtp_workspace_size_sparse_attn_decode(int B, int L, int Hq, int Hr, int topk, int window) {
@@ -184,7 +208,7 @@ rtp_status rtp_sparse_attn_decode(const void* q, const void* kc, rtp_strides ks,
 }
 
 size_t rtp_workspace_size_swa(int B, int Nq, int Nk, int n_heads, int window) {
-  if (Nq != 1) return 0;
+  if (Nq != 1) return kStatusBytes;
   return decode_attn_ws_bytes(B, Nk, n_heads, 0, window);
 }
 
@@ -210,6 +234,7 @@ rtp_status rtp_swa(const void* q, rtp_strides qs, const void* k, rtp_strides ks,
                                         nullptr, 0, window, 0, scale, ws, (cudaStream_t)stream));
   }
   if (Nq % RTP_BLOCK != 0) return RTP_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < kStatusBytes || !aligned256(ws)) return RTP_ERR_WORKSPACE;
   if ((st = check_device()) != RTP_OK) return st;
   PrefillAttnParams p{};
   p.q = {q, qs.b, qs.n, qs.h}; p.k = {k, ks.b, ks.n, ks.h}; p.v = {v, vs.b, vs.n, vs.h};
@@ -218,8 +243,9 @@ rtp_status rtp_swa(const void* q, rtp_strides qs, const void* k, rtp_strides ks,
   p.sparse = 0; p.window_tokens = window;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.n_heads = n_heads;
+  p.list_cap = 0;
   for (int j = 0; j < n_heads; ++j) p.head[j] = heads[j];
-  return from_cuda(launch_prefill_attn_simt(p, Nq / RTP_BLOCK, B, (cudaStream_t)stream));
+  return launch_tc(p, B, ws, (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -107,7 +107,8 @@ __device__ __forceinline__ int list_block(const PrefillAttnParams& p, const Bloc
   return p.sparse ? sm.list[it] : sm.kb_lo + it;
 }
 
-cudaError_t launch_prefill_attn_simt(const PrefillAttnParams& p, int n_qblocks, int B,
-                                     cudaStream_t stream);
+size_t prefill_attn_tc_smem_bytes(const PrefillAttnParams& p);
+cudaError_t launch_prefill_attn_tc(const PrefillAttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                   const CUtensorMap& tmV, int n_tiles, int B, int* status, cudaStream_t stream);
 
 }  // namespace rtp

@@ -1,5 +1,6 @@
 // Internal launch entry points behind the C ABI (validated arguments only).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -46,5 +47,17 @@ cudaError_t launch_prefill_attn(Tensor4 q, Tensor4 k, Tensor4 v, void* o, int64_
                                 int sparse, const int32_t* blocks, const int32_t* counts, int topk,
                                 int window_tokens, int window_blocks, int sink_blocks, float scale,
                                 cudaStream_t stream);
+
+bool make_tmap_bnhd(CUtensorMap* map, const void* ptr, int B, int N, int H, int64_t sb, int64_t sn,
+                    int64_t sh, int box_rows);
+
+bool make_tmap_index(CUtensorMap* map, const void* ptr, int B, int H, int N, int box_rows);
+size_t select_prefill_tc_smem(int nb);
+cudaError_t launch_select_prefill_tc(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
+                                     const int32_t* kv_of, int topk, int32_t* blocks, int32_t* counts,
+                                     int* status, cudaStream_t stream);
+
+// Bytes of the status word every prefill attention call keeps in its workspace.
+constexpr size_t kStatusBytes = 256;
 
 }  // namespace rtp

@@ -168,13 +168,19 @@ prefill_select_kernel(const uint4* __restrict__ qt, const uint4* __restrict__ kt
 
 size_t select_prefill_ws_bytes(int B, int N, int Hr, int topk) {
   (void)B; (void)N; (void)Hr; (void)topk;
-  return 0;
+  return kStatusBytes;
 }
 
 cudaError_t launch_select_prefill(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
                                   const int32_t* kv_of, int topk, int32_t* blocks,
                                   int32_t* counts, void* ws, cudaStream_t stream) {
-  (void)ws;
+  return launch_select_prefill_tc(qt, kt, B, N, Hr, Hkv, kv_of, topk, blocks, counts,
+                                  static_cast<int*>(ws), stream);
+}
+
+cudaError_t launch_select_prefill_simt(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
+                                       const int32_t* kv_of, int topk, int32_t* blocks,
+                                       int32_t* counts, cudaStream_t stream) {
   HeadList hl;
   fill_heads(hl, kv_of, Hr);
   const int nb = N / RTP_BLOCK;

@@ -48,7 +48,7 @@ def test_workspace_sizes(L):
     assert L.rtp_workspace_size_select_decode(8, 131072, 5, 2048) >= 8 * 5 * 131072 * 4
     assert L.rtp_workspace_size_sparse_attn_decode(8, 131072, 32, 5, 2048, 8192) > 0
     assert L.rtp_workspace_size_swa(8, 1, 131072, 27, 8192) > 0
-    assert L.rtp_workspace_size_swa(1, 4096, 4096, 27, 1024) == 0
+    assert L.rtp_workspace_size_swa(1, 4096, 4096, 27, 1024) == 256   # status word only
 
 
 def _heads(vals):

@@ -49,7 +49,7 @@ def run_prefill_fullsize(cfg, n_random=3):
                              cfg.topk, DEV)
     o = torch.zeros(cfg.B, cfg.N, cfg.Hq, 128, dtype=torch.bfloat16, device=DEV)
     layer(q, k, v, P, o)
-    torch.cuda.synchronize()
+    assert layer.device_status() == 0
     qb = sample_blocks(cfg, n_random)
     qc, kc, vc, Pc = q[0].cpu(), k[0].cpu(), v[0].cpu(), P.cpu()
     G = cfg.Hq // cfg.Hkv

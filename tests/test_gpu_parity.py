@@ -157,8 +157,9 @@ def test_swa_prefill_matches_oracle(N, window):
     q, k, v = _qkv(B, N, Hq, Hkv, 40)
     heads = [1, 2, 3]
     o = torch.zeros(B, N, Hq, 128, dtype=torch.bfloat16, device=DEV)
-    rtp.swa(q.to(DEV), k.to(DEV), v.to(DEV), o, heads, window)
-    torch.cuda.synchronize()
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    rtp.swa(q.to(DEV), k.to(DEV), v.to(DEV), o, heads, window, ws=ws)
+    assert rtp.workspace_status(ws) == 0
     o = o.cpu()
     scale = 1 / math.sqrt(128)
     for b in range(B):
@@ -280,7 +281,7 @@ def _prefill_e2e(cfg, data, qblocks, heads=None, check_kt=True):
                              dev)
     o = torch.zeros(B, N, cfg.Hq, 128, dtype=torch.bfloat16, device=dev)
     layer(q, k, v, P, o)
-    torch.cuda.synchronize()
+    assert layer.device_status() == 0
     qc, kc, vc, Pc = q[0].cpu(), k[0].cpu(), v[0].cpu(), P.cpu()
     res = O.prefill_layer(qc, kc, vc, Pc, cfg.ret_heads, cfg.window, cfg.ret_window, cfg.topk,
                           1 / math.sqrt(128), qblocks=qblocks, heads=heads)

@@ -242,12 +242,13 @@ def run_ours(args, rank, world):
         ev[1].record(stream)
         rtp.index_project(q, P, layer.ret, layer.kv_ret, out=layer.qt)
         ev[2].record(stream)
-        rtp.select_prefill(layer.qt, layer.kt, layer.kv_slot, layer.topk, layer.blocks, layer.counts)
+        rtp.select_prefill(layer.qt, layer.kt, layer.kv_slot, layer.topk, layer.blocks, layer.counts,
+                           ws=layer.ws_sel)
         ev[3].record(stream)
         rtp.sparse_attn_prefill(q, k, v, o, layer.ret, layer.blocks, layer.counts, layer.window_blocks,
-                                layer.sink_blocks, layer.scale)
+                                layer.sink_blocks, layer.scale, ws=layer.ws_sparse)
         ev[4].record(stream)
-        rtp.swa(q, k, v, o, layer.swa_heads, layer.window, 0, layer.scale)
+        rtp.swa(q, k, v, o, layer.swa_heads, layer.window, 0, layer.scale, ws=layer.ws_swa)
         ev[5].record(stream)
 
     def decode_step(ev):
@@ -293,6 +294,8 @@ def run_ours(args, rank, world):
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop() if rank == 0 else None
+    if layer.device_status() != 0:
+        raise RuntimeError("a prefill kernel reported a timed-out wait")
 
     def per_call(evs, names):
         tot = {n: 0.0 for n in names}

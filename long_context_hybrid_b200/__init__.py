@@ -244,6 +244,8 @@ class PrefillLayer:
                                      dtype=torch.uint8, device=device)
         self.ws_swa = torch.zeros(lib().rtp_workspace_size_swa(B, N, N, max(1, len(self.swa_heads)), window),
                                   dtype=torch.uint8, device=device)
+        self.ws_sel = torch.zeros(lib().rtp_workspace_size_select_prefill(B, N, max(1, len(self.ret)), topk),
+                                  dtype=torch.uint8, device=device)
         if self.ret:
             self.kt = torch.empty(B, len(self.kv_used), N, R_INDEX, dtype=torch.bfloat16, device=device)
             self.qt = torch.empty(B, len(self.ret), N, R_INDEX, dtype=torch.bfloat16, device=device)
@@ -255,7 +257,7 @@ class PrefillLayer:
             index_project(k, P, self.kv_used, self.kv_used, out=self.kt, stream=stream)
             index_project(q, P, self.ret, self.kv_ret, out=self.qt, stream=stream)
             select_prefill(self.qt, self.kt, self.kv_slot, self.topk, self.blocks, self.counts,
-                           stream=stream)
+                           ws=self.ws_sel, stream=stream)
             sparse_attn_prefill(q, k, v, o, self.ret, self.blocks, self.counts, self.window_blocks,
                                 self.sink_blocks, self.scale, ws=self.ws_sparse, stream=stream)
         if self.swa_heads:
@@ -264,7 +266,8 @@ class PrefillLayer:
 
     def device_status(self, stream=None) -> int:
         """Synchronises and returns the worst status word of the attention calls."""
-        return max(workspace_status(self.ws_sparse, stream), workspace_status(self.ws_swa, stream))
+        return max(workspace_status(self.ws_sparse, stream), workspace_status(self.ws_swa, stream),
+                   workspace_status(self.ws_sel, stream))
 
 
 class DecodeStep:

@@ -217,6 +217,33 @@ RTP_API rtp_status rtp_sparse_attn_decode(const void* q, const void* kc, rtp_str
                                   void* ws, size_t ws_bytes, rtp_stream_t stream);
 
 /*
+ * rtp_sparse_attn_decode_noalloc - rtp_sparse_attn_decode without a workspace
+ * argument and without allocating anything.
+ *   The method's sources have no counterpart of this call: it exists for
+ *   callers that cannot provide scratch memory, such as plugins whose host
+ *   framework owns every device allocation and gives them no way to call
+ *   cudaMalloc, or latency-bound decode loops that must not pay for a
+ *   cudaMalloc/cudaFree (both may synchronise the device) on every step.
+ *
+ *   Arguments, layouts and results are those of rtp_sparse_attn_decode. The
+ *   split-K partials go to a fixed array inside the library, 4 MiB per GPU,
+ *   held by every GPU that loads the library until the process exits. A call
+ *   whose partials would not fit (about B * Hr * (ceil(window/256) +
+ *   ceil(topk/256)) * 520 bytes > 4 MiB) returns RTP_ERR_WORKSPACE and
+ *   launches nothing. The first call on a device looks up the array's device
+ *   address (with that device current) and caches it; make that first call
+ *   before any stream capture. Every call shares the one array, so calls
+ *   whose work may overlap on the GPU (different streams, or concurrent host
+ *   threads) race on it and must be serialised by the caller. Nothing in the
+ *   array needs to start at zero: each call writes every partial it reads.
+ */
+RTP_API rtp_status rtp_sparse_attn_decode_noalloc(const void* q, const void* kc, rtp_strides ks,
+                                                  const void* vc, rtp_strides vs, void* o,
+                                                  int B, int L, int Hq, int Hkv, const int32_t* heads, int Hr,
+                                                  const int32_t* idx, int topk, int window, int sink, float scale,
+                                                  rtp_stream_t stream);
+
+/*
  * rtp_swa - causal sliding-window attention of streaming heads.
  *   Source: RTPurboV2 article (streaming heads use SWA, local window 8192).
  *   Query row t sits at position q_pos0 + t and attends the keys u with

@@ -207,6 +207,27 @@ rtp_status rtp_sparse_attn_decode(const void* q, const void* kc, rtp_strides ks,
                                       scale, ws, (cudaStream_t)stream));
 }
 
+rtp_status rtp_sparse_attn_decode_noalloc(const void* q, const void* kc, rtp_strides ks,
+                                          const void* vc, rtp_strides vs, void* o,
+                                          int B, int L, int Hq, int Hkv, const int32_t* heads, int Hr,
+                                          const int32_t* idx, int topk, int window, int sink, float scale,
+                                          rtp_stream_t stream) {
+  if (!q || !kc || !vc || !o || !idx) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || topk < 1) return RTP_ERR_INVALID_ARG;
+  if (window < 1 || sink < 0 || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(o) || !aligned16(idx)) return RTP_ERR_INVALID_ARG;
+  if (!stride_ok(ks) || !stride_ok(vs)) return RTP_ERR_INVALID_ARG;
+  rtp_status st = check_heads(heads, Hr, Hq);
+  if (st != RTP_OK) return st;
+  // The partials must fit the library's fixed scratch array.
+  if (decode_attn_ws_bytes(B, L, Hr, topk, window) > kNoAllocScratchBytes) return RTP_ERR_WORKSPACE;
+  if ((st = check_device()) != RTP_OK) return st;
+  return from_cuda(launch_decode_attn_noalloc(q, (int64_t)Hq * RTP_D, RTP_D, kc, ks.b, ks.n, ks.h,
+                                              vc, vs.b, vs.n, vs.h, o, (int64_t)Hq * RTP_D, RTP_D,
+                                              B, L, L - 1, Hq, Hkv, heads, Hr, idx, topk, window, sink,
+                                              scale, (cudaStream_t)stream));
+}
+
 size_t rtp_workspace_size_swa(int B, int Nq, int Nk, int n_heads, int window) {
   if (Nq != 1) return kStatusBytes;
   return decode_attn_ws_bytes(B, Nk, n_heads, 0, window);

@@ -11,6 +11,8 @@
 // which also carries the sink). One CTA per chunk produces an unnormalised
 // partial (running max m in the log2 domain, sum l, o[128]) in the workspace;
 // a merge kernel combines the chunks of each head with the usual rescaling.
+#include <mutex>
+
 #include "rtp_common.cuh"
 #include "rtp_internal.h"
 
@@ -196,6 +198,54 @@ cudaError_t launch_decode_attn(const void* q, int64_t q_sb, int64_t q_sh,
   dim3 g2(n_heads, B);
   decode_attn_merge_kernel<<<g2, RTP_D, 0, stream>>>(p);
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant: the split-K partials live in a fixed device array.
+// ---------------------------------------------------------------------------
+// Every GPU that loads the library holds this array until the process exits.
+// Host code must not pass `g_decode_scratch` itself to a kernel (on the host
+// that name is only a stand-in); it uses the device address fetched below.
+static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+}  // namespace
+
+// Device address of g_decode_scratch on the current device, looked up once
+// per device (with that device current) and cached.
+static cudaError_t decode_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_decode_attn_noalloc(const void* q, int64_t q_sb, int64_t q_sh,
+                                       const void* kc, int64_t k_sb, int64_t k_sn, int64_t k_sh,
+                                       const void* vc, int64_t v_sb, int64_t v_sn, int64_t v_sh,
+                                       void* o, int64_t o_sb, int64_t o_sh,
+                                       int B, int L, int q_pos, int Hq, int Hkv,
+                                       const int32_t* heads, int n_heads, const int32_t* idx, int topk,
+                                       int window, int sink, float scale, cudaStream_t stream) {
+  // Every partial the merge reads is written by the same call's partial
+  // kernel, so nothing in the array has to start at zero.
+  void* scratch = nullptr;
+  cudaError_t e = decode_scratch_address(&scratch);
+  if (e != cudaSuccess) return e;
+  return launch_decode_attn(q, q_sb, q_sh, kc, k_sb, k_sn, k_sh, vc, v_sb, v_sn, v_sh, o, o_sb, o_sh, B, L,
+                            q_pos, Hq, Hkv, heads, n_heads, 1, idx, topk, window, sink, scale, scratch, stream);
 }
 
 }  // namespace rtp

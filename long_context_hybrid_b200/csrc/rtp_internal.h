@@ -35,6 +35,17 @@ cudaError_t launch_decode_attn(const void* q, int64_t q_sb, int64_t q_sh,
                                const int32_t* idx, int topk, int window, int sink, float scale,
                                void* ws, cudaStream_t stream);
 
+// Same as launch_decode_attn for retrieval heads, with the partials in a
+// library-owned static device array of kNoAllocScratchBytes.
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;
+cudaError_t launch_decode_attn_noalloc(const void* q, int64_t q_sb, int64_t q_sh,
+                                       const void* kc, int64_t k_sb, int64_t k_sn, int64_t k_sh,
+                                       const void* vc, int64_t v_sb, int64_t v_sn, int64_t v_sh,
+                                       void* o, int64_t o_sb, int64_t o_sh,
+                                       int B, int L, int q_pos, int Hq, int Hkv,
+                                       const int32_t* heads, int n_heads, const int32_t* idx, int topk,
+                                       int window, int sink, float scale, cudaStream_t stream);
+
 // Prefill attention over per-query-block key-block lists (SWA band or
 // selected/sink/window union).
 struct Tensor4 {

@@ -234,7 +234,7 @@ def run_ours(args, rank, world):
     flush = synth.flush_buffer(dev)
 
     names_p = ["project_k", "project_q", "select_prefill", "sparse_attn_prefill", "swa_prefill"]
-    names_d = ["project_q", "select_decode", "sparse_attn_decode", "swa_decode"]
+    names_d = ["project_q", "select_decode", "decode_attn_hybrid"]
 
     def prefill_step(ev):
         ev[0].record(stream)
@@ -258,12 +258,9 @@ def run_ours(args, rank, world):
         ev[1].record(stream)
         rtp.select_decode(step.qt, kindex, step.kv_ret, step.topk, step.idx, step.ws_sel)
         ev[2].record(stream)
-        rtp.sparse_attn_decode(qd, kc, vc, od, step.ret, step.idx, step.ret_window, step.sink,
-                               step.scale, step.ws_att)
+        rtp.decode_attn_hybrid(qd, kc, vc, od, step.ret, step.idx, step.ret_window, step.swa_heads,
+                               step.window, step.sink, step.scale, step.ws_att)
         ev[3].record(stream)
-        rtp.swa(qd.unsqueeze(1), kc, vc, od.unsqueeze(1), step.swa_heads, step.window, L - 1,
-                step.scale, step.ws_swa)
-        ev[4].record(stream)
 
     def new_events(n):
         return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
@@ -272,7 +269,7 @@ def run_ours(args, rank, world):
     for _ in range(args.warmup):
         prefill_step(new_events(6))
         flush.zero_()
-        decode_step(new_events(5))
+        decode_step(new_events(4))
     torch.cuda.synchronize()
 
     # ---- timed region
@@ -287,7 +284,7 @@ def run_ours(args, rank, world):
         prefill_step(e)
         pev.append(e)
         flush.zero_()                       # L2 flush between timed decode steps (not timed)
-        e = new_events(5)
+        e = new_events(4)
         decode_step(e)
         dev_ev.append(e)
         flush.zero_()
@@ -354,21 +351,20 @@ def run_ours(args, rank, world):
 
     db = decode_bytes(dcfg, step.idx, L, Bd)
     d_kern = {}
-    d_work = {"project_q": Bd * len(step.ret) * (D * 2 + R * 4), "select_decode": db["scan"],
-              "sparse_attn_decode": None, "swa_decode": None}
     for n in names_d:
         d_kern[n] = {"ms": round(d_ms[n], 4)}
     d_ach = db["total"] / (d_step_ms / 1e3) / 1e9
-    d_kern["select_decode"].update({"achieved_gbs": round(db["scan"] / (d_ms["select_decode"] / 1e3) / 1e9, 1)})
-    att_ms = d_ms["sparse_attn_decode"] + d_ms["swa_decode"]
-    d_kern["attention_total"] = {"ms": round(att_ms, 4),
-                                 "achieved_gbs": round((db["window"] + db["gathered"] + db["qo"]) / (att_ms / 1e3) / 1e9, 1)}
+    d_kern["select_decode"].update({"achieved_gbs": round(db["scan"] / (d_ms["select_decode"] / 1e3) / 1e9, 1),
+                                    "bytes": db["scan"]})
+    att_bytes = db["window"] + db["gathered"] + db["qo"]
+    d_kern["decode_attn_hybrid"].update({"achieved_gbs": round(att_bytes / (d_ms["decode_attn_hybrid"] / 1e3) / 1e9, 1),
+                                         "bytes": att_bytes})
 
     total_tokens = pcfg.B * N * world
     value = total_tokens / (p_step_ms / 1e3)
     d_value = Bd * world / (d_step_ms / 1e3)
     launches_p = 5 if (layer.ret and layer.swa_heads) else 3
-    launches = launches_p + 7   # decode: project, scan, top-k, 2 sparse, 2 SWA (partial + merge)
+    launches = launches_p + 5   # decode: project, scan, top-k, attention partials, merge
 
     # ---- end to end through the API with host buffers (rank-local, fewer steps)
     e2e = None

@@ -207,7 +207,8 @@ RTP_API rtp_status rtp_sparse_attn_prefill(const void* q, rtp_strides qs, const 
  *            token indices, -1 padded, as written by rtp_select_decode
  *            (entries in the window or below `sink` are skipped there,
  *            since those keys are attended anyway).
- *   window >= 1, sink >= 0, scale > 0.
+ *   window >= 1, 0 <= sink <= 64, scale > 0; Hq / Hkv <= 16 (the query heads
+ *   of a KV group are packed into one 16-row tensor-core tile).
  */
 RTP_API size_t rtp_workspace_size_sparse_attn_decode(int B, int L, int Hq, int Hr, int topk, int window);
 RTP_API rtp_status rtp_sparse_attn_decode(const void* q, const void* kc, rtp_strides ks,
@@ -215,6 +216,26 @@ RTP_API rtp_status rtp_sparse_attn_decode(const void* q, const void* kc, rtp_str
                                   int B, int L, int Hq, int Hkv, const int32_t* heads, int Hr,
                                   const int32_t* idx, int topk, int window, int sink, float scale,
                                   void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * rtp_decode_attn_hybrid - one decode step's attention for retrieval and
+ * streaming heads together: rtp_sparse_attn_decode on `ret_heads` (window
+ * ret_window) and rtp_swa's decode form on `swa_heads` (window swa_window),
+ * in one launch that stages each window K/V row once per KV group, so the
+ * heads of a group share it (grouped-query heads read the same keys).
+ *   Sources: RTPurboV2 article (streaming heads SWA, retrieval heads sparse);
+ *   the 128K decode workload statement.
+ *   Arguments as in the two calls it combines; Hr or n_swa may be 0 (not
+ *   both); sink <= 64; Hq / Hkv <= 16. ws: rtp_workspace_size_decode_attn_hybrid(
+ *   B, L, Hq, topk, max(ret_window, swa_window)) bytes.
+ */
+RTP_API size_t rtp_workspace_size_decode_attn_hybrid(int B, int L, int Hq, int topk, int window);
+RTP_API rtp_status rtp_decode_attn_hybrid(const void* q, const void* kc, rtp_strides ks, const void* vc,
+                                          rtp_strides vs, void* o, int B, int L, int Hq, int Hkv,
+                                          const int32_t* ret_heads, int Hr, const int32_t* idx, int topk,
+                                          int ret_window, int sink, const int32_t* swa_heads, int n_swa,
+                                          int swa_window, float scale, void* ws, size_t ws_bytes,
+                                          rtp_stream_t stream);
 
 /*
  * rtp_sparse_attn_decode_noalloc - rtp_sparse_attn_decode without a workspace
@@ -228,8 +249,8 @@ RTP_API rtp_status rtp_sparse_attn_decode(const void* q, const void* kc, rtp_str
  *   Arguments, layouts and results are those of rtp_sparse_attn_decode. The
  *   split-K partials go to a fixed array inside the library, 4 MiB per GPU,
  *   held by every GPU that loads the library until the process exits. A call
- *   whose partials would not fit (about B * Hr * (ceil(window/256) +
- *   ceil(topk/256)) * 520 bytes > 4 MiB) returns RTP_ERR_WORKSPACE and
+ *   whose partials would not fit (about B * Hr * (ceil(window/128) +
+ *   ceil((topk+64)/128)) * 520 bytes > 4 MiB) returns RTP_ERR_WORKSPACE and
  *   launches nothing. The first call on a device looks up the array's device
  *   address (with that device current) and caches it; make that first call
  *   before any stream capture. Every call shares the one array, so calls

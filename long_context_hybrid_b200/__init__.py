@@ -53,6 +53,9 @@ _SIGNATURES = {
     "rtp_workspace_size_sparse_attn_decode": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "rtp_sparse_attn_decode": (_I, [_P, _P, Strides, _P, Strides, _P, _I, _I, _I, _I, _c_i32p, _I,
                                     _P, _I, _I, _I, _F, _P, _SZ, _P]),
+    "rtp_workspace_size_decode_attn_hybrid": (_SZ, [_I, _I, _I, _I, _I]),
+    "rtp_decode_attn_hybrid": (_I, [_P, _P, Strides, _P, Strides, _P, _I, _I, _I, _I, _c_i32p, _I, _P, _I,
+                                    _I, _I, _c_i32p, _I, _I, _F, _P, _SZ, _P]),
     "rtp_workspace_size_swa": (_SZ, [_I, _I, _I, _I, _I]),
     "rtp_swa": (_I, [_P, Strides, _P, Strides, _P, Strides, _P, Strides, _I, _I, _I, _I, _I, _I,
                      _c_i32p, _I, _I, _F, _P, _SZ, _P]),
@@ -206,6 +209,26 @@ def sparse_attn_decode(q, kc, vc, o, heads: Sequence[int], idx, window: int, sin
     return o
 
 
+def decode_attn_hybrid(q, kc, vc, o, ret_heads: Sequence[int], idx, ret_window: int,
+                       swa_heads: Sequence[int], swa_window: int, sink: int = 1,
+                       scale: Optional[float] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """Decode attention of retrieval heads (idx + sink + window) and streaming
+    heads (window) in one launch. q/o [B,Hq,D], kc/vc [B,L,Hkv,D]."""
+    B, Hq, D = q.shape
+    L, Hkv = kc.shape[1], kc.shape[2]
+    topk = idx.shape[-1] if idx is not None else 0
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    wmax = max(ret_window if ret_heads else 0, swa_window if swa_heads else 0)
+    need = lib().rtp_workspace_size_decode_attn_hybrid(B, L, Hq, topk, wmax)
+    buf, nbytes = _ws(need, q.device, ws)
+    _check(lib().rtp_decode_attn_hybrid(q.data_ptr(), kc.data_ptr(), _strides4(kc), vc.data_ptr(), _strides4(vc),
+                                        o.data_ptr(), B, L, Hq, Hkv, _i32(ret_heads), len(ret_heads),
+                                        idx.data_ptr() if idx is not None else None, topk, ret_window, sink,
+                                        _i32(swa_heads), len(swa_heads), swa_window, scale, _wsptr(buf), nbytes,
+                                        _stream(stream)), "rtp_decode_attn_hybrid")
+    return o
+
+
 def swa(q, k, v, o, heads: Sequence[int], window: int, q_pos0: int = 0,
         scale: Optional[float] = None, ws: Optional[torch.Tensor] = None, stream=None):
     """Streaming-head sliding-window attention. q/o [B,Nq,Hq,D], k/v [B,Nk,Hkv,D]."""
@@ -288,11 +311,9 @@ class DecodeStep:
             self.idx = torch.empty(B, len(self.ret), topk, dtype=torch.int32, device=device)
             self.ws_sel = torch.empty(lib().rtp_workspace_size_select_decode(B, L, len(self.ret), topk),
                                       dtype=torch.uint8, device=device)
-            self.ws_att = torch.empty(lib().rtp_workspace_size_sparse_attn_decode(
-                B, L, Hq, len(self.ret), topk, ret_window), dtype=torch.uint8, device=device)
-        if self.swa_heads:
-            self.ws_swa = torch.empty(lib().rtp_workspace_size_swa(B, 1, L, len(self.swa_heads), window),
-                                      dtype=torch.uint8, device=device)
+        wmax = max(ret_window if self.ret else 0, window if self.swa_heads else 0)
+        self.ws_att = torch.empty(lib().rtp_workspace_size_decode_attn_hybrid(B, L, Hq, topk if self.ret else 0,
+                                                                              wmax), dtype=torch.uint8, device=device)
 
     def __call__(self, q, kc, vc, kindex, P, o, stream=None):
         """q/o [B,Hq,D]; kc/vc [B,L,Hkv,D]; kindex [B,Hkv,L,r]."""
@@ -300,14 +321,11 @@ class DecodeStep:
             index_project(q.unsqueeze(1), P, self.ret, self.kv_ret, out=self.qt.view(self.B, len(self.ret), 1, R_INDEX),
                           stream=stream)
             select_decode(self.qt, kindex, self.kv_ret, self.topk, self.idx, self.ws_sel, stream=stream)
-            sparse_attn_decode(q, kc, vc, o, self.ret, self.idx, self.ret_window, self.sink,
-                               self.scale, self.ws_att, stream=stream)
-        if self.swa_heads:
-            swa(q.unsqueeze(1), kc, vc, o.unsqueeze(1), self.swa_heads, self.window, self.L - 1,
-                self.scale, self.ws_swa, stream=stream)
+        decode_attn_hybrid(q, kc, vc, o, self.ret, self.idx if self.ret else None, self.ret_window,
+                           self.swa_heads, self.window, self.sink, self.scale, self.ws_att, stream=stream)
         return o
 
 
 __all__ = ["lib", "RtpError", "index_project", "select_prefill", "select_decode",
-           "sparse_attn_prefill", "sparse_attn_decode", "swa", "PrefillLayer", "DecodeStep",
+           "sparse_attn_prefill", "sparse_attn_decode", "swa", "decode_attn_hybrid", "PrefillLayer", "DecodeStep",
            "kv_of", "LIB_PATH"]

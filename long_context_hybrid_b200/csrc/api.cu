@@ -193,7 +193,8 @@ rtp_status rtp_sparse_attn_decode(const void* q, const void* kc, rtp_strides ks,
                                   void* ws, size_t ws_bytes, rtp_stream_t stream) {
   if (!q || !kc || !vc || !o || !idx) return RTP_ERR_INVALID_ARG;
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || topk < 1) return RTP_ERR_INVALID_ARG;
-  if (window < 1 || sink < 0 || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
+  if (window < 1 || sink < 0 || sink > kMaxSink || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
+  if (Hq / Hkv > 16) return RTP_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(o) || !aligned16(idx)) return RTP_ERR_INVALID_ARG;
   if (!stride_ok(ks) || !stride_ok(vs)) return RTP_ERR_INVALID_ARG;
   rtp_status st = check_heads(heads, Hr, Hq);
@@ -214,7 +215,8 @@ rtp_status rtp_sparse_attn_decode_noalloc(const void* q, const void* kc, rtp_str
                                           rtp_stream_t stream) {
   if (!q || !kc || !vc || !o || !idx) return RTP_ERR_INVALID_ARG;
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || topk < 1) return RTP_ERR_INVALID_ARG;
-  if (window < 1 || sink < 0 || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
+  if (window < 1 || sink < 0 || sink > kMaxSink || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
+  if (Hq / Hkv > 16) return RTP_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(o) || !aligned16(idx)) return RTP_ERR_INVALID_ARG;
   if (!stride_ok(ks) || !stride_ok(vs)) return RTP_ERR_INVALID_ARG;
   rtp_status st = check_heads(heads, Hr, Hq);
@@ -226,6 +228,39 @@ rtp_status rtp_sparse_attn_decode_noalloc(const void* q, const void* kc, rtp_str
                                               vc, vs.b, vs.n, vs.h, o, (int64_t)Hq * RTP_D, RTP_D,
                                               B, L, L - 1, Hq, Hkv, heads, Hr, idx, topk, window, sink,
                                               scale, (cudaStream_t)stream));
+}
+
+size_t rtp_workspace_size_decode_attn_hybrid(int B, int L, int Hq, int topk, int window) {
+  return decode_attn_ws_bytes(B, L, Hq, topk, window);
+}
+
+rtp_status rtp_decode_attn_hybrid(const void* q, const void* kc, rtp_strides ks, const void* vc, rtp_strides vs,
+                                  void* o, int B, int L, int Hq, int Hkv,
+                                  const int32_t* ret_heads, int Hr, const int32_t* idx, int topk, int ret_window,
+                                  int sink, const int32_t* swa_heads, int n_swa, int swa_window, float scale,
+                                  void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  if (!q || !kc || !vc || !o) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return RTP_ERR_INVALID_ARG;
+  if (Hr < 0 || n_swa < 0 || Hr + n_swa < 1 || Hr + n_swa > kMaxHeads) return RTP_ERR_INVALID_ARG;
+  if (Hq / Hkv > 16) return RTP_ERR_UNSUPPORTED;
+  if (Hr > 0 && (!idx || topk < 1 || ret_window < 1 || !aligned16(idx))) return RTP_ERR_INVALID_ARG;
+  if (n_swa > 0 && swa_window < 1) return RTP_ERR_INVALID_ARG;
+  if (sink < 0 || sink > kMaxSink || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
+  if (!stride_ok(ks) || !stride_ok(vs)) return RTP_ERR_INVALID_ARG;
+  int32_t all[kMaxHeads];
+  for (int i = 0; i < Hr; ++i) all[i] = ret_heads ? ret_heads[i] : -1;
+  for (int i = 0; i < n_swa; ++i) all[Hr + i] = swa_heads ? swa_heads[i] : -1;
+  rtp_status st = check_heads(all, Hr + n_swa, Hq);
+  if (st != RTP_OK) return st;
+  const int wmax = (Hr > 0 && ret_window > swa_window) || n_swa == 0 ? ret_window : swa_window;
+  const size_t need = decode_attn_ws_bytes(B, L, Hr + n_swa, Hr > 0 ? topk : 0, wmax);
+  if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
+  if ((st = check_device()) != RTP_OK) return st;
+  return from_cuda(launch_decode_hybrid(q, (int64_t)Hq * RTP_D, RTP_D, kc, ks.b, ks.n, ks.h, vc, vs.b, vs.n, vs.h,
+                                        o, (int64_t)Hq * RTP_D, RTP_D, B, L, L - 1, Hq, Hkv, ret_heads, Hr, idx, topk,
+                                        ret_window, sink, swa_heads, n_swa, swa_window, scale, ws,
+                                        (cudaStream_t)stream));
 }
 
 size_t rtp_workspace_size_swa(int B, int Nq, int Nk, int n_heads, int window) {
@@ -247,6 +282,7 @@ rtp_status rtp_swa(const void* q, rtp_strides qs, const void* k, rtp_strides ks,
   rtp_status st = check_heads(heads, n_heads, Hq);
   if (st != RTP_OK) return st;
   if (Nq == 1) {
+    if (Hq / Hkv > 16) return RTP_ERR_UNSUPPORTED;
     const size_t need = decode_attn_ws_bytes(B, Nk, n_heads, 0, window);
     if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
     if ((st = check_device()) != RTP_OK) return st;

@@ -1,28 +1,35 @@
 // Prefill attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
 //
-// One CTA computes 128 query rows of one head against a list of 64-key blocks:
-//   * streaming heads (RTPurboV2 article: SWA with a local window): the band of
-//     key blocks overlapping (pos - W, pos] for the 128 rows, with a per-element
-//     window/causal mask;
+// A CTA computes 128 * NQ query rows of one head against a list of 64-key
+// blocks:
+//   * streaming heads (RTPurboV2 article: SWA with a local window), NQ = 2:
+//     two 128-row query tiles share the band of key blocks overlapping
+//     (pos - W, pos] of their 256 rows; each row masks its own window;
 //   * retrieval heads (RTPurbo digest: exact attention at full dimension over
-//     the indexer-selected set): the rows are query blocks 2t and 2t+1, and the
-//     list is the union of their attended sets (selected blocks, sink blocks,
-//     window blocks); every entry carries which of the two halves attends it,
-//     so a row only ever sees its own block's set, with the causal mask.
+//     the indexer-selected set), NQ = 1: the 128 rows are query blocks 2t and
+//     2t+1 and the list is the union of their attended sets (selected blocks,
+//     sink blocks, window blocks); each entry carries which half attends it, so
+//     a row only sees its own block's set, with the causal mask.
 //
-// Warp roles (256 threads):
-//   warp 0      TMA producer: Q once, then K/V tiles of two list blocks per
-//               step into a 2-stage ring (128-byte swizzle);
-//   warp 1      TMEM owner and single-thread MMA issuer:
-//               S_j = Q K_j^T (M=128, N=128, K=128) into one of two TMEM S
-//               buffers, then O += P_{j-1} V_{j-1} (V read MN-major);
-//   warps 4..7  softmax: thread r owns query row r (TMEM lane r); reads S_j,
-//               masks, online softmax in the log2 domain with lazy rescaling
-//               (O in TMEM is rescaled only when the running max grows by
-//               more than 2^8), writes P_j (bf16) into swizzled shared memory
-//               for the next MMA, and finally normalises O and stores it.
-// Every wait is bounded; a wait that runs out marks the CTA aborted, all
-// roles drain, TMEM is freed and RTP_ERR_TIMEOUT is written to `status`.
+// Warp roles (64 + 128 * NQ threads):
+//   warp 0   TMA producer: the Q tiles once, then K and V of two list blocks
+//            (128 keys) per step into a 2-stage ring (128-byte swizzle);
+//   warp 1   TMEM owner and single-thread MMA issuer:
+//            S_t = Q_t K^T (M=128, N=128, K=128, both operands in shared
+//            memory) and O_t += P_t V (P read from TMEM, V read MN-major);
+//   softmax  warps 2.. : one warpgroup of 4 warps per query tile; warp w reads
+//            TMEM lanes 32 (w % 4) .. +31, so thread r owns row r (TMEM lane r):
+//            it reads S, masks, keeps an online softmax in the log2 domain
+//            with lazy rescaling (O is rescaled in TMEM only when the running
+//            max grows by more than 8), computes P with packed f32x2
+//            arithmetic (a quarter of the exponentials on the FMA pipe through
+//            a cubic for 2^f, the rest on MUFU; key halves that are masked for
+//            the whole row skip the exponentials), and writes P as bf16 back
+//            over the first half of S in TMEM, where the next MMA reads it.
+// With NQ = 2 the MMA order QK0 QK1 | PV0 QK0' PV1 QK1' | ... keeps the tensor
+// core busy on one tile while the other tile's softmax runs.
+// Every wait is bounded; a wait that runs out marks the CTA aborted, all roles
+// drain, TMEM is freed and RTP_ERR_TIMEOUT is written to `status`.
 #include "attn_prefill_common.cuh"
 #include "rtp_common.cuh"
 #include "rtp_internal.h"
@@ -33,62 +40,118 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kThreads = 256;
 constexpr int kStages = 2;
-constexpr uint32_t kQOff = 0;                                 // [D half][128 rows][128 B] = 32 KB
-constexpr uint32_t kKVOff = 32768;                            // stage s: K at s*64K, V at s*64K + 32K
-constexpr uint32_t kPOff = kKVOff + kStages * 65536u;         // [key half][128 rows][128 B] = 32 KB
-constexpr uint32_t kListOff = kPOff + 32768u;
+constexpr uint32_t kQTileBytes = 32768;                       // [D half][128 rows][128 B]
+constexpr uint32_t kStageBytes = 65536;                       // K 32 KB + V 32 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kOCol = 256;                               // O accumulator columns [256, 384)
-constexpr int kStatusTimeout = 4;                             // RTP_ERR_TIMEOUT
+constexpr int kStatusTimeout = 4;
+
+// Cubic for 2^f on [-1/2, 1/2]: Chebyshev-node least squares refined toward
+// minimax by Lawson iterations (max relative error 7.5e-5), derived for this
+// library; far below the 2^-9 rounding that P then takes as bf16.
+constexpr float kP0 = 0.99992806f, kP1 = 0.69326097f, kP2 = 0.24261113f, kP3 = 0.055171665f;
+
+template <int NQ>
+struct Layout {
+  static constexpr int kThreads = 64 + 128 * NQ;
+  static constexpr uint32_t kQOff = 0;
+  static constexpr uint32_t kKVOff = NQ * kQTileBytes;
+  static constexpr uint32_t kListOff = kKVOff + kStages * kStageBytes;
+  // TMEM columns: NQ = 2 -> tile t: S at 256 t, O at 256 t + 128.
+  //               NQ = 1 -> S buffers at 0 and 128, O at 256.
+};
 
 struct Bars {
   uint64_t q_full;
   uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full, pv_done, fin;
+  uint64_t s_full[2], p_full[2], pv_done;
+  uint64_t fin;
   uint32_t tmem_base;
   int abort;
-  int n_list;
   int kb_lo;
-  BlockScanSmem<kThreads> scan;
+  BlockScanSmem<384> scan;
 };
 
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// 2^x for a pair with x <= 8, on the FMA pipe: x = n + f, n = round(x),
+// 2^f from the cubic, 2^n added into the exponent field.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  const float magic = 12582912.f;                          // 1.5 * 2^23: round to integer
+  const uint64_t x = f2(x0, x1);
+  const uint64_t j = f2_add(x, f2(magic, magic));
+  const uint64_t n = f2_add(j, f2(-magic, -magic));
+  const uint64_t f = f2_fma(n, f2(-1.f, -1.f), x);
+  uint64_t q = f2_fma(f, f2(kP3, kP3), f2(kP2, kP2));
+  q = f2_fma(q, f, f2(kP1, kP1));
+  q = f2_fma(q, f, f2(kP0, kP0));
+  float q0, q1, j0, j1;
+  f2_split(q, q0, q1);
+  f2_split(j, j0, j1);
+  // bits(j) << 23 carries round(x) into the exponent; the magic's own bits vanish mod 2^32
+  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(j0) << 23));
+  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(j1) << 23));
+}
+
 // Marks the attended key blocks of query block q in `bits`.
+template <int NT>
 __device__ void mark_blocks(const PrefillAttnParams& p, int b, int jh, int q, unsigned* bits) {
   const int nb = p.Nq / RTP_BLOCK;
   const size_t row = ((size_t)b * p.n_heads + jh) * nb + q;
   const int cnt = min(p.counts[row], p.topk);
   const int32_t* sel = p.blocks + row * p.topk;
-  for (int e = threadIdx.x; e < cnt; e += kThreads) {
+  for (int e = threadIdx.x; e < cnt; e += NT) {
     const int x = sel[e];
     if (x >= 0 && x <= q) atomicOr(&bits[x >> 5], 1u << (x & 31));
   }
-  for (int x = threadIdx.x; x < min(p.sink_blocks, q + 1); x += kThreads) atomicOr(&bits[x >> 5], 1u << (x & 31));
-  for (int x = max(0, q - p.window_blocks + 1) + threadIdx.x; x <= q; x += kThreads)
+  for (int x = threadIdx.x; x < min(p.sink_blocks, q + 1); x += NT) atomicOr(&bits[x >> 5], 1u << (x & 31));
+  for (int x = max(0, q - p.window_blocks + 1) + threadIdx.x; x <= q; x += NT)
     atomicOr(&bits[x >> 5], 1u << (x & 31));
 }
 
 // Union list of query blocks 2t and 2t+1: entries (block, membership bits).
+template <int NT>
 __device__ int build_pair_list(const PrefillAttnParams& p, int b, int jh, int tile, unsigned* bitsA,
-                               unsigned* bitsB, int2* list, BlockScanSmem<kThreads>& scan) {
+                               unsigned* bitsB, int2* list, BlockScanSmem<NT>& scan) {
   const int nb = p.Nq / RTP_BLOCK;
   const int qa = 2 * tile, qb = 2 * tile + 1;
   const bool has_b = qb < nb;
   const int qmax = has_b ? qb : qa;
   const int nw = qmax / 32 + 1;
-  for (int w = threadIdx.x; w < nw; w += kThreads) { bitsA[w] = 0u; bitsB[w] = 0u; }
+  for (int w = threadIdx.x; w < nw; w += NT) { bitsA[w] = 0u; bitsB[w] = 0u; }
   __syncthreads();
-  mark_blocks(p, b, jh, qa, bitsA);
-  if (has_b) mark_blocks(p, b, jh, qb, bitsB);
+  mark_blocks<NT>(p, b, jh, qa, bitsA);
+  if (has_b) mark_blocks<NT>(p, b, jh, qb, bitsB);
   __syncthreads();
-  const int per = (nw + kThreads - 1) / kThreads;
+  const int per = (nw + NT - 1) / NT;
   const int w0 = threadIdx.x * per, w1 = min(nw, w0 + per);
   int c = 0;
   for (int w = w0; w < w1; ++w) c += __popc(bitsA[w] | bitsB[w]);
   int total;
-  int off = block_exclusive_scan<kThreads>(c, total, scan);
+  int off = block_exclusive_scan<NT>(c, total, scan);
   for (int w = w0; w < w1; ++w) {
     const unsigned a = bitsA[w], bb = bitsB[w];
     unsigned x = a | bb;
@@ -109,12 +172,44 @@ __device__ __forceinline__ bool wait_short(uint32_t bar, uint32_t parity) {
   return true;
 }
 
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Issue S = Q K^T for one Q tile (8 K-steps of 16 over D = 128).
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+    mma_bf16_ss(d_tmem, desc_sw128(q_smem + off, 16, 1024), desc_sw128(k_smem + off, 16, 1024), idesc,
+                kk > 0 ? 1u : 0u);
+  }
+}
+// Issue O (+)= P V for one Q tile (P in TMEM: 8 K-steps of 16 keys = 8 columns each).
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_bf16_ts(o_tmem, p_tmem + kk * 8u, desc_sw128(v_smem + kk * 2048u, 16384, 1024), idesc,
+                (accumulate || kk > 0) ? 1u : 0u);
+}
+
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int NQ>
+__global__ void __launch_bounds__(64 + 128 * NQ, 1)
 prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        int* status) {
+  using Lay = Layout<NQ>;
+  constexpr int NT = Lay::kThreads;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -122,20 +217,27 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
   const int tile = blockIdx.x, jh = blockIdx.y, b = blockIdx.z;
   const int h = p.head[jh], g = h / p.G;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int2* list = reinterpret_cast<int2*>(smem + kListOff);
-  Bars& bars = *reinterpret_cast<Bars*>(smem + kListOff + (size_t)p.list_cap * sizeof(int2));
+  int2* list = reinterpret_cast<int2*>(smem + Lay::kListOff);
+  Bars& bars = *reinterpret_cast<Bars*>(smem + Lay::kListOff + (size_t)p.list_cap * sizeof(int2));
   volatile int* abort_flag = &bars.abort;
+  const int row0 = tile * 128 * NQ;               // first query row of the CTA
 
   // ---- prologue: key-block list, barriers, TMEM
   int n_list;
-  if (p.sparse) {
-    unsigned* bitsA = reinterpret_cast<unsigned*>(smem + kPOff);
-    unsigned* bitsB = bitsA + 4096;
-    n_list = build_pair_list(p, b, jh, tile, bitsA, bitsB, list, bars.scan);
-  } else {
-    const int pos0 = p.q_pos0 + tile * 128;
+  if constexpr (NQ == 1) {
+   if (p.sparse) {
+    unsigned* bitsA = reinterpret_cast<unsigned*>(smem + Lay::kKVOff);   // stage 0 is free until the first load
+    unsigned* bitsB = bitsA + 8192;
+    n_list = build_pair_list<NT>(p, b, jh, tile, bitsA, bitsB, list,
+                                 *reinterpret_cast<BlockScanSmem<NT>*>(&bars.scan));
+   } else {
+    n_list = 0;
+   }
+  }
+  if (NQ == 2 || !p.sparse) {
+    const int pos0 = p.q_pos0 + row0;
     const int lo = max(0, pos0 - p.window_tokens + 1) / RTP_BLOCK;
-    const int hi = min(p.Nk - 1, pos0 + 127) / RTP_BLOCK;
+    const int hi = min(p.Nk - 1, pos0 + 128 * NQ - 1) / RTP_BLOCK;
     n_list = hi - lo + 1;
     if (tid == 0) bars.kb_lo = lo;
   }
@@ -148,13 +250,11 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&bars.s_full[s]), 1);
-      mbar_init(smem_u32(&bars.s_free[s]), 128);
+      mbar_init(smem_u32(&bars.p_full[s]), 128);
     }
-    mbar_init(smem_u32(&bars.p_full), 128);
     mbar_init(smem_u32(&bars.pv_done), 1);
     mbar_init(smem_u32(&bars.fin), 1);
     bars.abort = 0;
-    bars.n_list = n_list;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -175,22 +275,25 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
       tma_prefetch(&tmK);
       tma_prefetch(&tmV);
       const uint32_t qbar = smem_u32(&bars.q_full);
-      mbar_arrive_expect_tx(qbar, 32768);
-      tma_load_4d(sb + kQOff, &tmQ, qbar, 0, h, tile * 128, b);
-      tma_load_4d(sb + kQOff + 16384, &tmQ, qbar, 64, h, tile * 128, b);
+      mbar_arrive_expect_tx(qbar, kQTileBytes * NQ);
+#pragma unroll
+      for (int t = 0; t < NQ; ++t) {
+        tma_load_4d(sb + Lay::kQOff + t * kQTileBytes, &tmQ, qbar, 0, h, row0 + t * 128, b);
+        tma_load_4d(sb + Lay::kQOff + t * kQTileBytes + 16384, &tmQ, qbar, 64, h, row0 + t * 128, b);
+      }
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j & 1;
         if (j >= kStages && !mbar_wait(smem_u32(&bars.kv_empty[s]), ((j - kStages) >> 1) & 1, abort_flag)) break;
         int kb0, kb1;
-        if (p.sparse) {
+        if (NQ == 1 && p.sparse) {
           kb0 = list[2 * j].x;
           kb1 = (2 * j + 1 < n_list) ? list[2 * j + 1].x : kb0;
         } else {
           kb0 = kb_lo + 2 * j;
           kb1 = kb0 + 1;
         }
-        const uint32_t kdst = sb + kKVOff + s * 65536u, vdst = kdst + 32768u;
+        const uint32_t kdst = sb + Lay::kKVOff + s * kStageBytes, vdst = kdst + 32768u;
         const uint32_t kbar = smem_u32(&bars.k_full[s]), vbar = smem_u32(&bars.v_full[s]);
         mbar_arrive_expect_tx(kbar, 32768);
 #pragma unroll
@@ -218,76 +321,102 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
+      const uint32_t q_s = sb + Lay::kQOff;
       bool ok = mbar_wait(smem_u32(&bars.q_full), 0, abort_flag);
-      for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles) {
-          const int s = j & 1;
-          if (!mbar_wait(smem_u32(&bars.k_full[s]), (j >> 1) & 1, abort_flag)) { ok = false; break; }
-          if (j >= 2 && !mbar_wait(smem_u32(&bars.s_free[s]), ((j - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t kbase = sb + kKVOff + s * 65536u;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t koff = (kk >> 2) * 16384u + (kk & 3) * 32u;
-            mma_bf16_ss(tmem + s * 128u, desc_sw128(sb + kQOff + koff, 16, 1024),
-                        desc_sw128(kbase + koff, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+      if (NQ == 2) {
+        // QK0(0) QK1(0) | PV0(j) QK0(j+1) PV1(j) QK1(j+1) | ...
+        if (ok && n_tiles > 0) {
+          ok = mbar_wait(smem_u32(&bars.k_full[0]), 0, abort_flag);
+          if (ok) {
+            tc_fence_after();
+            issue_qk(tmem + 0, q_s, sb + Lay::kKVOff);
+            mma_commit(smem_u32(&bars.s_full[0]));
+            issue_qk(tmem + 256, q_s + kQTileBytes, sb + Lay::kKVOff);
+            mma_commit(smem_u32(&bars.s_full[1]));
           }
-          mma_commit(smem_u32(&bars.s_full[s]));
         }
-        if (j >= 1) {
-          const int jp = j - 1, s = jp & 1;
-          if (!mbar_wait(smem_u32(&bars.p_full), jp & 1, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(smem_u32(&bars.v_full[s]), (jp >> 1) & 1, abort_flag)) { ok = false; break; }
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const int s = j & 1, s1 = (j + 1) & 1;
+          const uint32_t v_s = sb + Lay::kKVOff + s * kStageBytes + 32768u;
+          const bool more = j + 1 < n_tiles;
+          if (!mbar_wait(smem_u32(&bars.p_full[0]), j & 1, abort_flag)) break;
+          if (!mbar_wait(smem_u32(&bars.v_full[s]), (j >> 1) & 1, abort_flag)) break;
           tc_fence_after();
-          const uint32_t vbase = sb + kKVOff + s * 65536u + 32768u;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t poff = (kk >> 2) * 16384u + (kk & 3) * 32u;
-            mma_bf16_ss(tmem + kOCol, desc_sw128(sb + kPOff + poff, 16, 1024),
-                        desc_sw128(vbase + kk * 2048u, 16384, 1024), idesc_pv,
-                        (jp > 0 || kk > 0) ? 1u : 0u);
+          issue_pv(tmem + 128, tmem + 0, v_s, j > 0);
+          if (more) {
+            if (!mbar_wait(smem_u32(&bars.k_full[s1]), ((j + 1) >> 1) & 1, abort_flag)) break;
+            tc_fence_after();
+            issue_qk(tmem + 0, q_s, sb + Lay::kKVOff + s1 * kStageBytes);
+            mma_commit(smem_u32(&bars.s_full[0]));
           }
-          mma_commit(smem_u32(&bars.pv_done));
+          if (!mbar_wait(smem_u32(&bars.p_full[1]), j & 1, abort_flag)) break;
+          tc_fence_after();
+          issue_pv(tmem + 384, tmem + 256, v_s, j > 0);
           mma_commit(smem_u32(&bars.kv_empty[s]));
+          if (more) {
+            issue_qk(tmem + 256, q_s + kQTileBytes, sb + Lay::kKVOff + s1 * kStageBytes);
+            mma_commit(smem_u32(&bars.s_full[1]));
+          }
+        }
+      } else {
+        // QK(0) | QK(j+1) PV(j) | ... with S double-buffered
+        for (int j = 0; ok && j <= n_tiles; ++j) {
+          if (j < n_tiles) {
+            const int s = j & 1;
+            if (!mbar_wait(smem_u32(&bars.k_full[s]), (j >> 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_qk(tmem + s * 128u, q_s, sb + Lay::kKVOff + s * kStageBytes);
+            mma_commit(smem_u32(&bars.s_full[s]));
+          }
+          if (j >= 1) {
+            const int jp = j - 1, s = jp & 1;
+            if (!mbar_wait(smem_u32(&bars.p_full[s]), (jp >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(smem_u32(&bars.v_full[s]), (jp >> 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(tmem + 256, tmem + s * 128u, sb + Lay::kKVOff + s * kStageBytes + 32768u, jp > 0);
+            mma_commit(smem_u32(&bars.pv_done));
+            mma_commit(smem_u32(&bars.kv_empty[s]));
+          }
         }
       }
       mma_commit(smem_u32(&bars.fin));
       wait_short(smem_u32(&bars.fin), 0);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------------ softmax
-    const int r = tid - 128;
-    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const int row = tile * 128 + r;
+    const int t = (warp - 2) >> 2;                  // query tile of this warpgroup
+    const int r = (warp & 3) * 32 + lane;           // row within the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const int row = row0 + t * 128 + r;
     const int pos = p.q_pos0 + row;
     const int rowbit = r < 64 ? 1 : 2;
     const float sl2 = p.scale_log2;
+    const uint32_t o_col = NQ == 2 ? (uint32_t)(t * 256 + 128) : 256u;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      const int sbuf = j & 1;
-      bool w = mbar_wait(smem_u32(&bars.s_full[sbuf]), (j >> 1) & 1, abort_flag);
+      const int sbuf = NQ == 2 ? t : (j & 1);
+      const uint32_t s_col = NQ == 2 ? (uint32_t)(t * 256) : (uint32_t)(sbuf * 128);
+      const uint32_t par = NQ == 2 ? (uint32_t)(j & 1) : (uint32_t)((j >> 1) & 1);
+      bool w = mbar_wait(smem_u32(&bars.s_full[sbuf]), par, abort_flag);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[128];
-      tmem_ld32(lane_base + sbuf * 128u + 0u, sr);
-      tmem_ld32(lane_base + sbuf * 128u + 32u, sr + 32);
-      tmem_ld32(lane_base + sbuf * 128u + 64u, sr + 64);
-      tmem_ld32(lane_base + sbuf * 128u + 96u, sr + 96);
+      tmem_ld32(tmem + lane_off + s_col + 0u, sr);
+      tmem_ld32(tmem + lane_off + s_col + 32u, sr + 32);
+      tmem_ld32(tmem + lane_off + s_col + 64u, sr + 64);
+      tmem_ld32(tmem + lane_off + s_col + 96u, sr + 96);
       tc_wait_ld();
-      tc_fence_before();
-      mbar_arrive(smem_u32(&bars.s_free[sbuf]));
 
-      // masks: each half of the tile is one 64-key block
+      // masks: each half of the tile is one 64-key block; 0 = none, 1 = all, 2 = partial
+      int state[2];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const int e = 2 * j + half;
         int kb;
         bool att;
-        if (p.sparse) {
+        if (NQ == 1 && p.sparse) {
           att = e < n_list && (list[e].y & rowbit);
           kb = e < n_list ? list[e].x : 0;
         } else {
@@ -295,79 +424,95 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
           kb = kb_lo + e;
         }
         const int key0 = kb * RTP_BLOCK;
-        if (!att) {
+        const bool sparse_row = NQ == 1 && p.sparse;
+        const bool none = !att || key0 > pos || (!sparse_row && key0 + 63 <= pos - p.window_tokens) ||
+                          key0 >= p.Nk;
+        const bool full = !none && key0 + 63 <= pos && (sparse_row || key0 > pos - p.window_tokens) &&
+                          key0 + 63 < p.Nk;
+        state[half] = none ? 0 : (full ? 1 : 2);
+        if (state[half] == 2) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) sr[half * 64 + c] = __float_as_uint(-INFINITY);
-        } else {
-          const bool full = (key0 + 63 <= pos) && (p.sparse || key0 > pos - p.window_tokens) &&
-                            (key0 + 63 < p.Nk);
-          if (!full) {
-#pragma unroll
-            for (int c = 0; c < 64; ++c) {
-              const int u = key0 + c;
-              const bool okk = u <= pos && (p.sparse || u > pos - p.window_tokens) && u < p.Nk;
-              if (!okk) sr[half * 64 + c] = __float_as_uint(-INFINITY);
-            }
+          for (int c = 0; c < 64; ++c) {
+            const int u = key0 + c;
+            const bool okk = u <= pos && (sparse_row || u > pos - p.window_tokens) && u < p.Nk;
+            if (!okk) sr[half * 64 + c] = __float_as_uint(-INFINITY);
           }
         }
       }
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+      for (int half = 0; half < 2; ++half) {
+        if (state[half] == 0) continue;
+        float a = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; c += 2)
+          a = max3f(a, __uint_as_float(sr[half * 64 + c]), __uint_as_float(sr[half * 64 + c + 1]));
+        mx = fmaxf(mx, a);
+      }
       const float m_cand = mx * sl2;
       const bool need = m_cand > m_run + 8.f;
-      bool pv_waited = false;
-      if (__any_sync(0xffffffffu, need && j > 0 && m_run != -INFINITY)) {
-        w = mbar_wait(smem_u32(&bars.pv_done), (j - 1) & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-        pv_waited = true;
-        tc_fence_after();
-        const float f = (need && m_run != -INFINITY) ? ex2(m_run - m_cand) : 1.f;
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + kOCol + c4 * 32u, o);
-          tc_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
-          tmem_st32(lane_base + kOCol + c4 * 32u, o);
-        }
-        tc_wait_st();
-      }
+      const bool rescale_o = __any_sync(0xffffffffu, need && j > 0 && m_run != -INFINITY);
+      const float o_factor = (need && m_run != -INFINITY) ? ex2(m_run - m_cand) : 1.f;
       if (need) {
         l_run *= ex2(m_run - m_cand);
         m_run = m_cand;
       }
       const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      float sum = 0.f;
-      uint32_t pk[64];
+      const uint64_t sc2 = f2(sl2, sl2), nb2 = f2(-base, -base);
+      uint64_t sum2 = f2(0.f, 0.f);
+      // P (bf16 pairs) of each 64-key half goes over columns [32 half, 32 half + 32)
+      // of this tile's S: the first half of S is already in registers.
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), sl2, -base));
-        const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -base));
-        sum += p0 + p1;
-        pk[c] = pack_bf16x2(p0, p1);
-      }
-      l_run += sum;
-      if (j > 0 && !pv_waited) {
-        w = mbar_wait(smem_u32(&bars.pv_done), (j - 1) & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-      }
-      // P row r into the 128-byte-swizzled K-major tile (two 64-key chunks).
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+        if (state[half] == 0) {
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch)
+          for (int c = 0; c < 32; ++c) pk[c] = 0u;
+        } else {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint32_t addr = sb + kPOff + ch * 16384u + (uint32_t)r * 128u + (uint32_t)((u ^ (r & 7)) * 16);
-          st_shared_v4(addr, pk[ch * 32 + u * 4], pk[ch * 32 + u * 4 + 1], pk[ch * 32 + u * 4 + 2],
-                       pk[ch * 32 + u * 4 + 3]);
+          for (int c = 0; c < 32; ++c) {
+            const int e = half * 64 + 2 * c;
+            const uint64_t x = f2_fma(f2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), sc2, nb2);
+            float x0, x1, p0, p1;
+            f2_split(x, x0, x1);
+            if ((c & 3) == 3 && state[half] == 1) {
+              exp2_poly2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            sum2 = f2_add(sum2, f2(p0, p1));
+            pk[c] = pack_bf16x2(p0, p1);
+          }
         }
-      fence_proxy_async_smem();
+        tmem_st32(tmem + lane_off + s_col + half * 32u, pk);
+      }
+      float s0, s1;
+      f2_split(sum2, s0, s1);
+      l_run += s0 + s1;
+      if (rescale_o) {
+        // the running max grew by more than 8: rescale O in TMEM before PV(j)
+        if (NQ == 1) {
+          w = mbar_wait(smem_u32(&bars.pv_done), (j - 1) & 1, abort_flag);   // PV(j-1) must be done
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_off + o_col + c4 * 32u, o);
+          tc_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * o_factor);
+          tmem_st32(tmem + lane_off + o_col + c4 * 32u, o);
+        }
+      }
+      tc_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&bars.p_full));
+      mbar_arrive(smem_u32(&bars.p_full[sbuf]));
     }
     if (ok) {
-      bool w = mbar_wait(smem_u32(&bars.pv_done), (n_tiles - 1) & 1, abort_flag);
+      bool w = mbar_wait(smem_u32(&bars.fin), 0, abort_flag);
       if (__all_sync(0xffffffffu, w)) {
         tc_fence_after();
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
@@ -376,7 +521,7 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
           uint32_t o[32];
-          tmem_ld32(lane_base + kOCol + c4 * 32u, o);
+          tmem_ld32(tmem + lane_off + o_col + c4 * 32u, o);
           tc_wait_ld();
           if (row < p.Nq) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
@@ -406,17 +551,27 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
 }
 
 size_t prefill_attn_tc_smem_bytes(const PrefillAttnParams& p) {
-  return 1024 + kListOff + (size_t)p.list_cap * sizeof(int2) + sizeof(Bars);
+  const uint32_t list_off = p.sparse ? Layout<1>::kListOff : Layout<2>::kListOff;
+  return 1024 + list_off + (size_t)p.list_cap * sizeof(int2) + sizeof(Bars);
 }
 
 cudaError_t launch_prefill_attn_tc(const PrefillAttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                                    const CUtensorMap& tmV, int n_tiles, int B, int* status, cudaStream_t stream) {
   const size_t smem = prefill_attn_tc_smem_bytes(p);
-  cudaError_t e = cudaFuncSetAttribute(prefill_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(n_tiles, p.n_heads, B);
-  prefill_attn_tc_kernel<<<grid, kThreads, smem, stream>>>(p, tmQ, tmK, tmV, status);
+  (void)n_tiles;
+  if (p.sparse) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_attn_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((p.Nq + 127) / 128, p.n_heads, B);
+    prefill_attn_tc_kernel<1><<<grid, Layout<1>::kThreads, smem, stream>>>(p, tmQ, tmK, tmV, status);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(prefill_attn_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((p.Nq + 255) / 256, p.n_heads, B);
+    prefill_attn_tc_kernel<2><<<grid, Layout<2>::kThreads, smem, stream>>>(p, tmQ, tmK, tmV, status);
+  }
   return cudaGetLastError();
 }
 

@@ -74,24 +74,18 @@ struct TopkSmem {
   int digit, above;
 };
 
-// Block-wide exact top-k by (key desc, index asc) over n elements whose keys
-// come from get_key(i). Writes the selected indices in ascending order to
-// out[0 .. min(k,n)), pads out[min(k,n) .. k) with -1. Radix select over the
-// 32-bit key in three digit passes (11, 11, 10 bits), then an ordered
-// compaction that takes every key above the threshold and the lowest-index
-// keys equal to it.
+// Block-wide radix search for the k-th largest 32-bit key among n elements
+// (keys from get_key(i)), digits of 11, 11 and 10 bits from the top. Starting
+// at `first_pass` with the bits of `prefix` under `mask` already fixed (the
+// elements considered are those matching it), and `need` the number still to
+// take from them. Returns the threshold key; on return `need` is how many
+// elements equal to it are taken (the others above it are all taken).
 template <int NT, class GetKey>
-__device__ void block_topk_ascending(GetKey get_key, int n, int k, int32_t* __restrict__ out,
-                                     TopkSmem<NT>& sm) {
+__device__ uint32_t block_radix_threshold(GetKey get_key, int n, int& need, TopkSmem<NT>& sm,
+                                          int first_pass = 0, uint32_t prefix = 0, uint32_t mask = 0) {
   const int tid = threadIdx.x;
-  if (n <= k) {
-    for (int i = tid; i < k; i += NT) out[i] = (i < n) ? i : -1;
-    return;
-  }
-  uint32_t prefix = 0, mask = 0;
-  int need = k;
 #pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
+  for (int pass = first_pass; pass < 3; ++pass) {
     const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
     const int nbins = pass == 2 ? 1024 : 2048;
     for (int b = tid; b < nbins; b += NT) sm.hist[b] = 0;
@@ -126,8 +120,24 @@ __device__ void block_topk_ascending(GetKey get_key, int n, int k, int32_t* __re
     mask |= (uint32_t)(nbins - 1) << shift;
     __syncthreads();
   }
-  // prefix is now the k-th largest key; `need` keys equal to it are taken.
-  const uint32_t thr = prefix;
+  return prefix;
+}
+
+// Block-wide exact top-k by (key desc, index asc) over n elements whose keys
+// come from get_key(i). Writes the selected indices in ascending order to
+// out[0 .. min(k,n)), pads out[min(k,n) .. k) with -1: a radix search for the
+// k-th key, then an ordered compaction that takes every key above it and the
+// lowest-index keys equal to it.
+template <int NT, class GetKey>
+__device__ void block_topk_ascending(GetKey get_key, int n, int k, int32_t* __restrict__ out,
+                                     TopkSmem<NT>& sm) {
+  const int tid = threadIdx.x;
+  if (n <= k) {
+    for (int i = tid; i < k; i += NT) out[i] = (i < n) ? i : -1;
+    return;
+  }
+  int need = k;
+  const uint32_t thr = block_radix_threshold<NT>(get_key, n, need, sm);
   int eq_seen = 0, written = 0;
   for (int base = 0; base < n; base += NT) {
     int i = base + tid;
@@ -142,6 +152,22 @@ __device__ void block_topk_ascending(GetKey get_key, int n, int k, int32_t* __re
     written += take_tot;
     eq_seen += eq_tot;
     if (written >= k) break;
+  }
+}
+
+// Ascending bitonic sort of a[0 .. n) in shared memory, n a power of two.
+template <int NT>
+__device__ void block_bitonic_sort(int* a, int n) {
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < n / 2; i += NT) {
+        const int lo = 2 * stride * (i / stride) + (i % stride), hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const int x = a[lo], y = a[hi];
+        if ((x > y) == up) { a[lo] = y; a[hi] = x; }
+      }
+      __syncthreads();
+    }
   }
 }
 

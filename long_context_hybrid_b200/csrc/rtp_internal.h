@@ -35,6 +35,20 @@ cudaError_t launch_decode_attn(const void* q, int64_t q_sb, int64_t q_sh,
                                const int32_t* idx, int topk, int window, int sink, float scale,
                                void* ws, cudaStream_t stream);
 
+// Retrieval heads (selected tokens + sink + window) and streaming heads
+// (window) of one decode step in one launch; each window K/V row is staged
+// once per KV group.
+constexpr int kMaxSink = 64;
+cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
+                                 const void* kc, int64_t k_sb, int64_t k_sn, int64_t k_sh,
+                                 const void* vc, int64_t v_sb, int64_t v_sn, int64_t v_sh,
+                                 void* o, int64_t o_sb, int64_t o_sh,
+                                 int B, int L, int q_pos, int Hq, int Hkv,
+                                 const int32_t* ret_heads, int n_ret, const int32_t* idx, int topk,
+                                 int ret_window, int sink,
+                                 const int32_t* swa_heads, int n_swa, int swa_window,
+                                 float scale, void* ws, cudaStream_t stream);
+
 // Same as launch_decode_attn for retrieval heads, with the partials in a
 // library-owned static device array of kNoAllocScratchBytes.
 constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;

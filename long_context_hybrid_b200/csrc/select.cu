@@ -1,29 +1,51 @@
-// Indexer selection: decode token top-k and prefill block top-k.
+// Decode token selection: every retrieval head scores every cached token by
+// q~ . k~ (r = 16) and keeps its top-k tokens (the 128K decode workload
+// statement: token-level top-2048 over the whole cache; RTPurbo digest: the
+// 16-d indexer is the scout). Exact ties rank the smaller token first.
 //
-// Decode (the 128K decode workload statement): every retrieval head scores
-// every cached token by q~ . k~ (r = 16) and keeps the top-k tokens. The key
-// index of a KV group is read once for all retrieval heads of that group
-// (grouped-query heads share keys); scores go to the caller's workspace, then
-// one CTA per (sequence, head) runs an exact radix select over them.
-//
-// Prefill (the tiny 2K prefill workload statement): the block score of query
-// block i against key block j is the max of q~_t . k~_u over causal pairs of
-// the two 64-token blocks; each query block keeps its top-k key blocks. The
-// block scores of one query block live in shared memory and never reach HBM.
+// Two kernels:
+//   scan   one pass over the key index; a KV group's index is read once for all
+//          retrieval heads of that group (grouped-query heads share keys). It
+//          writes every score (fp32, to the workspace, sized to stay in L2) and
+//          a histogram of the top 11 bits of each score's order-preserving key.
+//   top-k  one CTA per (sequence, head): from the histogram it knows the bin
+//          holding the k-th score; one pass over the scores takes every score
+//          above that bin and gathers the bin's members as candidates in
+//          shared memory, where a radix search over the remaining bits (and the
+//          token index for exact ties) settles the rest; the list is then
+//          sorted ascending. If the candidates overflow shared memory the CTA
+//          falls back to a full radix select over the scores.
 #include "rtp_common.cuh"
 #include "rtp_internal.h"
 
 namespace rtp {
 
-// ---------------------------------------------------------------------------
-// Decode
-// ---------------------------------------------------------------------------
+namespace {
 constexpr int kScanThreads = 256;
-constexpr int kScanTokensPerThread = 4;
+constexpr int kScanTokensPerThread = 32;
+constexpr int kScanTokens = kScanThreads * kScanTokensPerThread;   // 8192 per CTA
+constexpr int kBins = 2048;                                        // top 11 bits
+constexpr int kTopkThreads = 1024;
+constexpr int kCandCap = 12288;
+constexpr int kMaxTopk = 4096;
+
+struct DecodeTopkSmem {
+  TopkSmem<kTopkThreads> tk;
+  uint32_t cand_key[kCandCap];
+  int cand_idx[kCandCap];
+  int sel[kMaxTopk];
+  int n_sel, n_cand, n_eq;
+};
+
+size_t hist_offset(int B, int L, int Hr) {
+  return (((size_t)B * Hr * L * sizeof(float)) + 255) & ~(size_t)255;
+}
+}  // namespace
 
 __global__ void __launch_bounds__(kScanThreads)
-decode_scan_kernel(const float* __restrict__ qt, const uint4* __restrict__ kindex, int L, int Hr,
-                   int Hkv, const HeadList hl, float* __restrict__ scores) {
+decode_scan_kernel(const float* __restrict__ qt, const uint4* __restrict__ kindex, int L, int Hr, int Hkv,
+                   const HeadList hl, float* __restrict__ scores, uint32_t* __restrict__ ghist) {
+  extern __shared__ uint32_t shist[];                  // [n_j][kBins]
   const int b = blockIdx.z, g = blockIdx.y;
   __shared__ float qs[kMaxHeads][RTP_R];
   __shared__ int js[kMaxHeads];
@@ -37,162 +59,154 @@ decode_scan_kernel(const float* __restrict__ qt, const uint4* __restrict__ kinde
   __syncthreads();
   const int n = nj;
   if (n == 0) return;
-  for (int e = threadIdx.x; e < n * RTP_R; e += blockDim.x)
+  for (int e = threadIdx.x; e < n * RTP_R; e += kScanThreads)
     qs[e / RTP_R][e % RTP_R] = qt[((size_t)b * Hr + js[e / RTP_R]) * RTP_R + e % RTP_R];
+  for (int e = threadIdx.x; e < n * kBins; e += kScanThreads) shist[e] = 0u;
   __syncthreads();
   const uint4* krow = kindex + ((size_t)b * Hkv + g) * (size_t)L * 2;
-  const int base = blockIdx.x * kScanThreads * kScanTokensPerThread;
-#pragma unroll
+  const int base = blockIdx.x * kScanTokens;
+#pragma unroll 4
   for (int s = 0; s < kScanTokensPerThread; ++s) {
     const int u = base + s * kScanThreads + threadIdx.x;
     if (u >= L) break;
     const uint4 lo = __ldg(krow + (size_t)u * 2), hi = __ldg(krow + (size_t)u * 2 + 1);
-    float k[16] = {bf16_lo(lo.x), bf16_hi(lo.x), bf16_lo(lo.y), bf16_hi(lo.y),
-                   bf16_lo(lo.z), bf16_hi(lo.z), bf16_lo(lo.w), bf16_hi(lo.w),
-                   bf16_lo(hi.x), bf16_hi(hi.x), bf16_lo(hi.y), bf16_hi(hi.y),
-                   bf16_lo(hi.z), bf16_hi(hi.z), bf16_lo(hi.w), bf16_hi(hi.w)};
+    const float k[16] = {bf16_lo(lo.x), bf16_hi(lo.x), bf16_lo(lo.y), bf16_hi(lo.y),
+                         bf16_lo(lo.z), bf16_hi(lo.z), bf16_lo(lo.w), bf16_hi(lo.w),
+                         bf16_lo(hi.x), bf16_hi(hi.x), bf16_lo(hi.y), bf16_hi(hi.y),
+                         bf16_lo(hi.z), bf16_hi(hi.z), bf16_lo(hi.w), bf16_hi(hi.w)};
     for (int jj = 0; jj < n; ++jj) {
       float acc = 0.f;
 #pragma unroll
       for (int c = 0; c < RTP_R; ++c) acc = fmaf(qs[jj][c], k[c], acc);
       scores[((size_t)b * Hr + js[jj]) * L + u] = acc;
+      atomicAdd(&shist[jj * kBins + (f2key(acc) >> 21)], 1u);
     }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n * kBins; e += kScanThreads) {
+    const uint32_t c = shist[e];
+    if (c) atomicAdd(&ghist[((size_t)b * Hr + js[e / kBins]) * kBins + (e % kBins)], c);
   }
 }
 
-constexpr int kSelThreads = 1024;
-
-__global__ void __launch_bounds__(kSelThreads)
-decode_topk_kernel(const float* __restrict__ scores, int L, int Hr, int topk, int32_t* __restrict__ idx) {
-  __shared__ TopkSmem<kSelThreads> sm;
-  const int j = blockIdx.x, b = blockIdx.y;
+__global__ void __launch_bounds__(kTopkThreads)
+decode_topk_kernel(const float* __restrict__ scores, const uint32_t* __restrict__ ghist, int L, int Hr, int topk,
+                   int32_t* __restrict__ idx) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  DecodeTopkSmem& sm = *reinterpret_cast<DecodeTopkSmem*>(smem_raw);
+  const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const float* s = scores + ((size_t)b * Hr + j) * L;
-  auto get_key = [s](int i) { return f2key(__ldg(s + i)); };
-  block_topk_ascending<kSelThreads>(get_key, L, topk, idx + ((size_t)b * Hr + j) * topk, sm);
+  int32_t* out = idx + ((size_t)b * Hr + j) * topk;
+  auto key_of = [s](int i) { return f2key(__ldg(s + i)); };
+  if (L <= topk) {
+    for (int i = tid; i < topk; i += kTopkThreads) out[i] = (i < L) ? i : -1;
+    return;
+  }
+  // 1. bin of the k-th score from the scan's histogram
+  const uint32_t* h = ghist + ((size_t)b * Hr + j) * kBins;
+  for (int x = tid; x < kBins; x += kTopkThreads) sm.tk.hist[x] = h[x];
+  if (tid == 0) { sm.n_sel = 0; sm.n_cand = 0; sm.n_eq = 0; }
+  __syncthreads();
+  constexpr int per = kBins / kTopkThreads;
+  int local = 0;
+  for (int q = 0; q < per; ++q) local += sm.tk.hist[kBins - 1 - (tid * per + q)];
+  int tot;
+  const int above_t = block_exclusive_scan<kTopkThreads>(local, tot, sm.tk.scan);
+  if (above_t < topk && above_t + local >= topk) {
+    int run = above_t;
+    for (int q = 0; q < per; ++q) {
+      const int bin = kBins - 1 - (tid * per + q);
+      const int c = sm.tk.hist[bin];
+      if (run + c >= topk) { sm.tk.digit = bin; sm.tk.above = run; break; }
+      run += c;
+    }
+  }
+  __syncthreads();
+  const uint32_t d1 = (uint32_t)sm.tk.digit;
+  const int above = sm.tk.above;
+  // 2. one pass: take keys above the bin, gather the bin's members
+  for (int i = tid; i < L; i += kTopkThreads) {
+    const uint32_t key = key_of(i);
+    const uint32_t d = key >> 21;
+    if (d > d1) {
+      sm.sel[atomicAdd(&sm.n_sel, 1)] = i;
+    } else if (d == d1) {
+      const int pos = atomicAdd(&sm.n_cand, 1);
+      if (pos < kCandCap) { sm.cand_key[pos] = key; sm.cand_idx[pos] = i; }
+    }
+  }
+  __syncthreads();
+  const int n_cand = sm.n_cand;
+  if (n_cand > kCandCap || sm.n_sel != above) {
+    // candidates do not fit: exact radix select over all scores instead
+    block_topk_ascending<kTopkThreads>(key_of, L, topk, out, sm.tk);
+    return;
+  }
+  // 3. settle the bin: radix search over its remaining bits, then the lowest
+  //    token indices among keys equal to the threshold
+  int need = topk - above;
+  const uint32_t* ck = sm.cand_key;
+  auto cand_key = [ck](int x) { return ck[x]; };
+  const uint32_t thr = block_radix_threshold<kTopkThreads>(cand_key, n_cand, need, sm.tk, 1, d1 << 21,
+                                                            0x7FFu << 21);
+  for (int x = tid; x < n_cand; x += kTopkThreads)
+    if (sm.cand_key[x] > thr) sm.sel[atomicAdd(&sm.n_sel, 1)] = sm.cand_idx[x];
+  __syncthreads();
+  // equal keys: each takes its rank among the equal ones by token index
+  for (int x = tid; x < n_cand; x += kTopkThreads) {
+    if (sm.cand_key[x] != thr) continue;
+    const int me = sm.cand_idx[x];
+    int rank = 0;
+    for (int y = 0; y < n_cand; ++y)
+      if (sm.cand_key[y] == thr && sm.cand_idx[y] < me) ++rank;
+    if (rank < need) sm.sel[atomicAdd(&sm.n_sel, 1)] = me;
+  }
+  __syncthreads();
+  // 4. ascending order
+  int n_pow2 = 1;
+  while (n_pow2 < topk) n_pow2 <<= 1;
+  for (int x = topk + tid; x < n_pow2; x += kTopkThreads) sm.sel[x] = 0x7fffffff;
+  __syncthreads();
+  block_bitonic_sort<kTopkThreads>(sm.sel, n_pow2);
+  for (int x = tid; x < topk; x += kTopkThreads) out[x] = sm.sel[x];
 }
 
 size_t select_decode_ws_bytes(int B, int L, int Hr, int topk) {
   (void)topk;
-  return (size_t)B * Hr * L * sizeof(float);
+  return hist_offset(B, L, Hr) + (size_t)B * Hr * kBins * sizeof(uint32_t);
 }
 
-static void fill_heads(HeadList& hl, const int32_t* kv_of, int Hr) {
-  hl.n = Hr;
-  for (int j = 0; j < Hr; ++j) { hl.head[j] = j; hl.kv[j] = kv_of[j]; }
-}
-
-cudaError_t launch_select_decode(const float* qt, const void* kindex, int B, int L, int Hr,
-                                 int Hkv, const int32_t* kv_of, int topk, int32_t* idx,
-                                 void* ws, cudaStream_t stream) {
+cudaError_t launch_select_decode(const float* qt, const void* kindex, int B, int L, int Hr, int Hkv,
+                                 const int32_t* kv_of, int topk, int32_t* idx, void* ws, cudaStream_t stream) {
+  if (topk > kMaxTopk) return cudaErrorInvalidValue;
   HeadList hl;
-  fill_heads(hl, kv_of, Hr);
+  hl.n = Hr;
+  int max_nj = 0;
+  for (int g = 0; g < Hkv; ++g) {
+    int c = 0;
+    for (int j = 0; j < Hr; ++j) c += (kv_of[j] == g);
+    max_nj = c > max_nj ? c : max_nj;
+  }
+  for (int j = 0; j < Hr; ++j) { hl.head[j] = j; hl.kv[j] = kv_of[j]; }
   float* scores = static_cast<float*>(ws);
-  dim3 g1((L + kScanThreads * kScanTokensPerThread - 1) / (kScanThreads * kScanTokensPerThread), Hkv, B);
-  decode_scan_kernel<<<g1, kScanThreads, 0, stream>>>(qt, static_cast<const uint4*>(kindex), L, Hr,
-                                                      Hkv, hl, scores);
-  cudaError_t e = cudaGetLastError();
+  uint32_t* ghist = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + hist_offset(B, L, Hr));
+  cudaError_t e = cudaMemsetAsync(ghist, 0, (size_t)B * Hr * kBins * sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return e;
+  const size_t scan_smem = (size_t)max_nj * kBins * sizeof(uint32_t);
+  if (scan_smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(decode_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 g1((L + kScanTokens - 1) / kScanTokens, Hkv, B);
+  decode_scan_kernel<<<g1, kScanThreads, scan_smem, stream>>>(qt, static_cast<const uint4*>(kindex), L, Hr, Hkv,
+                                                              hl, scores, ghist);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t topk_smem = sizeof(DecodeTopkSmem);
+  e = cudaFuncSetAttribute(decode_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)topk_smem);
   if (e != cudaSuccess) return e;
   dim3 g2(Hr, B);
-  decode_topk_kernel<<<g2, kSelThreads, 0, stream>>>(scores, L, Hr, topk, idx);
-  return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
-// Prefill
-// ---------------------------------------------------------------------------
-constexpr int kPSelThreads = 256;
-
-struct PrefillSelectSmem {
-  float q[RTP_BLOCK][RTP_R];
-  float part[kPSelThreads / 32];
-  TopkSmem<kPSelThreads> topk;
-};
-
-__global__ void __launch_bounds__(kPSelThreads)
-prefill_select_kernel(const uint4* __restrict__ qt, const uint4* __restrict__ kt, int N, int Hr,
-                      int Hkv, const HeadList hl, int topk, int32_t* __restrict__ blocks,
-                      int32_t* __restrict__ counts) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  PrefillSelectSmem& sm = *reinterpret_cast<PrefillSelectSmem*>(smem_raw);
-  float* s = reinterpret_cast<float*>(smem_raw + sizeof(PrefillSelectSmem));
-  const int nb = N / RTP_BLOCK;
-  const int i = nb - 1 - blockIdx.x;          // longest lists first
-  const int j = blockIdx.y, b = blockIdx.z;
-  const int g = hl.kv[j];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-  const uint4* qrow = qt + (((size_t)b * Hr + j) * N + (size_t)i * RTP_BLOCK) * 2;
-  for (int e = tid; e < RTP_BLOCK * 2; e += kPSelThreads) {
-    uint4 w = __ldg(qrow + e);
-    float* d = &sm.q[e >> 1][(e & 1) * 8];
-    d[0] = bf16_lo(w.x); d[1] = bf16_hi(w.x); d[2] = bf16_lo(w.y); d[3] = bf16_hi(w.y);
-    d[4] = bf16_lo(w.z); d[5] = bf16_hi(w.z); d[6] = bf16_lo(w.w); d[7] = bf16_hi(w.w);
-  }
-  __syncthreads();
-  const uint4* krows = kt + ((size_t)b * Hkv + g) * (size_t)N * 2;
-  const int keys_per_iter = kPSelThreads;                 // 4 key blocks per iteration
-  const int n_keys = (i + 1) * RTP_BLOCK;
-  for (int u0 = 0; u0 < n_keys; u0 += keys_per_iter) {
-    const int u = u0 + tid;
-    float best = -INFINITY;
-    if (u < n_keys) {
-      const uint4 lo = __ldg(krows + (size_t)u * 2), hi = __ldg(krows + (size_t)u * 2 + 1);
-      const float k[16] = {bf16_lo(lo.x), bf16_hi(lo.x), bf16_lo(lo.y), bf16_hi(lo.y),
-                           bf16_lo(lo.z), bf16_hi(lo.z), bf16_lo(lo.w), bf16_hi(lo.w),
-                           bf16_lo(hi.x), bf16_hi(hi.x), bf16_lo(hi.y), bf16_hi(hi.y),
-                           bf16_lo(hi.z), bf16_hi(hi.z), bf16_lo(hi.w), bf16_hi(hi.w)};
-      // Causal pairs only: query t = 64 i + r needs u <= t.
-      const int r0 = (u >= i * RTP_BLOCK) ? (u - i * RTP_BLOCK) : 0;
-      for (int r = r0; r < RTP_BLOCK; ++r) {
-        float acc = 0.f;
-#pragma unroll
-        for (int c = 0; c < RTP_R; ++c) acc = fmaf(sm.q[r][c], k[c], acc);
-        best = fmaxf(best, acc);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
-    if (lane == 0) sm.part[warp] = best;
-    __syncthreads();
-    if (tid < kPSelThreads / 64) {
-      const int jb = u0 / RTP_BLOCK + tid;
-      if (jb <= i) s[jb] = fmaxf(sm.part[2 * tid], sm.part[2 * tid + 1]);
-    }
-    __syncthreads();
-  }
-  int32_t* out = blocks + (((size_t)b * Hr + j) * nb + i) * topk;
-  auto get_key = [s](int x) { return f2key(s[x]); };
-  block_topk_ascending<kPSelThreads>(get_key, i + 1, topk, out, sm.topk);
-  if (tid == 0) counts[((size_t)b * Hr + j) * nb + i] = min(topk, i + 1);
-}
-
-size_t select_prefill_ws_bytes(int B, int N, int Hr, int topk) {
-  (void)B; (void)N; (void)Hr; (void)topk;
-  return kStatusBytes;
-}
-
-cudaError_t launch_select_prefill(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
-                                  const int32_t* kv_of, int topk, int32_t* blocks,
-                                  int32_t* counts, void* ws, cudaStream_t stream) {
-  return launch_select_prefill_tc(qt, kt, B, N, Hr, Hkv, kv_of, topk, blocks, counts,
-                                  static_cast<int*>(ws), stream);
-}
-
-cudaError_t launch_select_prefill_simt(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
-                                       const int32_t* kv_of, int topk, int32_t* blocks,
-                                       int32_t* counts, cudaStream_t stream) {
-  HeadList hl;
-  fill_heads(hl, kv_of, Hr);
-  const int nb = N / RTP_BLOCK;
-  const size_t smem = sizeof(PrefillSelectSmem) + (size_t)nb * sizeof(float);
-  if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(prefill_select_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(nb, Hr, B);
-  prefill_select_kernel<<<grid, kPSelThreads, smem, stream>>>(
-      static_cast<const uint4*>(qt), static_cast<const uint4*>(kt), N, Hr, Hkv, hl, topk, blocks,
-      counts);
+  decode_topk_kernel<<<g2, kTopkThreads, topk_smem, stream>>>(scores, ghist, L, Hr, topk, idx);
   return cudaGetLastError();
 }
 

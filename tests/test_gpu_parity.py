@@ -344,3 +344,38 @@ def test_e2e_decode_reduced():
             outs.append(_f64(o[b, h].cpu()))
             refs.append(res["out"][h])
     assert_attn_close(np.stack(outs), np.stack(refs), "decode")
+
+
+@pytest.mark.parametrize("L,ret_window,swa_window,topk", [(6000, 512, 256, 300), (6000, 256, 1024, 129),
+                                                          (700, 4096, 4096, 100), (20000, 8192, 8192, 2048)])
+def test_decode_attn_hybrid_matches_oracle(L, ret_window, swa_window, topk):
+    """Retrieval and streaming heads in one launch, windows of different sizes."""
+    B, Hq, Hkv = 2, 16, 2
+    q = _clustered_bf16((B, Hq, 128), 90)
+    kc, vc = _clustered_bf16((B, L, Hkv, 128), 91), _randn_bf16((B, L, Hkv, 128), 92)
+    ret = [0, 3, 9]
+    swa_heads = [h for h in range(Hq) if h not in ret]
+    rs = np.random.default_rng(L + topk)
+    idx = -np.ones((B, len(ret), topk), np.int32)
+    for b in range(B):
+        for j in range(len(ret)):
+            n = min(topk, L)
+            idx[b, j, :n] = np.sort(rs.choice(L, n, replace=False))
+    o = torch.zeros(B, Hq, 128, dtype=torch.bfloat16, device=DEV)
+    rtp.decode_attn_hybrid(q.to(DEV), kc.to(DEV), vc.to(DEV), o, ret, torch.from_numpy(idx).to(DEV), ret_window,
+                           swa_heads, swa_window, sink=1)
+    torch.cuda.synchronize()
+    o = o.cpu()
+    scale = 1 / math.sqrt(128)
+    outs, refs = [], []
+    for b in range(B):
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            if h in ret:
+                sel = idx[b, ret.index(h)]
+                att = O.decode_attended(sel[sel >= 0], L, ret_window, 1)
+            else:
+                att = np.arange(max(0, L - swa_window), L)
+            outs.append(_f64(o[b, h]))
+            refs.append(O.attend_decode(q[b, h], kc[b, :, g], vc[b, :, g], att, scale))
+    assert_attn_close(np.stack(outs), np.stack(refs), "hybrid decode")

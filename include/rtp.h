@@ -93,6 +93,18 @@ RTP_API int rtp_version(void);
 RTP_API rtp_status rtp_workspace_status(const void* ws, rtp_stream_t stream);
 
 /*
+ * rtp_debug_prefill_timeout_probe - test hook for the bounded waits.
+ *   Launches one CTA of the prefill attention kernel on a 128-token, one-head
+ *   sliding-window problem whose producer deliberately never loads Q, so the
+ *   CTA's waits run out (about 2 s), it drains its copies, frees its tensor
+ *   memory and records RTP_ERR_TIMEOUT in the status word of `ws` (read it
+ *   with rtp_workspace_status). q, k, v, o: bf16 [1, 128, 1, 128] device
+ *   buffers (o is not written). The device stays usable afterwards.
+ */
+RTP_API rtp_status rtp_debug_prefill_timeout_probe(const void* q, const void* k, const void* v, void* o, void* ws,
+                                                   size_t ws_bytes, rtp_stream_t stream);
+
+/*
  * rtp_index_project - the low-rank indexer projection x~ = x . P.
  *   Source: RTPurboV2 article, paragraph on the low-rank projector (feature
  *   dimension compressed from D to r = 16); the precomputed 16-d key index
@@ -207,8 +219,9 @@ RTP_API rtp_status rtp_sparse_attn_prefill(const void* q, rtp_strides qs, const 
  *            token indices, -1 padded, as written by rtp_select_decode
  *            (entries in the window or below `sink` are skipped there,
  *            since those keys are attended anyway).
- *   window >= 1, 0 <= sink <= 64, scale > 0; Hq / Hkv <= 16 (the query heads
- *   of a KV group are packed into one 16-row tensor-core tile).
+ *   window >= 1, 0 <= sink <= 64, scale > 0; Hq / Hkv <= 16 and Hkv <= 16
+ *   (the query heads of a KV group are packed into one 16-row tensor-core
+ *   tile).
  */
 RTP_API size_t rtp_workspace_size_sparse_attn_decode(int B, int L, int Hq, int Hr, int topk, int window);
 RTP_API rtp_status rtp_sparse_attn_decode(const void* q, const void* kc, rtp_strides ks,
@@ -226,7 +239,7 @@ RTP_API rtp_status rtp_sparse_attn_decode(const void* q, const void* kc, rtp_str
  *   Sources: RTPurboV2 article (streaming heads SWA, retrieval heads sparse);
  *   the 128K decode workload statement.
  *   Arguments as in the two calls it combines; Hr or n_swa may be 0 (not
- *   both); sink <= 64; Hq / Hkv <= 16. ws: rtp_workspace_size_decode_attn_hybrid(
+ *   both); sink <= 64; Hq / Hkv <= 16, Hkv <= 16. ws: rtp_workspace_size_decode_attn_hybrid(
  *   B, L, Hq, topk, max(ret_window, swa_window)) bytes.
  */
 RTP_API size_t rtp_workspace_size_decode_attn_hybrid(int B, int L, int Hq, int topk, int window);

@@ -194,7 +194,7 @@ rtp_status rtp_sparse_attn_decode(const void* q, const void* kc, rtp_strides ks,
   if (!q || !kc || !vc || !o || !idx) return RTP_ERR_INVALID_ARG;
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || topk < 1) return RTP_ERR_INVALID_ARG;
   if (window < 1 || sink < 0 || sink > kMaxSink || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
-  if (Hq / Hkv > 16) return RTP_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 16 || Hkv > 16) return RTP_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(o) || !aligned16(idx)) return RTP_ERR_INVALID_ARG;
   if (!stride_ok(ks) || !stride_ok(vs)) return RTP_ERR_INVALID_ARG;
   rtp_status st = check_heads(heads, Hr, Hq);
@@ -216,7 +216,7 @@ rtp_status rtp_sparse_attn_decode_noalloc(const void* q, const void* kc, rtp_str
   if (!q || !kc || !vc || !o || !idx) return RTP_ERR_INVALID_ARG;
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || topk < 1) return RTP_ERR_INVALID_ARG;
   if (window < 1 || sink < 0 || sink > kMaxSink || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
-  if (Hq / Hkv > 16) return RTP_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 16 || Hkv > 16) return RTP_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(o) || !aligned16(idx)) return RTP_ERR_INVALID_ARG;
   if (!stride_ok(ks) || !stride_ok(vs)) return RTP_ERR_INVALID_ARG;
   rtp_status st = check_heads(heads, Hr, Hq);
@@ -242,7 +242,7 @@ rtp_status rtp_decode_attn_hybrid(const void* q, const void* kc, rtp_strides ks,
   if (!q || !kc || !vc || !o) return RTP_ERR_INVALID_ARG;
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return RTP_ERR_INVALID_ARG;
   if (Hr < 0 || n_swa < 0 || Hr + n_swa < 1 || Hr + n_swa > kMaxHeads) return RTP_ERR_INVALID_ARG;
-  if (Hq / Hkv > 16) return RTP_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 16 || Hkv > 16) return RTP_ERR_UNSUPPORTED;
   if (Hr > 0 && (!idx || topk < 1 || ret_window < 1 || !aligned16(idx))) return RTP_ERR_INVALID_ARG;
   if (n_swa > 0 && swa_window < 1) return RTP_ERR_INVALID_ARG;
   if (sink < 0 || sink > kMaxSink || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
@@ -261,6 +261,25 @@ rtp_status rtp_decode_attn_hybrid(const void* q, const void* kc, rtp_strides ks,
                                         o, (int64_t)Hq * RTP_D, RTP_D, B, L, L - 1, Hq, Hkv, ret_heads, Hr, idx, topk,
                                         ret_window, sink, swa_heads, n_swa, swa_window, scale, ws,
                                         (cudaStream_t)stream));
+}
+
+rtp_status rtp_debug_prefill_timeout_probe(const void* q, const void* k, const void* v, void* o, void* ws,
+                                           size_t ws_bytes, rtp_stream_t stream) {
+  if (!q || !k || !v || !o) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < kStatusBytes || !aligned256(ws)) return RTP_ERR_WORKSPACE;
+  rtp_status st = check_device();
+  if (st != RTP_OK) return st;
+  // One CTA: a 128-row sliding-window problem, one head, whose Q never arrives.
+  PrefillAttnParams p{};
+  p.q = {q, 128 * RTP_D, RTP_D, RTP_D}; p.k = {k, 128 * RTP_D, RTP_D, RTP_D}; p.v = {v, 128 * RTP_D, RTP_D, RTP_D};
+  p.o = o; p.o_sb = 128 * RTP_D; p.o_sn = RTP_D; p.o_sh = RTP_D;
+  p.Nq = 128; p.Nk = 128; p.q_pos0 = 0; p.Hq = 1; p.Hkv = 1; p.G = 1;
+  p.sparse = 0; p.window_tokens = 128;
+  p.scale_log2 = 0.1f;
+  p.n_heads = 1; p.head[0] = 0; p.list_cap = 0;
+  p.withhold_q = 1;
+  return launch_tc(p, 1, ws, (cudaStream_t)stream);
 }
 
 size_t rtp_workspace_size_swa(int B, int Nq, int Nk, int n_heads, int window) {
@@ -282,7 +301,7 @@ rtp_status rtp_swa(const void* q, rtp_strides qs, const void* k, rtp_strides ks,
   rtp_status st = check_heads(heads, n_heads, Hq);
   if (st != RTP_OK) return st;
   if (Nq == 1) {
-    if (Hq / Hkv > 16) return RTP_ERR_UNSUPPORTED;
+    if (Hq / Hkv > 16 || Hkv > 16) return RTP_ERR_UNSUPPORTED;
     const size_t need = decode_attn_ws_bytes(B, Nk, n_heads, 0, window);
     if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
     if ((st = check_device()) != RTP_OK) return st;

@@ -28,6 +28,7 @@ struct PrefillAttnParams {
   int n_heads;
   int bitmap_words;   // words of the block bitmap (sparse)
   int list_cap;       // capacity of the compacted list (sparse)
+  int withhold_q;     // test hook: the producer never loads Q, so every wait must run out
   int head[kMaxHeads];
 };
 

@@ -22,10 +22,10 @@
 //            it reads S, masks, keeps an online softmax in the log2 domain
 //            with lazy rescaling (O is rescaled in TMEM only when the running
 //            max grows by more than 8), computes P with packed f32x2
-//            arithmetic (a quarter of the exponentials on the FMA pipe through
-//            a cubic for 2^f, the rest on MUFU; key halves that are masked for
-//            the whole row skip the exponentials), and writes P as bf16 back
-//            over the first half of S in TMEM, where the next MMA reads it.
+//            arithmetic (key halves that are masked for the whole row skip the
+//            exponentials), and writes P as bf16 back over the first half of S
+//            in TMEM, where the next MMA reads it; each 64-key half is handled
+//            on its own so that a thread holds 64 scores at a time.
 // With NQ = 2 the MMA order QK0 QK1 | PV0 QK0' PV1 QK1' | ... keeps the tensor
 // core busy on one tile while the other tile's softmax runs.
 // Every wait is bounded; a wait that runs out marks the CTA aborted, all roles
@@ -45,11 +45,6 @@ constexpr uint32_t kQTileBytes = 32768;                       // [D half][128 ro
 constexpr uint32_t kStageBytes = 65536;                       // K 32 KB + V 32 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr int kStatusTimeout = 4;
-
-// Cubic for 2^f on [-1/2, 1/2]: Chebyshev-node least squares refined toward
-// minimax by Lawson iterations (max relative error 7.5e-5), derived for this
-// library; far below the 2^-9 rounding that P then takes as bf16.
-constexpr float kP0 = 0.99992806f, kP1 = 0.69326097f, kP2 = 0.24261113f, kP3 = 0.055171665f;
 
 template <int NQ>
 struct Layout {
@@ -95,27 +90,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
-// 2^x for a pair with x <= 8, on the FMA pipe: x = n + f, n = round(x),
-// 2^f from the cubic, 2^n added into the exponent field.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
-  const float magic = 12582912.f;                          // 1.5 * 2^23: round to integer
-  const uint64_t x = f2(x0, x1);
-  const uint64_t j = f2_add(x, f2(magic, magic));
-  const uint64_t n = f2_add(j, f2(-magic, -magic));
-  const uint64_t f = f2_fma(n, f2(-1.f, -1.f), x);
-  uint64_t q = f2_fma(f, f2(kP3, kP3), f2(kP2, kP2));
-  q = f2_fma(q, f, f2(kP1, kP1));
-  q = f2_fma(q, f, f2(kP0, kP0));
-  float q0, q1, j0, j1;
-  f2_split(q, q0, q1);
-  f2_split(j, j0, j1);
-  // bits(j) << 23 carries round(x) into the exponent; the magic's own bits vanish mod 2^32
-  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(j0) << 23));
-  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(j1) << 23));
-}
-
 // Marks the attended key blocks of query block q in `bits`.
 template <int NT>
 __device__ void mark_blocks(const PrefillAttnParams& p, int b, int jh, int q, unsigned* bits) {
@@ -275,11 +249,13 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
       tma_prefetch(&tmK);
       tma_prefetch(&tmV);
       const uint32_t qbar = smem_u32(&bars.q_full);
-      mbar_arrive_expect_tx(qbar, kQTileBytes * NQ);
+      if (!p.withhold_q) {
+        mbar_arrive_expect_tx(qbar, kQTileBytes * NQ);
 #pragma unroll
-      for (int t = 0; t < NQ; ++t) {
-        tma_load_4d(sb + Lay::kQOff + t * kQTileBytes, &tmQ, qbar, 0, h, row0 + t * 128, b);
-        tma_load_4d(sb + Lay::kQOff + t * kQTileBytes + 16384, &tmQ, qbar, 64, h, row0 + t * 128, b);
+        for (int t = 0; t < NQ; ++t) {
+          tma_load_4d(sb + Lay::kQOff + t * kQTileBytes, &tmQ, qbar, 0, h, row0 + t * 128, b);
+          tma_load_4d(sb + Lay::kQOff + t * kQTileBytes + 16384, &tmQ, qbar, 64, h, row0 + t * 128, b);
+        }
       }
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
@@ -309,9 +285,16 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
         }
         issued = j + 1;
       }
+      // The MMA side ends every path by committing `fin`; once it has (or the
+      // CTA has aborted), copies this thread issued but nobody consumed are
+      // waited for, with a short bound, before the CTA exits.
+      {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(smem_u32(&bars.fin), 0) && !*abort_flag && clock64() - t0 < kWaitLimitCycles) {
+        }
+      }
       if (*abort_flag) {
-        // let copies already in flight land before the CTA exits
-        wait_short(qbar, 0);
+        if (!p.withhold_q) wait_short(qbar, 0);
         for (int j = max(0, issued - kStages); j < issued; ++j) {
           wait_short(smem_u32(&bars.k_full[j & 1]), (j >> 1) & 1);
           wait_short(smem_u32(&bars.v_full[j & 1]), (j >> 1) & 1);
@@ -402,15 +385,14 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
       bool w = mbar_wait(smem_u32(&bars.s_full[sbuf]), par, abort_flag);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld32(tmem + lane_off + s_col + 0u, sr);
-      tmem_ld32(tmem + lane_off + s_col + 32u, sr + 32);
-      tmem_ld32(tmem + lane_off + s_col + 64u, sr + 64);
-      tmem_ld32(tmem + lane_off + s_col + 96u, sr + 96);
-      tc_wait_ld();
-
-      // masks: each half of the tile is one 64-key block; 0 = none, 1 = all, 2 = partial
-      int state[2];
+      // Each 64-key half of the tile (one key block): mask state (0 none, 1 all,
+      // 2 partial), a lazy max update, exponentials, and P written as bf16 pairs
+      // over S columns [32 half, 32 half + 32). If the second half raises the
+      // running max by more than 8, the first half's P is rescaled in TMEM.
+      const uint32_t s_addr = tmem + lane_off + s_col;
+      float o_factor = 1.f;
+      bool o_scaled = false;
+      float sum_a = 0.f, sum_b = 0.f;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const int e = 2 * j + half;
@@ -429,81 +411,85 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
                           key0 >= p.Nk;
         const bool full = !none && key0 + 63 <= pos && (sparse_row || key0 > pos - p.window_tokens) &&
                           key0 + 63 < p.Nk;
-        state[half] = none ? 0 : (full ? 1 : 2);
-        if (state[half] == 2) {
+        uint32_t v[64];
+        tmem_ld32(s_addr + half * 64u, v);
+        tmem_ld32(s_addr + half * 64u + 32u, v + 32);
+        tc_wait_ld();
+        if (!none && !full) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
             const int u = key0 + c;
             const bool okk = u <= pos && (sparse_row || u > pos - p.window_tokens) && u < p.Nk;
-            if (!okk) sr[half * 64 + c] = __float_as_uint(-INFINITY);
+            if (!okk) v[c] = __float_as_uint(-INFINITY);
           }
         }
-      }
-      float mx = -INFINITY;
+        float mx = -INFINITY;
+        if (!none) {
+          float a0 = -INFINITY, a1 = -INFINITY;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        if (state[half] == 0) continue;
-        float a = -INFINITY;
+          for (int c = 0; c < 64; c += 4) {
+            a0 = max3f(a0, __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+            a1 = max3f(a1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+          }
+          mx = fmaxf(a0, a1);
+        }
+        const float m_cand = mx * sl2;
+        const bool need = m_cand > m_run + 8.f;
+        if (half == 1 && __any_sync(0xffffffffu, need && m_run != -INFINITY)) {
+          const float f = (need && m_run != -INFINITY) ? ex2(m_run - m_cand) : 1.f;
+          uint32_t w[32];
+          tmem_ld32(s_addr, w);
+          tc_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 64; c += 2)
-          a = max3f(a, __uint_as_float(sr[half * 64 + c]), __uint_as_float(sr[half * 64 + c + 1]));
-        mx = fmaxf(mx, a);
-      }
-      const float m_cand = mx * sl2;
-      const bool need = m_cand > m_run + 8.f;
-      const bool rescale_o = __any_sync(0xffffffffu, need && j > 0 && m_run != -INFINITY);
-      const float o_factor = (need && m_run != -INFINITY) ? ex2(m_run - m_cand) : 1.f;
-      if (need) {
-        l_run *= ex2(m_run - m_cand);
-        m_run = m_cand;
-      }
-      const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      const uint64_t sc2 = f2(sl2, sl2), nb2 = f2(-base, -base);
-      uint64_t sum2 = f2(0.f, 0.f);
-      // P (bf16 pairs) of each 64-key half goes over columns [32 half, 32 half + 32)
-      // of this tile's S: the first half of S is already in registers.
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+          for (int c = 0; c < 32; ++c)
+            w[c] = pack_bf16x2(__uint_as_float(w[c] << 16) * f, __uint_as_float(w[c] & 0xffff0000u) * f);
+          tmem_st32(s_addr, w);
+        }
+        if (need) {
+          const float f = ex2(m_run - m_cand);      // 0 while nothing was attended yet
+          if (m_run != -INFINITY) o_scaled = true;
+          l_run *= f;
+          o_factor *= f;
+          sum_a *= f;
+          sum_b *= f;
+          m_run = m_cand;
+        }
+        const float base = (m_run == -INFINITY) ? 0.f : m_run;
         uint32_t pk[32];
-        if (state[half] == 0) {
+        if (none) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) pk[c] = 0u;
         } else {
+          const uint64_t sc2 = f2(sl2, sl2), nb2 = f2(-base, -base);
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const int e = half * 64 + 2 * c;
-            const uint64_t x = f2_fma(f2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), sc2, nb2);
-            float x0, x1, p0, p1;
+            const uint64_t x = f2_fma(f2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])), sc2, nb2);
+            float x0, x1;
             f2_split(x, x0, x1);
-            if ((c & 3) == 3 && state[half] == 1) {
-              exp2_poly2(x0, x1, p0, p1);
-            } else {
-              p0 = ex2(x0);
-              p1 = ex2(x1);
-            }
-            sum2 = f2_add(sum2, f2(p0, p1));
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            if (c & 1) sum_b += p0 + p1;
+            else sum_a += p0 + p1;
             pk[c] = pack_bf16x2(p0, p1);
           }
         }
-        tmem_st32(tmem + lane_off + s_col + half * 32u, pk);
+        tmem_st32(s_addr + half * 32u, pk);
       }
-      float s0, s1;
-      f2_split(sum2, s0, s1);
-      l_run += s0 + s1;
-      if (rescale_o) {
+      l_run += sum_a + sum_b;
+      if (__any_sync(0xffffffffu, o_scaled && j > 0)) {
         // the running max grew by more than 8: rescale O in TMEM before PV(j)
         if (NQ == 1) {
-          w = mbar_wait(smem_u32(&bars.pv_done), (j - 1) & 1, abort_flag);   // PV(j-1) must be done
-          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          bool w2 = mbar_wait(smem_u32(&bars.pv_done), (j - 1) & 1, abort_flag);   // PV(j-1) must be done
+          if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
           tc_fence_after();
         }
+        const float f = o_scaled ? o_factor : 1.f;
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
           uint32_t o[32];
           tmem_ld32(tmem + lane_off + o_col + c4 * 32u, o);
           tc_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * o_factor);
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
           tmem_st32(tmem + lane_off + o_col + c4 * 32u, o);
         }
       }

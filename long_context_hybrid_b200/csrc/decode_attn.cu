@@ -152,12 +152,13 @@ decode_attn_partial_kernel(const DecodeParams p) {
   // stage K, V (128 rows x 256 B each) and the query rows
   const __nv_bfloat16* kb = p.k + (int64_t)b * p.k_sb + (int64_t)g * p.k_sh;
   const __nv_bfloat16* vb = p.v + (int64_t)b * p.v_sb + (int64_t)g * p.v_sh;
+  // two copy groups: K and the query rows first, V second (S and the softmax
+  // run while V is still arriving)
   for (int e = tid; e < kChunk * 16; e += kThreads) {
     const int s = e >> 4, c = (e & 15) * 8;
     const int pos = sm.pos[s];
     const int64_t off = pos >= 0 ? (int64_t)pos : 0;
     cp_async16(su32(&sm.k[s][c]), kb + off * p.k_sn + c, pos >= 0);
-    cp_async16(su32(&sm.v[s][c]), vb + off * p.v_sn + c, pos >= 0);
   }
   for (int e = tid; e < kMaxGroup * 16; e += kThreads) {
     const int r = e >> 4, c = (e & 15) * 8;
@@ -166,7 +167,14 @@ decode_attn_partial_kernel(const DecodeParams p) {
     cp_async16(su32(&sm.q[r][c]), src, j >= 0);
   }
   asm volatile("cp.async.commit_group;\n" ::: "memory");
-  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+  for (int e = tid; e < kChunk * 16; e += kThreads) {
+    const int s = e >> 4, c = (e & 15) * 8;
+    const int pos = sm.pos[s];
+    const int64_t off = pos >= 0 ? (int64_t)pos : 0;
+    cp_async16(su32(&sm.v[s][c]), vb + off * p.v_sn + c, pos >= 0);
+  }
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+  asm volatile("cp.async.wait_group 1;\n" ::: "memory");
   __syncthreads();
 
   const int gq = lane >> 2, tq = lane & 3;
@@ -232,6 +240,8 @@ decode_attn_partial_kernel(const DecodeParams p) {
   l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
   l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
   l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+  __syncthreads();
   // O = P V (16 rows x 128 dims)
   float oacc[16][4];
 #pragma unroll
@@ -288,19 +298,37 @@ decode_attn_partial_kernel(const DecodeParams p) {
 
 __global__ void __launch_bounds__(RTP_D)
 decode_attn_merge_kernel(const DecodeParams p) {
+  extern __shared__ float wsm[];             // [n_splits] weights
+  __shared__ float red[2][4];
   const int j = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const int lane = d & 31, warp = d >> 5;
   const float* part = p.part + ((size_t)b * p.n_heads + j) * p.max_splits * kPartStride;
   const bool ret = p.ret_row[j] >= 0;
   const int n_splits = p.n_wc + (ret ? p.n_gc : 0);
   float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, part[s * kPartStride]);
-  float L = 0.f, acc = 0.f;
-  for (int s = 0; s < n_splits; ++s) {
+  for (int s = d; s < n_splits; s += RTP_D) M = fmaxf(M, part[s * kPartStride]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) red[0][warp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
+  float L = 0.f;
+  for (int s = d; s < n_splits; s += RTP_D) {
     const float ms = part[s * kPartStride];
-    if (ms == -INFINITY) continue;
-    const float w = exp2f(ms - M);
+    const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
+    wsm[s] = w;
     L += w * part[s * kPartStride + 1];
-    acc += w * part[s * kPartStride + 2 + d];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  if (lane == 0) red[1][warp] = L;
+  __syncthreads();
+  L = red[1][0] + red[1][1] + red[1][2] + red[1][3];
+  float acc = 0.f;
+#pragma unroll 4
+  for (int s = 0; s < n_splits; ++s) {
+    const float w = wsm[s];
+    if (w != 0.f) acc += w * part[s * kPartStride + 2 + d];
   }
   p.o[b * p.o_sb + (int64_t)p.head[j] * p.o_sh + d] = __float2bfloat16_rn(acc / L);
 }
@@ -355,6 +383,7 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
   p.n_wc = (p.whi - wlo_union + kChunk - 1) / kChunk;
   p.n_gc = n_ret > 0 ? n_gathered_chunks(p.topk, sink) : 0;
   p.max_splits = p.n_wc + p.n_gc;
+  if (Hkv > kMaxGroup) return cudaErrorInvalidValue;
   p.n_window_items = B * Hkv * p.n_wc;
   p.part = static_cast<float*>(ws);
   const int n_items = p.n_window_items + B * n_ret * p.n_gc;
@@ -366,7 +395,12 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 g2(p.n_heads, B);
-  decode_attn_merge_kernel<<<g2, RTP_D, 0, stream>>>(p);
+  const size_t msmem = (size_t)p.max_splits * sizeof(float);
+  if (msmem > 48 * 1024) {
+    e = cudaFuncSetAttribute(decode_attn_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+    if (e != cudaSuccess) return e;
+  }
+  decode_attn_merge_kernel<<<g2, RTP_D, msmem, stream>>>(p);
   return cudaGetLastError();
 }
 

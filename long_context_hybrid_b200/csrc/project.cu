@@ -1,6 +1,9 @@
 // Index projection x~ = x . P (D = 128 -> r = 16), the low-rank indexer of
 // the RTPurboV2 article (paragraph on the low-rank projector).
 //
+// Up to 64 rows per (sequence, head) take a small shared-memory kernel (the
+// decode step's queries); longer sequences the tensor-core kernel below.
+//
 // The work is HBM-bound: 256 bytes of x per row in, 32 (bf16) or 64 (fp32)
 // bytes out, 2048 multiply-adds per row. One warp computes 16 rows x 16
 // outputs with bf16 mma.sync (m16n8k16, fp32 accumulation): the K dimension
@@ -111,6 +114,33 @@ project_kernel(const ProjectParams p) {
   }
 }
 
+// Few rows (a decode step's queries): one CTA per (sequence, listed head)
+// stages the projector and the rows in shared memory with coalesced loads;
+// thread (row, c) forms one output with an fp32 dot product of length 128.
+constexpr int kSmallRows = 64;
+
+__global__ void __launch_bounds__(256)
+project_small_kernel(const ProjectParams p) {
+  __shared__ float Ps[RTP_D][RTP_R];
+  __shared__ float xs[kSmallRows][RTP_D + 1];
+  const int j = blockIdx.x, b = blockIdx.y;
+  const __nv_bfloat16* P = p.P + (size_t)p.proj[j] * RTP_D * RTP_R;
+  for (int e = threadIdx.x; e < RTP_D * RTP_R; e += blockDim.x) Ps[e / RTP_R][e % RTP_R] = __bfloat162float(P[e]);
+  const __nv_bfloat16* xb = p.x + (size_t)b * p.sb + (size_t)p.head[j] * p.sh;
+  for (int e = threadIdx.x; e < p.N * RTP_D; e += blockDim.x)
+    xs[e / RTP_D][e % RTP_D] = __bfloat162float(xb[(size_t)(e / RTP_D) * p.sn + e % RTP_D]);
+  __syncthreads();
+  const size_t obase = ((size_t)b * p.n_heads + j) * (size_t)p.N;
+  for (int e = threadIdx.x; e < p.N * RTP_R; e += blockDim.x) {
+    const int row = e / RTP_R, c = e % RTP_R;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int d = 0; d < RTP_D; ++d) acc = fmaf(xs[row][d], Ps[d][c], acc);
+    if (p.out_f32) reinterpret_cast<float*>(p.out)[(obase + row) * RTP_R + c] = acc;
+    else reinterpret_cast<__nv_bfloat16*>(p.out)[(obase + row) * RTP_R + c] = __float2bfloat16_rn(acc);
+  }
+}
+
 cudaError_t launch_project(const void* x, int64_t sb, int64_t sn, int64_t sh, int B, int N,
                            const void* P, const int32_t* heads, const int32_t* proj, int n_heads,
                            void* out, int out_f32, cudaStream_t stream) {
@@ -120,6 +150,11 @@ cudaError_t launch_project(const void* x, int64_t sb, int64_t sn, int64_t sh, in
   p.P = static_cast<const __nv_bfloat16*>(P);
   p.out = out; p.out_f32 = out_f32; p.n_heads = n_heads;
   for (int i = 0; i < n_heads; ++i) { p.head[i] = heads[i]; p.proj[i] = proj[i]; }
+  if (N <= kSmallRows) {
+    dim3 grid(n_heads, B);
+    project_small_kernel<<<grid, 256, 0, stream>>>(p);
+    return cudaGetLastError();
+  }
   const int rows_per_cta = kProjWarps * kProjRowsPerWarp;
   int gx = (N + rows_per_cta - 1) / rows_per_cta;
   // Enough CTAs to fill the GPU a few times; each loops over row tiles.

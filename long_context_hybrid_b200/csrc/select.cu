@@ -9,12 +9,14 @@
 //          writes every score (fp32, to the workspace, sized to stay in L2) and
 //          a histogram of the top 11 bits of each score's order-preserving key.
 //   top-k  one CTA per (sequence, head): from the histogram it knows the bin
-//          holding the k-th score; one pass over the scores takes every score
-//          above that bin and gathers the bin's members as candidates in
-//          shared memory, where a radix search over the remaining bits (and the
+//          holding the k-th score (top 11 bits). Pass 1 over the L2-resident
+//          scores takes every score above that bin and histograms the next 11
+//          bits of the scores inside it; pass 2 takes the scores above the
+//          finer bin and gathers that bin's few members as candidates in
+//          shared memory, where a radix search over the last 10 bits (and the
 //          token index for exact ties) settles the rest; the list is then
-//          sorted ascending. If the candidates overflow shared memory the CTA
-//          falls back to a full radix select over the scores.
+//          sorted ascending. If the candidates still overflow shared memory
+//          the CTA falls back to a full radix select over the scores.
 #include "rtp_common.cuh"
 #include "rtp_internal.h"
 
@@ -36,6 +38,44 @@ struct DecodeTopkSmem {
   int sel[kMaxTopk];
   int n_sel, n_cand, n_eq;
 };
+
+// Calls f(i, key, valid) over one score list [0, L): each warp takes 512
+// consecutive scores per step (16 per lane, four 16-byte loads issued
+// together; scalar loads when L is not a multiple of 4). Every lane of a warp
+// makes the same calls, so f may use warp votes; `valid` is false past L.
+template <int NT, class F>
+__device__ __forceinline__ void for_each_key(const float* __restrict__ s, int L, F f) {
+  const bool vec = (L & 3) == 0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int wbase = warp * 512; wbase < L; wbase += NT * 16) {
+    const int base = wbase + lane * 16;
+    float x[16];
+    if (vec && base + 16 <= L) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 w = __ldg(reinterpret_cast<const float4*>(s + base) + q);
+        x[4 * q] = w.x; x[4 * q + 1] = w.y; x[4 * q + 2] = w.z; x[4 * q + 3] = w.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) x[e] = base + e < L ? __ldg(s + base + e) : 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) f(base + e, f2key(x[e]), base + e < L);
+  }
+}
+
+// Appends `i` to list[] (counter *n) for the lanes with `take`, one shared
+// atomic per warp.
+__device__ __forceinline__ void warp_append(bool take, int i, int* list, int* n) {
+  const unsigned m = __ballot_sync(0xffffffffu, take);
+  if (m == 0) return;
+  const int lane = threadIdx.x & 31, leader = __ffs(m) - 1;
+  int base = 0;
+  if (lane == leader) base = atomicAdd(n, __popc(m));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  if (take) list[base + __popc(m & ((1u << lane) - 1u))] = i;
+}
 
 size_t hist_offset(int B, int L, int Hr) {
   return (((size_t)B * Hr * L * sizeof(float)) + 255) & ~(size_t)255;
@@ -123,18 +163,47 @@ decode_topk_kernel(const float* __restrict__ scores, const uint32_t* __restrict_
   }
   __syncthreads();
   const uint32_t d1 = (uint32_t)sm.tk.digit;
-  const int above = sm.tk.above;
-  // 2. one pass: take keys above the bin, gather the bin's members
-  for (int i = tid; i < L; i += kTopkThreads) {
-    const uint32_t key = key_of(i);
+  const int above1 = sm.tk.above;
+  __syncthreads();
+  // 2a. pass 1: take keys above bin d1, histogram bits [20:10] inside it
+  for (int x = tid; x < kBins; x += kTopkThreads) sm.tk.hist[x] = 0u;
+  __syncthreads();
+  for_each_key<kTopkThreads>(s, L, [&](int i, uint32_t key, bool valid) {
     const uint32_t d = key >> 21;
-    if (d > d1) {
-      sm.sel[atomicAdd(&sm.n_sel, 1)] = i;
-    } else if (d == d1) {
+    warp_append(valid && d > d1, i, sm.sel, &sm.n_sel);
+    if (valid && d == d1) atomicAdd(&sm.tk.hist[(key >> 10) & 2047u], 1u);
+  });
+  __syncthreads();
+  const int need1 = topk - above1;
+  {
+    int loc = 0;
+    for (int q = 0; q < per; ++q) loc += sm.tk.hist[kBins - 1 - (tid * per + q)];
+    int t2;
+    const int ab = block_exclusive_scan<kTopkThreads>(loc, t2, sm.tk.scan);
+    if (ab < need1 && ab + loc >= need1) {
+      int run = ab;
+      for (int q = 0; q < per; ++q) {
+        const int bin = kBins - 1 - (tid * per + q);
+        const int c = sm.tk.hist[bin];
+        if (run + c >= need1) { sm.tk.digit = bin; sm.tk.above = run; break; }
+        run += c;
+      }
+    }
+    __syncthreads();
+  }
+  const uint32_t pre22 = (d1 << 11) | (uint32_t)sm.tk.digit;   // key >> 10 of the k-th key
+  const int above = above1 + sm.tk.above;
+  __syncthreads();
+  // 2b. pass 2: take keys above the 22-bit bin, gather the bin's members
+  for_each_key<kTopkThreads>(s, L, [&](int i, uint32_t key, bool valid) {
+    const bool in1 = valid && (key >> 21) == d1;
+    const uint32_t d = key >> 10;
+    warp_append(in1 && d > pre22, i, sm.sel, &sm.n_sel);
+    if (in1 && d == pre22) {
       const int pos = atomicAdd(&sm.n_cand, 1);
       if (pos < kCandCap) { sm.cand_key[pos] = key; sm.cand_idx[pos] = i; }
     }
-  }
+  });
   __syncthreads();
   const int n_cand = sm.n_cand;
   if (n_cand > kCandCap || sm.n_sel != above) {
@@ -147,8 +216,8 @@ decode_topk_kernel(const float* __restrict__ scores, const uint32_t* __restrict_
   int need = topk - above;
   const uint32_t* ck = sm.cand_key;
   auto cand_key = [ck](int x) { return ck[x]; };
-  const uint32_t thr = block_radix_threshold<kTopkThreads>(cand_key, n_cand, need, sm.tk, 1, d1 << 21,
-                                                            0x7FFu << 21);
+  const uint32_t thr = block_radix_threshold<kTopkThreads>(cand_key, n_cand, need, sm.tk, 2, pre22 << 10,
+                                                            0x3FFFFFu << 10);
   for (int x = tid; x < n_cand; x += kTopkThreads)
     if (sm.cand_key[x] > thr) sm.sel[atomicAdd(&sm.n_sel, 1)] = sm.cand_idx[x];
   __syncthreads();

@@ -8,16 +8,13 @@
 // are taken.
 //
 // One CTA handles query blocks 2t and 2t+1 (128 query rows) of one retrieval
-// head, longest key ranges first. Warp roles (640 threads):
+// head, longest key ranges first. Warp roles (384 threads):
 //   warp 0       TMA: the 128 x 16 query-index tile once, then 256 x 16
 //                key-index tiles (4 key blocks) into a 4-stage ring (32-byte
 //                swizzle);
 //   warp 1       TMEM owner and MMA issuer: one tcgen05.mma M=128 N=256 K=16
 //                per key tile into one of two TMEM score buffers;
-//   warps 4..19  four epilogue warpgroups; warpgroup w reduces key block w of
-//                every tile (one 64-column TMEM load per thread), so the four
-//                blocks of a tile are reduced at once while the tensor core
-//                fills the other buffer: thread r reads
+//   warps 4..11  two epilogue warpgroups, one per score buffer: thread r reads
 //                row r of the tile, takes the causal max of each 64-column
 //                block (3-input max), reduces over the 32 rows of its warp
 //                (redux.sync), and folds the result into the block-score array
@@ -34,22 +31,18 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kThreads = 640;
+constexpr int kThreads = 384;
 constexpr int kKStages = 4;
-constexpr int kBufs = 2;                           // TMEM score buffers
-constexpr int kEpiWGs = 4;                         // epilogue warpgroups, one key block each
 constexpr int kChunkKeys = 256;                    // 4 key blocks per MMA
-constexpr int kBlocksPerChunk = kChunkKeys / RTP_BLOCK;
-constexpr uint32_t kStageBytes = kChunkKeys * 32u; // 128 rows x 32 B
 constexpr uint32_t kQOff = 0;                      // 128 rows x 32 B
-constexpr uint32_t kKOff = 4096;                   // stage s at +s*kStageBytes
-constexpr uint32_t kScoreOff = kKOff + kKStages * kStageBytes;
+constexpr uint32_t kKOff = 4096;                   // stage s at +s*8192 (256 rows x 32 B)
+constexpr uint32_t kScoreOff = kKOff + kKStages * 8192u;
 constexpr int kStatusTimeout = 4;
 
 struct SelBars {
   uint64_t q_full;
   uint64_t k_full[kKStages], k_empty[kKStages];
-  uint64_t s_full[kBufs], s_free[kBufs];
+  uint64_t s_full[2], s_free[2];
   uint64_t fin;
   uint32_t tmem_base;
   int abort;
@@ -104,7 +97,7 @@ prefill_select_tc_kernel(const SelectTcParams p, const __grid_constant__ CUtenso
   const int qa = 2 * t, qb = 2 * t + 1;
   const bool has_b = qb < p.nb;
   const int last_blk = has_b ? qb : qa;
-  const int n_chunks = (last_blk + kBlocksPerChunk) / kBlocksPerChunk;
+  const int n_chunks = (last_blk + 1 + 3) / 4;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint32_t* sA = reinterpret_cast<uint32_t*>(smem + kScoreOff);
   uint32_t* sB = sA + p.nb;
@@ -118,9 +111,9 @@ prefill_select_tc_kernel(const SelectTcParams p, const __grid_constant__ CUtenso
       mbar_init(smem_u32(&bars.k_full[s]), 1);
       mbar_init(smem_u32(&bars.k_empty[s]), 1);
     }
-    for (int s = 0; s < kBufs; ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&bars.s_full[s]), 1);
-      mbar_init(smem_u32(&bars.s_free[s]), 128 * kEpiWGs);
+      mbar_init(smem_u32(&bars.s_free[s]), 128);
     }
     mbar_init(smem_u32(&bars.fin), 1);
     bars.abort = 0;
@@ -147,8 +140,8 @@ prefill_select_tc_kernel(const SelectTcParams p, const __grid_constant__ CUtenso
         const int s = c % kKStages;
         if (c >= kKStages && !mbar_wait(smem_u32(&bars.k_empty[s]), ((c / kKStages) - 1) & 1, abort_flag)) break;
         const uint32_t kbar = smem_u32(&bars.k_full[s]);
-        mbar_arrive_expect_tx(kbar, kStageBytes);
-        tma_load_4d(sb + kKOff + s * kStageBytes, &tmK, kbar, 0, c * kChunkKeys, g, b);
+        mbar_arrive_expect_tx(kbar, 8192);
+        tma_load_4d(sb + kKOff + s * 8192u, &tmK, kbar, 0, c * kChunkKeys, g, b);
         issued = c + 1;
       }
       if (*abort_flag) {
@@ -159,15 +152,15 @@ prefill_select_tc_kernel(const SelectTcParams p, const __grid_constant__ CUtenso
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, kChunkKeys, false, false);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false, false);
       bool ok = mbar_wait(smem_u32(&bars.q_full), 0, abort_flag);
       const uint64_t qdesc = desc_sw32(sb + kQOff);
       for (int c = 0; ok && c < n_chunks; ++c) {
-        const int s = c % kKStages, buf = c % kBufs;
+        const int s = c % kKStages, buf = c & 1;
         if (!mbar_wait(smem_u32(&bars.k_full[s]), (c / kKStages) & 1, abort_flag)) break;
-        if (c >= kBufs && !mbar_wait(smem_u32(&bars.s_free[buf]), ((c / kBufs) - 1) & 1, abort_flag)) break;
+        if (c >= 2 && !mbar_wait(smem_u32(&bars.s_free[buf]), ((c >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();
-        mma_bf16_ss(tmem + buf * (uint32_t)kChunkKeys, qdesc, desc_sw32(sb + kKOff + s * kStageBytes), idesc, 0u);
+        mma_bf16_ss(tmem + buf * 256u, qdesc, desc_sw32(sb + kKOff + s * 8192u), idesc, 0u);
         mma_commit(smem_u32(&bars.s_full[buf]));
         mma_commit(smem_u32(&bars.k_empty[s]));
       }
@@ -176,38 +169,38 @@ prefill_select_tc_kernel(const SelectTcParams p, const __grid_constant__ CUtenso
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int wg = (warp - 4) >> 2;                 // 0..3: which key block of each tile
-    const int r = (warp & 3) * 32 + lane;           // row 0..127 of the tile (TMEM lane)
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const int wg = (warp - 4) >> 2;                 // 0 or 1: which score buffer
+    const int r = tid - 128 - wg * 128;             // row 0..127 of the tile
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16) + wg * 256u;
     const bool in_a = r < 64;
     const int my_last = in_a ? qa : last_blk;       // key blocks this row's query block may see
     const int rq = in_a ? r : r - 64;               // row within its query block
     const int my_q = in_a ? qa : qb;
     uint32_t* dst = in_a ? sA : sB;
-    for (int c = 0; c < n_chunks; ++c) {
-      const int buf = c % kBufs;
-      bool w = mbar_wait(smem_u32(&bars.s_full[buf]), (c / kBufs) & 1, abort_flag);
+    for (int c = wg; c < n_chunks; c += 2) {
+      bool w = mbar_wait(smem_u32(&bars.s_full[wg]), (c >> 1) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after();
-      const int kb = c * kBlocksPerChunk + wg;
-      if (kb <= last_blk) {                         // CTA-uniform per warpgroup
+#pragma unroll
+      for (int bi = 0; bi < 4; ++bi) {
+        const int kb = c * 4 + bi;
+        if (kb > last_blk) break;                   // warp-uniform: same for the whole CTA
         uint32_t v[64];
-        const uint32_t col = tmem + lane_off + buf * (uint32_t)kChunkKeys + wg * 64u;
-        tmem_ld32(col, v);
-        tmem_ld32(col + 32u, v + 32);
+        tmem_ld32(lane_base + bi * 64u, v);
+        tmem_ld32(lane_base + bi * 64u + 32u, v + 32);
         tc_wait_ld();
         float m = -INFINITY;
         if (kb < my_q) {
           // 64 -> 1 in a tree of 3-input maxima (32 instructions, depth 4)
-          float a[22], cc[8];
+          float a[22], c[8];
 #pragma unroll
           for (int x = 0; x < 21; ++x)
             a[x] = max3f(__uint_as_float(v[3 * x]), __uint_as_float(v[3 * x + 1]), __uint_as_float(v[3 * x + 2]));
           a[21] = __uint_as_float(v[63]);
 #pragma unroll
-          for (int x = 0; x < 7; ++x) cc[x] = max3f(a[3 * x], a[3 * x + 1], a[3 * x + 2]);
-          cc[7] = a[21];
-          m = max3f(max3f(cc[0], cc[1], cc[2]), max3f(cc[3], cc[4], cc[5]), fmaxf(cc[6], cc[7]));
+          for (int x = 0; x < 7; ++x) c[x] = max3f(a[3 * x], a[3 * x + 1], a[3 * x + 2]);
+          c[7] = a[21];
+          m = max3f(max3f(c[0], c[1], c[2]), max3f(c[3], c[4], c[5]), fmaxf(c[6], c[7]));
         } else if (kb == my_q) {
           // diagonal block: key column x is causal for this row iff x <= rq
 #pragma unroll
@@ -219,7 +212,7 @@ prefill_select_tc_kernel(const SelectTcParams p, const __grid_constant__ CUtenso
         if (lane == 0 && kb <= my_last && wm != -INFINITY) atomicMax(&dst[kb], f2key(wm));
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&bars.s_free[buf]));
+      mbar_arrive(smem_u32(&bars.s_free[wg]));
     }
   }
 
@@ -274,16 +267,10 @@ cudaError_t launch_select_prefill_tc(const void* qt, const void* kt, int B, int 
   return cudaGetLastError();
 }
 
-size_t select_prefill_ws_bytes(int B, int N, int Hr, int topk) {
-  (void)B; (void)N; (void)Hr; (void)topk;
-  return kStatusBytes;
-}
-
+size_t select_prefill_ws_bytes(int B, int N, int Hr, int topk) { (void)B; (void)N; (void)Hr; (void)topk; return kStatusBytes; }
 cudaError_t launch_select_prefill(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
                                   const int32_t* kv_of, int topk, int32_t* blocks, int32_t* counts, void* ws,
                                   cudaStream_t stream) {
-  return launch_select_prefill_tc(qt, kt, B, N, Hr, Hkv, kv_of, topk, blocks, counts, static_cast<int*>(ws),
-                                  stream);
+  return launch_select_prefill_tc(qt, kt, B, N, Hr, Hkv, kv_of, topk, blocks, counts, static_cast<int*>(ws), stream);
 }
-
 }  // namespace rtp

@@ -107,3 +107,13 @@ def test_binding_raises_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(rtp, "_lib", None)
     with pytest.raises(rtp.RtpError):
         rtp.lib()
+
+
+def test_timeout_probe_validates_before_launch(L):
+    import long_context_hybrid_b200 as rtp
+    fn = L.rtp_debug_prefill_timeout_probe
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_size_t, ctypes.c_void_p]
+    fake = 0x10000
+    assert fn(None, fake, fake, fake, fake, 256, None) == 1          # null input
+    assert fn(fake, fake, fake, fake, fake, 16, None) == 5           # workspace too small

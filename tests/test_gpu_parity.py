@@ -117,6 +117,21 @@ def test_select_decode_ties_pick_lowest_index():
     assert list(idx[0, 0]) == list(range(topk))
 
 
+def test_select_decode_candidate_overflow_falls_back_exactly():
+    """More equal scores in the k-th score's bin than the candidate list holds:
+    the full radix select must still pick the lowest indices; a second row with
+    distinct scores in the same call takes the normal path."""
+    L, topk = 20000, 300
+    kindex = torch.ones(1, 2, L, 16, dtype=torch.bfloat16)
+    kindex[0, 1] = _clustered_bf16((1, 1, L, 16), 77)[0, 0]
+    qt = torch.ones(1, 2, 16)
+    idx = rtp.select_decode(qt.to(DEV), kindex.to(DEV), [0, 1], topk).cpu().numpy()
+    assert list(idx[0, 0]) == list(range(topk))
+    sc = O.decode_scores(qt[0, 1].double().numpy(), kindex[0, 1])
+    ok, amb, msg = band_check(idx[0, 1], O.topk_desc(sc, topk), sc, topk)
+    assert ok, msg
+
+
 # ---------------------------------------------------------------------------
 # Prefill selection
 # ---------------------------------------------------------------------------

@@ -84,8 +84,8 @@ RTP_API int rtp_version(void);
 
 /*
  * rtp_workspace_status - device-side status of the last call that used `ws`.
- *   The prefill attention calls keep a status word in the first bytes of
- *   their workspace: cleared on the stream before the launch, set to
+ *   The prefill and decode attention calls keep a status word in the first
+ *   bytes of their workspace: cleared on the stream before the launch, set to
  *   RTP_ERR_TIMEOUT by a CTA whose bounded wait ran out (the kernel then
  *   drains and returns instead of spinning). This call synchronises `stream`
  *   and returns RTP_OK or the recorded status.
@@ -260,16 +260,18 @@ RTP_API rtp_status rtp_decode_attn_hybrid(const void* q, const void* kc, rtp_str
  *   cudaMalloc/cudaFree (both may synchronise the device) on every step.
  *
  *   Arguments, layouts and results are those of rtp_sparse_attn_decode. The
- *   split-K partials go to a fixed array inside the library, 4 MiB per GPU,
- *   held by every GPU that loads the library until the process exits. A call
- *   whose partials would not fit (about B * Hr * (ceil(window/128) +
- *   ceil((topk+64)/128)) * 520 bytes > 4 MiB) returns RTP_ERR_WORKSPACE and
+ *   split-K partials, the per-head tickets and the status word go to a fixed
+ *   array inside the library, 4 MiB per GPU, held by every GPU that loads the
+ *   library until the process exits. A call whose workspace would not fit
+ *   (about 512 + 4 * B * Hr + B * Hr * (ceil(window/128) +
+ *   ceil((topk+64)/128)) * 528 bytes > 4 MiB) returns RTP_ERR_WORKSPACE and
  *   launches nothing. The first call on a device looks up the array's device
  *   address (with that device current) and caches it; make that first call
  *   before any stream capture. Every call shares the one array, so calls
  *   whose work may overlap on the GPU (different streams, or concurrent host
  *   threads) race on it and must be serialised by the caller. Nothing in the
- *   array needs to start at zero: each call writes every partial it reads.
+ *   array needs to start at zero: each call clears its status word and
+ *   tickets on the stream and writes every partial it reads.
  */
 RTP_API rtp_status rtp_sparse_attn_decode_noalloc(const void* q, const void* kc, rtp_strides ks,
                                                   const void* vc, rtp_strides vs, void* o,

@@ -7,19 +7,26 @@
 // exact softmax at D = 128).
 //
 // The work is HBM-bound (512 bytes of K and V per attended token), so the
-// design goal is to read every K/V row once:
-//   * window items: one CTA per (sequence, KV group, 128-token chunk of the
-//     window); every listed query head of that group is one row of a
-//     16 x 128 query tile (grouped-query heads share the chunk's K/V), and
-//     each row masks keys outside its own window;
-//   * gathered items: one CTA per (sequence, retrieval head, 128-entry chunk
-//     of its selected list, the sink tokens first); entries inside the
-//     window or below `sink` are masked (those keys come from elsewhere).
-// A CTA stages its 128 K and V rows in shared memory with cp.async (zero-fill
-// for masked slots), computes S = Q K^T and O = P V with bf16 mma.sync
-// (fp32 accumulate) in four warps of 32 keys, and writes an unnormalised
-// partial (running max in the log2 domain, sum, o[128]) per head; a merge
-// kernel combines the partials of each head.
+// design goal is to read every K/V row once and keep enough bytes in flight:
+//   * the work is two lists of 128-key chunks in segments: a window segment
+//     per (sequence, KV group) covers the union of the window, with every
+//     listed query head of the group as one row of a 16 x 128 query tile
+//     (grouped heads share the chunk's K/V; each row masks keys outside its
+//     own window); a gathered segment per (sequence, retrieval head) covers
+//     its sink tokens and selected list (entries inside the window or below
+//     `sink` are masked: those keys come from elsewhere);
+//   * one persistent CTA per SM takes a contiguous run of each list, so both
+//     kinds of chunk are spread evenly. Each of its four warps owns 32 keys of
+//     every chunk: it copies its own K and V rows with 16-byte cp.async
+//     (zero-filled where masked) three chunks ahead into a private ring of
+//     256-byte rows whose 16-byte pieces are XOR-swizzled (conflict-free
+//     ldmatrix), and computes S = Q K^T and O += P V with bf16 mma.sync (fp32
+//     accumulate) and an online softmax carried across the run's chunks of a
+//     segment. The warps never wait for one another inside a segment;
+//   * where a run leaves a segment the four warps combine their states and
+//     write one partial per head (running max in the log2 domain, sum,
+//     o[128]); the CTA that completes a head's chunk count (an atomic ticket)
+//     merges that head's partials and writes its output.
 #include <mutex>
 
 #include "rtp_common.cuh"
@@ -28,46 +35,53 @@
 namespace rtp {
 
 namespace {
-constexpr int kThreads = 128;
-constexpr int kChunk = 128;                 // keys per CTA (32 per warp)
-constexpr int kRowPad = RTP_D + 8;          // shared row stride in elements (272 B: conflict-free ldmatrix)
-constexpr int kPartStride = 2 + RTP_D;
-constexpr int kMaxGroup = 16;               // query heads per KV group packed in one MMA tile
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kChunk = 128;                   // keys per chunk
+constexpr int kKeys = kChunk / kWarps;        // keys per warp and chunk (32)
+constexpr int kStages = 3;
+constexpr int kRowBytes = RTP_D * 2;          // 256
+constexpr int kSlab = kKeys * kRowBytes;      // one warp's K (or V) rows of one chunk
+constexpr int kPartStride = 4 + RTP_D;        // m, l, 2 pad, o[128] (16-byte aligned rows)
+constexpr int kPartO = 4;
+constexpr int kMaxGroup = 16;                 // query heads per KV group packed in one MMA tile
+constexpr size_t kHeaderBytes = 256;          // status word (cleared by every call)
 
 struct DecodeParams {
   const __nv_bfloat16* q; int64_t q_sb, q_sh;
   const __nv_bfloat16* k; int64_t k_sb, k_sn, k_sh;
   const __nv_bfloat16* v; int64_t v_sb, v_sn, v_sh;
   __nv_bfloat16* o; int64_t o_sb, o_sh;
-  int B, L, q_pos, Hq, Hkv, G;
+  int B, G;
   const int32_t* idx; int topk;
   int sink;
   float scale_log2;
-  int n_heads, max_splits;
+  int n_heads, n_ret;                // call heads: retrieval heads first (0..n_ret-1)
+  int max_slots;                     // partial slots per head
   int n_wc, wlo_union, whi;          // window chunks over [wlo_union, whi)
   int n_gc;                          // gathered chunks per retrieval head
-  int n_window_items;                // B * Hkv * n_wc
-  float* part;
-  int head[kMaxHeads];
-  int ret_row[kMaxHeads];            // row of idx for a retrieval head, -1 for a streaming head
-  int wlo[kMaxHeads];                // first position of each head's window
-  int ret_list[kMaxHeads];           // call-head index of the r-th retrieval head
-  int n_ret;
+  int n_ag;                          // KV groups with at least one listed head
+  int n_win_chunks;                  // B * n_ag * n_wc
+  int n_gat_chunks;                  // B * n_ret * n_gc
+  float* part;                       // [B, n_heads, max_slots, kPartStride]
+  int* ticket;                       // [B, n_heads] chunks accounted for
+  int head[kMaxHeads];               // query head of each call head
+  int wlo[kMaxHeads];                // first position of each call head's window
+  int ag_of[kMaxHeads];              // active-group index of each call head
+  int ag_kv[kMaxGroup];              // KV group of each active group
+  int ag_n[kMaxGroup];               // rows (call heads) of each active group
+  int ag_rows[kMaxGroup][kMaxGroup];
 };
 
 struct Smem {
-  __nv_bfloat16 k[kChunk][kRowPad];
-  __nv_bfloat16 v[kChunk][kRowPad];
-  __nv_bfloat16 q[kMaxGroup][kRowPad];
-  int pos[kChunk];
-  int rows[kMaxGroup];               // call-head index per tile row, -1 if unused
-  float m[4][kMaxGroup], l[4][kMaxGroup];
+  unsigned char ring[kWarps][kStages][2][kSlab];   // [warp][stage][K, V]
+  float comb[2][kMaxGroup][RTP_D];                 // cross-warp combine buffer
+  float cm[kWarps][kMaxGroup], cl[kWarps][kMaxGroup];
+  int pos[kWarps][kStages][kKeys];
+  int todo[kMaxGroup];                             // heads completed by the current flush
+  int n_todo;
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-               : "memory");
-}
 __device__ __forceinline__ void ldsm_x4(uint32_t* r, uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
@@ -89,261 +103,384 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return r;
 }
 __device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-}  // namespace
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
-__global__ void __launch_bounds__(kThreads)
-decode_attn_partial_kernel(const DecodeParams p) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int item = blockIdx.x;
-  int b, g, split, n_rows;
-  const bool is_window = item < p.n_window_items;
-  if (is_window) {
-    const int wc = item % p.n_wc;
-    const int bg = item / p.n_wc;
-    g = bg % p.Hkv; b = bg / p.Hkv; split = wc;
-    if (tid == 0) {
-      int c = 0;
-      for (int j = 0; j < p.n_heads && c < kMaxGroup; ++j)
-        if (p.head[j] / p.G == g) sm.rows[c++] = j;
-      for (int r = c; r < kMaxGroup; ++r) sm.rows[r] = -1;
-    }
-  } else {
-    const int it = item - p.n_window_items;
-    const int gc = it % p.n_gc;
-    const int rr = (it / p.n_gc) % p.n_ret;
-    b = it / (p.n_gc * p.n_ret);
-    const int j = p.ret_list[rr];
-    g = p.head[j] / p.G; split = p.n_wc + gc;
-    if (tid == 0) {
-      sm.rows[0] = j;
-      for (int r = 1; r < kMaxGroup; ++r) sm.rows[r] = -1;
-    }
-  }
-  __syncthreads();
-  // key positions of the chunk's slots (-1: masked for every row)
-  if (is_window) {
-    for (int s = tid; s < kChunk; s += kThreads) {
-      const int u = p.wlo_union + split * kChunk + s;
-      sm.pos[s] = u < p.whi ? u : -1;
-    }
-  } else {
-    const int j = sm.rows[0];
-    const int wlo = p.wlo[j];
-    const int n_sink = min(p.sink, wlo);
-    const int gc = split - p.n_wc;
-    const int32_t* sel = p.idx + ((size_t)b * p.n_ret + p.ret_row[j]) * p.topk;
-    for (int s = tid; s < kChunk; s += kThreads) {
-      const int e = gc * kChunk + s;          // virtual list: sink tokens, then the selected entries
-      int pos = -1;
-      if (e < n_sink) pos = e;
-      else if (e - n_sink < p.topk) {
-        const int u = __ldg(sel + (e - n_sink));
-        pos = (u >= p.sink && u < wlo) ? u : -1;
-      }
-      sm.pos[s] = pos;
-    }
-  }
-  __syncthreads();
-  n_rows = 0;
-  for (int r = 0; r < kMaxGroup; ++r) n_rows += sm.rows[r] >= 0;
-
-  // stage K, V (128 rows x 256 B each) and the query rows
-  const __nv_bfloat16* kb = p.k + (int64_t)b * p.k_sb + (int64_t)g * p.k_sh;
-  const __nv_bfloat16* vb = p.v + (int64_t)b * p.v_sb + (int64_t)g * p.v_sh;
-  // two copy groups: K and the query rows first, V second (S and the softmax
-  // run while V is still arriving)
-  for (int e = tid; e < kChunk * 16; e += kThreads) {
-    const int s = e >> 4, c = (e & 15) * 8;
-    const int pos = sm.pos[s];
-    const int64_t off = pos >= 0 ? (int64_t)pos : 0;
-    cp_async16(su32(&sm.k[s][c]), kb + off * p.k_sn + c, pos >= 0);
-  }
-  for (int e = tid; e < kMaxGroup * 16; e += kThreads) {
-    const int r = e >> 4, c = (e & 15) * 8;
-    const int j = sm.rows[r];
-    const __nv_bfloat16* src = p.q + (int64_t)b * p.q_sb + (int64_t)(j >= 0 ? p.head[j] : 0) * p.q_sh + c;
-    cp_async16(su32(&sm.q[r][c]), src, j >= 0);
-  }
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-  for (int e = tid; e < kChunk * 16; e += kThreads) {
-    const int s = e >> 4, c = (e & 15) * 8;
-    const int pos = sm.pos[s];
-    const int64_t off = pos >= 0 ? (int64_t)pos : 0;
-    cp_async16(su32(&sm.v[s][c]), vb + off * p.v_sn + c, pos >= 0);
-  }
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-  asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-  __syncthreads();
-
-  const int gq = lane >> 2, tq = lane & 3;
-  const int key0 = warp * 32;                 // this warp's 32 keys: 4 n-tiles of 8
-  // S = Q K^T (16 rows x 32 keys)
-  float sacc[4][4];
-#pragma unroll
-  for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-    for (int x = 0; x < 4; ++x) sacc[nt][x] = 0.f;
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    uint32_t a[4];
-    {
-      const int m = lane >> 3;
-      const int row = (lane & 7) + 8 * (m & 1), col = kk * 16 + 8 * (m >> 1);
-      ldsm_x4(a, su32(&sm.q[row][col]));
-    }
-#pragma unroll
-    for (int np = 0; np < 2; ++np) {          // two n-tiles per ldmatrix.x4
-      uint32_t bf[4];
-      const int m = lane >> 3;
-      const int key = key0 + 8 * (2 * np + (m >> 1)) + (lane & 7), col = kk * 16 + 8 * (m & 1);
-      ldsm_x4(bf, su32(&sm.k[key][col]));
-      mma16816(sacc[2 * np], a, bf[0], bf[1]);
-      mma16816(sacc[2 * np + 1], a, bf[2], bf[3]);
-    }
-  }
-  // mask + per-row max over this warp's keys (rows gq and gq+8)
-  const int ja = sm.rows[gq], jb = sm.rows[gq + 8];
-  const int lo_a = ja >= 0 ? (is_window ? p.wlo[ja] : 0) : 0x7fffffff;
-  const int lo_b = jb >= 0 ? (is_window ? p.wlo[jb] : 0) : 0x7fffffff;
-  float mx_a = -INFINITY, mx_b = -INFINITY;
-#pragma unroll
-  for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      const int pos = sm.pos[key0 + nt * 8 + 2 * tq + x];
-      const bool oka = pos >= 0 && pos >= lo_a && ja >= 0;
-      const bool okb = pos >= 0 && pos >= lo_b && jb >= 0;
-      sacc[nt][x] = oka ? sacc[nt][x] * p.scale_log2 : -INFINITY;
-      sacc[nt][2 + x] = okb ? sacc[nt][2 + x] * p.scale_log2 : -INFINITY;
-      mx_a = fmaxf(mx_a, sacc[nt][x]);
-      mx_b = fmaxf(mx_b, sacc[nt][2 + x]);
-    }
-  mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-  mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-  mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-  mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-  const float base_a = mx_a == -INFINITY ? 0.f : mx_a, base_b = mx_b == -INFINITY ? 0.f : mx_b;
-  float l_a = 0.f, l_b = 0.f;
-  uint32_t pa[2][4];                          // A fragments of P for the two 16-key steps
-#pragma unroll
-  for (int nt = 0; nt < 4; ++nt) {
-    const float e0 = exp2f(sacc[nt][0] - base_a), e1 = exp2f(sacc[nt][1] - base_a);
-    const float e2 = exp2f(sacc[nt][2] - base_b), e3 = exp2f(sacc[nt][3] - base_b);
-    l_a += e0 + e1;
-    l_b += e2 + e3;
-    pa[nt >> 1][(nt & 1) * 2 + 0] = pack2(e0, e1);
-    pa[nt >> 1][(nt & 1) * 2 + 1] = pack2(e2, e3);
-  }
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-  __syncthreads();
-  // O = P V (16 rows x 128 dims)
-  float oacc[16][4];
-#pragma unroll
-  for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-    for (int x = 0; x < 4; ++x) oacc[nt][x] = 0.f;
-#pragma unroll
-  for (int ks = 0; ks < 2; ++ks) {
-#pragma unroll
-    for (int np = 0; np < 8; ++np) {
-      uint32_t bf[4];
-      const int m = lane >> 3;
-      const int key = key0 + 16 * ks + 8 * (m & 1) + (lane & 7), col = 8 * (2 * np + (m >> 1));
-      ldsm_x4_t(bf, su32(&sm.v[key][col]));
-      mma16816(oacc[2 * np], pa[ks], bf[0], bf[1]);
-      mma16816(oacc[2 * np + 1], pa[ks], bf[2], bf[3]);
-    }
-  }
-  // combine the four warps: stats through shared memory, O rows through the K tile
-  if (tq == 0) {
-    sm.m[warp][gq] = mx_a; sm.m[warp][gq + 8] = mx_b;
-    sm.l[warp][gq] = l_a; sm.l[warp][gq + 8] = l_b;
-  }
-  __syncthreads();                            // everyone is done with K and V
-  float* obuf = reinterpret_cast<float*>(&sm.k[0][0]);   // [4 warps][16 rows][128]
-#pragma unroll
-  for (int nt = 0; nt < 16; ++nt) {
-    const int col = nt * 8 + 2 * tq;
-    obuf[(warp * kMaxGroup + gq) * RTP_D + col] = oacc[nt][0];
-    obuf[(warp * kMaxGroup + gq) * RTP_D + col + 1] = oacc[nt][1];
-    obuf[(warp * kMaxGroup + gq + 8) * RTP_D + col] = oacc[nt][2];
-    obuf[(warp * kMaxGroup + gq + 8) * RTP_D + col + 1] = oacc[nt][3];
-  }
-  __syncthreads();
-  const int d = tid;                           // one output column per thread
-  for (int r = 0; r < n_rows; ++r) {
-    const int j = sm.rows[r];
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm.m[w][r]);
-    float Lsum = 0.f, acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float mw = sm.m[w][r];
-      const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
-      Lsum += f * sm.l[w][r];
-      acc += f * obuf[(w * kMaxGroup + r) * RTP_D + d];
-    }
-    float* part = p.part + (((size_t)b * p.n_heads + j) * p.max_splits + split) * kPartStride;
-    part[2 + d] = acc;
-    if (d == 0) { part[0] = M; part[1] = Lsum; }
-  }
+// Byte offset of 16-byte piece c (0..15) of row r in a slab of 256-byte rows:
+// the piece index is XORed with r mod 8, so the eight rows of an ldmatrix
+// read hit distinct banks.
+__device__ __forceinline__ uint32_t slab_off(int r, int c) {
+  return (uint32_t)(r * kRowBytes + ((c ^ (r & 7)) << 4));
 }
 
-__global__ void __launch_bounds__(RTP_D)
-decode_attn_merge_kernel(const DecodeParams p) {
-  extern __shared__ float wsm[];             // [n_splits] weights
-  __shared__ float red[2][4];
-  const int j = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
-  const int lane = d & 31, warp = d >> 5;
-  const float* part = p.part + ((size_t)b * p.n_heads + j) * p.max_splits * kPartStride;
-  const bool ret = p.ret_row[j] >= 0;
-  const int n_splits = p.n_wc + (ret ? p.n_gc : 0);
-  float M = -INFINITY;
-  for (int s = d; s < n_splits; s += RTP_D) M = fmaxf(M, part[s * kPartStride]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if (lane == 0) red[0][warp] = M;
-  __syncthreads();
-  M = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
-  float L = 0.f;
-  for (int s = d; s < n_splits; s += RTP_D) {
-    const float ms = part[s * kPartStride];
-    const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
-    wsm[s] = w;
-    L += w * part[s * kPartStride + 1];
+// Contiguous runs: CTA c takes chunks [run_start(c), run_start(c + 1)) of a
+// list of n chunks (empty runs when there are more CTAs than chunks).
+__device__ __forceinline__ int run_start(int c, int n, int n_ctas) { return (int)((int64_t)c * n / n_ctas); }
+// CTA whose run holds chunk x.
+__device__ __forceinline__ int cta_of(int x, int n, int n_ctas) { return (int)(((int64_t)(x + 1) * n_ctas - 1) / n); }
+// Pieces (runs) of a segment [s0, s0 + len) of a list of n chunks, numbered
+// 0, 1, ... in chunk order. With n_ctas <= n no run is empty and piece i is
+// the i-th CTA from the segment's first; otherwise every run holds at most one
+// chunk and piece i is the segment's chunk i.
+__device__ __forceinline__ int n_pieces(int s0, int len, int n, int n_ctas) {
+  return n_ctas <= n ? cta_of(s0 + len - 1, n, n_ctas) - cta_of(s0, n, n_ctas) + 1 : len;
+}
+__device__ __forceinline__ int piece_of(int cta, int x_first, int s0, int n, int n_ctas) {
+  return n_ctas <= n ? cta - cta_of(s0, n, n_ctas) : x_first - s0;
+}
+
+// Segment of the t-th chunk of a CTA: its window run, then its gathered run.
+struct Seg {
+  int id;        // segment index (window segments first)
+  int b;
+  int gathered;
+  int a;         // active group (window) or retrieval head (gathered)
+  int s0, len;   // first chunk and chunk count of the segment in its list
+  int x;         // the chunk's index in its list
+};
+__device__ __forceinline__ Seg seg_of(const DecodeParams& p, int x, bool gathered) {
+  Seg s;
+  s.x = x;
+  s.gathered = gathered;
+  if (!gathered) {
+    const int sg = x / p.n_wc;
+    s.id = sg; s.b = sg / p.n_ag; s.a = sg - s.b * p.n_ag;
+    s.s0 = sg * p.n_wc; s.len = p.n_wc;
+  } else {
+    const int sg = x / p.n_gc;
+    s.id = p.B * p.n_ag + sg; s.b = sg / p.n_ret; s.a = sg - s.b * p.n_ret;
+    s.s0 = sg * p.n_gc; s.len = p.n_gc;
   }
+  return s;
+}
+
+// Key position of slot `s` (0..127) of a chunk (-1: masked for every row).
+__device__ __forceinline__ int slot_pos(const DecodeParams& p, const Seg& sg, int s) {
+  const int local = sg.x - sg.s0;
+  if (!sg.gathered) {
+    const int u = p.wlo_union + local * kChunk + s;
+    return u < p.whi ? u : -1;
+  }
+  const int j = sg.a;                         // retrieval heads are call heads 0..n_ret-1
+  const int wlo = p.wlo[j];
+  const int n_sink = min(p.sink, wlo);
+  const int e = local * kChunk + s;           // virtual list: sink tokens, then the selected entries
+  if (e < n_sink) return e;
+  if (e - n_sink >= p.topk) return -1;
+  const int u = __ldg(p.idx + ((size_t)sg.b * p.n_ret + j) * p.topk + (e - n_sink));
+  return (u >= p.sink && u < wlo) ? u : -1;
+}
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+decode_attn_kernel(const DecodeParams p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int n_ctas = gridDim.x;
+  const int w0 = run_start(blockIdx.x, p.n_win_chunks, n_ctas);
+  const int n_w = run_start(blockIdx.x + 1, p.n_win_chunks, n_ctas) - w0;
+  const int g0 = p.n_gat_chunks ? run_start(blockIdx.x, p.n_gat_chunks, n_ctas) : 0;
+  const int n_g = p.n_gat_chunks ? run_start(blockIdx.x + 1, p.n_gat_chunks, n_ctas) - g0 : 0;
+  const int n_t = n_w + n_g;                  // this CTA's chunks: window run, then gathered run
+  auto seg_at = [&](int t) { return t < n_w ? seg_of(p, w0 + t, false) : seg_of(p, g0 + t - n_w, true); };
+
+  // this warp's ring and its copies of chunk t into stage t % kStages
+  const uint32_t ring = su32(sm.ring[warp]);
+  auto issue = [&](int t) {
+    if (t < n_t) {
+      const Seg sg = seg_at(t);
+      const int st = t % kStages;
+      const int pos = slot_pos(p, sg, warp * kKeys + lane);   // lane owns row `lane`
+      sm.pos[warp][st][lane] = pos;
+      const int g = sg.gathered ? p.head[sg.a] / p.G : p.ag_kv[sg.a];
+      const __nv_bfloat16* kb = p.k + (int64_t)sg.b * p.k_sb + (int64_t)g * p.k_sh;
+      const __nv_bfloat16* vb = p.v + (int64_t)sg.b * p.v_sb + (int64_t)g * p.v_sh;
+      const uint32_t kdst = ring + (uint32_t)(st * 2) * kSlab, vdst = kdst + kSlab;
+      const int c = lane & 15;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  if (lane == 0) red[1][warp] = L;
-  __syncthreads();
-  L = red[1][0] + red[1][1] + red[1][2] + red[1][3];
-  float acc = 0.f;
+      for (int i = 0; i < kKeys / 2; ++i) {
+        const int r = 2 * i + (lane >> 4);
+        const int pr = __shfl_sync(0xffffffffu, pos, r);
+        const int64_t u = pr >= 0 ? pr : 0;
+        cp_async16(kdst + slab_off(r, c), kb + u * p.k_sn + c * 8, pr >= 0);
+        cp_async16(vdst + slab_off(r, c), vb + u * p.v_sn + c * 8, pr >= 0);
+      }
+    }
+    cp_async_commit();                        // one group per chunk, empty past the run
+  };
+
+  uint32_t qa[8][4];
+  float o[16][4];
+  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+  int ja = -1, jb = -1, lo_a = 0, lo_b = 0;
+  Seg cur;
+  cur.id = -1;
+  int piece_chunks = 0;
+
+  // Combines the four warps' states, writes one partial per row of the
+  // segment and merges every head this piece completes.
+  auto flush = [&]() {
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    // two rounds: warps 2,3 -> 0,1, then warp 1 -> 0
+#pragma unroll 1
+    for (int round = 0; round < 2; ++round) {
+      const int src_lo = round == 0 ? 2 : 1, n_src = round == 0 ? 2 : 1;
+      if (warp >= src_lo && warp < src_lo + n_src) {
+        const int slot = warp - src_lo;
+        if (tq == 0) {
+          sm.cm[slot][gq] = m_a; sm.cm[slot][gq + 8] = m_b;
+          sm.cl[slot][gq] = l_a; sm.cl[slot][gq + 8] = l_b;
+        }
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+          const int col = nt * 8 + 2 * tq;
+          *reinterpret_cast<float2*>(&sm.comb[slot][gq][col]) = make_float2(o[nt][0], o[nt][1]);
+          *reinterpret_cast<float2*>(&sm.comb[slot][gq + 8][col]) = make_float2(o[nt][2], o[nt][3]);
+        }
+      }
+      __syncthreads();
+      if (warp < n_src) {
+        const int slot = warp;
+        const float mpa = sm.cm[slot][gq], mpb = sm.cm[slot][gq + 8];
+        const float Ma = fmaxf(m_a, mpa), Mb = fmaxf(m_b, mpb);
+        const float fa = m_a == -INFINITY ? 0.f : exp2f(m_a - Ma), fpa = mpa == -INFINITY ? 0.f : exp2f(mpa - Ma);
+        const float fb = m_b == -INFINITY ? 0.f : exp2f(m_b - Mb), fpb = mpb == -INFINITY ? 0.f : exp2f(mpb - Mb);
+        l_a = l_a * fa + sm.cl[slot][gq] * fpa;
+        l_b = l_b * fb + sm.cl[slot][gq + 8] * fpb;
+        m_a = Ma; m_b = Mb;
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+          const int col = nt * 8 + 2 * tq;
+          const float2 pa = *reinterpret_cast<const float2*>(&sm.comb[slot][gq][col]);
+          const float2 pb = *reinterpret_cast<const float2*>(&sm.comb[slot][gq + 8][col]);
+          o[nt][0] = o[nt][0] * fa + pa.x * fpa; o[nt][1] = o[nt][1] * fa + pa.y * fpa;
+          o[nt][2] = o[nt][2] * fb + pb.x * fpb; o[nt][3] = o[nt][3] * fb + pb.y * fpb;
+        }
+      }
+      __syncthreads();
+    }
+    if (warp == 0) {
+      // warp 0 holds the piece's state: one partial per row, then the tickets
+      const int n_list = cur.gathered ? p.n_gat_chunks : p.n_win_chunks;
+      int kslot = piece_of((int)blockIdx.x, cur.x, cur.s0, n_list, n_ctas);   // cur.x: the piece's first chunk
+      if (cur.gathered)
+        kslot += n_pieces((cur.b * p.n_ag + p.ag_of[cur.a]) * p.n_wc, p.n_wc, p.n_win_chunks, n_ctas);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int j = half ? jb : ja;
+        if (j < 0) continue;
+        float* part = p.part + (((size_t)cur.b * p.n_heads + j) * p.max_slots + kslot) * kPartStride;
+        if (tq == 0) { part[0] = half ? m_b : m_a; part[1] = half ? l_b : l_a; }
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+          const int col = nt * 8 + 2 * tq;
+          *reinterpret_cast<float2*>(part + kPartO + col) = make_float2(o[nt][half * 2], o[nt][half * 2 + 1]);
+        }
+      }
+      __threadfence();
+      __syncwarp();
+      // lane r (< 16) accounts row r's chunks; the heads it completes are merged below
+      int jr = -1;
+      if (lane < kMaxGroup)
+        jr = cur.gathered ? (lane == 0 ? cur.a : -1) : (lane < p.ag_n[cur.a] ? p.ag_rows[cur.a][lane] : -1);
+      bool done = false;
+      if (jr >= 0) {
+        const int total = p.n_wc + (jr < p.n_ret ? p.n_gc : 0);
+        done = atomicAdd(p.ticket + (size_t)cur.b * p.n_heads + jr, piece_chunks) + piece_chunks == total;
+      }
+      const unsigned todo = __ballot_sync(0xffffffffu, done);
+      if (done) sm.todo[__popc(todo & ((1u << lane) - 1u))] = jr;
+      if (lane == 0) sm.n_todo = __popc(todo);
+      if (todo) __threadfence();
+    }
+    __syncthreads();
+    // every warp merges its share of the completed heads
+    const int n_todo = sm.n_todo;
+    for (int i = warp; i < n_todo; i += kWarps) {
+      const int j = sm.todo[i];
+      // this head's pieces: its window segment's, then its gathered segment's
+      int n = n_pieces((cur.b * p.n_ag + p.ag_of[j]) * p.n_wc, p.n_wc, p.n_win_chunks, n_ctas);
+      if (j < p.n_ret) n += n_pieces((cur.b * p.n_ret + j) * p.n_gc, p.n_gc, p.n_gat_chunks, n_ctas);
+      const float* part = p.part + ((size_t)cur.b * p.n_heads + j) * p.max_slots * kPartStride;
+      float M = -INFINITY;
+      for (int s = lane; s < n; s += 32) M = fmaxf(M, __ldcg(part + s * kPartStride));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+      float Lsum = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s0 = 0; s0 < n; s0 += 32) {
+        // lane s holds piece s0 + s's weight
+        float w = 0.f;
+        if (s0 + lane < n) {
+          const float ms = __ldcg(part + (s0 + lane) * kPartStride);
+          if (ms != -INFINITY) {
+            w = exp2f(ms - M);
+            Lsum += w * __ldcg(part + (s0 + lane) * kPartStride + 1);
+          }
+        }
+        const int cnt = min(32, n - s0);
 #pragma unroll 4
-  for (int s = 0; s < n_splits; ++s) {
-    const float w = wsm[s];
-    if (w != 0.f) acc += w * part[s * kPartStride + 2 + d];
+        for (int s = 0; s < cnt; ++s) {
+          const float ws = __shfl_sync(0xffffffffu, w, s);
+          const float4 v4 = __ldcg(reinterpret_cast<const float4*>(part + (s0 + s) * kPartStride + kPartO) + lane);
+          acc.x += ws * v4.x; acc.y += ws * v4.y; acc.z += ws * v4.z; acc.w += ws * v4.w;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, off);
+      const float inv = 1.f / Lsum;
+      __nv_bfloat16* dst = p.o + (int64_t)cur.b * p.o_sb + (int64_t)p.head[j] * p.o_sh + lane * 4;
+      uint2 packed;
+      packed.x = pack2(acc.x * inv, acc.y * inv);
+      packed.y = pack2(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2*>(dst) = packed;
+    }
+  };
+
+  // prologue: the first kStages - 1 chunks in flight
+#pragma unroll
+  for (int t = 0; t < kStages - 1; ++t) issue(t);
+  for (int t = 0; t < n_t; ++t) {
+    issue(t + kStages - 1);
+    const Seg sg = seg_at(t);
+    if (sg.id != cur.id) {
+      if (cur.id >= 0) flush();
+      cur = sg;
+      piece_chunks = 0;
+      // rows of the tile: the group's heads (window) or the one retrieval head
+      if (sg.gathered) {
+        ja = gq == 0 ? sg.a : -1;
+        jb = -1;
+      } else {
+        ja = gq < p.ag_n[sg.a] ? p.ag_rows[sg.a][gq] : -1;
+        jb = gq + 8 < p.ag_n[sg.a] ? p.ag_rows[sg.a][gq + 8] : -1;
+      }
+      lo_a = ja >= 0 ? (sg.gathered ? 0 : p.wlo[ja]) : 0x7fffffff;
+      lo_b = jb >= 0 ? (sg.gathered ? 0 : p.wlo[jb]) : 0x7fffffff;
+      // query fragments straight from global memory (A operand, 16 x 128)
+      const __nv_bfloat16* qra = p.q + (int64_t)sg.b * p.q_sb + (int64_t)(ja >= 0 ? p.head[ja] : 0) * p.q_sh;
+      const __nv_bfloat16* qrb = p.q + (int64_t)sg.b * p.q_sb + (int64_t)(jb >= 0 ? p.head[jb] : 0) * p.q_sh;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const int c = kk * 16 + 2 * tq;
+        qa[kk][0] = ja >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(qra + c)) : 0u;
+        qa[kk][1] = jb >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(qrb + c)) : 0u;
+        qa[kk][2] = ja >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(qra + c + 8)) : 0u;
+        qa[kk][3] = jb >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(qrb + c + 8)) : 0u;
+      }
+      m_a = m_b = -INFINITY;
+      l_a = l_b = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+    }
+    cp_async_wait<kStages - 1>();               // chunk t has landed (this lane's copies)
+    __syncwarp();                                // ... and every lane's
+    const int st = t % kStages;
+    const uint32_t kbase = ring + (uint32_t)(st * 2) * kSlab, vbase = kbase + kSlab;
+    // S = Q K^T (16 rows x this warp's 32 keys)
+    float sacc[4][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {          // two n-tiles per ldmatrix.x4
+        uint32_t bf[4];
+        const int m = lane >> 3;
+        const int key = 8 * (2 * np + (m >> 1)) + (lane & 7), c = kk * 2 + (m & 1);
+        ldsm_x4(bf, kbase + slab_off(key, c));
+        mma16816(sacc[2 * np], qa[kk], bf[0], bf[1]);
+        mma16816(sacc[2 * np + 1], qa[kk], bf[2], bf[3]);
+      }
+    }
+    // mask, online softmax (rows gq and gq + 8)
+    float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int pos = sm.pos[warp][st][nt * 8 + 2 * tq + e];
+        const bool oka = pos >= 0 && pos >= lo_a;
+        const bool okb = pos >= 0 && pos >= lo_b;
+        sacc[nt][e] = oka ? sacc[nt][e] * p.scale_log2 : -INFINITY;
+        sacc[nt][2 + e] = okb ? sacc[nt][2 + e] * p.scale_log2 : -INFINITY;
+        mx_a = fmaxf(mx_a, sacc[nt][e]);
+        mx_b = fmaxf(mx_b, sacc[nt][2 + e]);
+      }
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+    const float na = fmaxf(m_a, mx_a), nb = fmaxf(m_b, mx_b);
+    const float ra = na == -INFINITY ? 1.f : (m_a == -INFINITY ? 0.f : exp2f(m_a - na));
+    const float rb = nb == -INFINITY ? 1.f : (m_b == -INFINITY ? 0.f : exp2f(m_b - nb));
+    const float base_a = na == -INFINITY ? 0.f : na, base_b = nb == -INFINITY ? 0.f : nb;
+    m_a = na; m_b = nb;
+    l_a *= ra; l_b *= rb;
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      o[nt][0] *= ra; o[nt][1] *= ra;
+      o[nt][2] *= rb; o[nt][3] *= rb;
+    }
+    uint32_t pa[2][4];                          // A fragments of P for the two 16-key steps
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const float e0 = exp2f(sacc[nt][0] - base_a), e1 = exp2f(sacc[nt][1] - base_a);
+      const float e2 = exp2f(sacc[nt][2] - base_b), e3 = exp2f(sacc[nt][3] - base_b);
+      l_a += e0 + e1;
+      l_b += e2 + e3;
+      pa[nt >> 1][(nt & 1) * 2 + 0] = pack2(e0, e1);
+      pa[nt >> 1][(nt & 1) * 2 + 1] = pack2(e2, e3);
+    }
+    // O += P V (16 rows x 128 dims)
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+#pragma unroll
+      for (int np = 0; np < 8; ++np) {
+        uint32_t bf[4];
+        const int m = lane >> 3;
+        const int key = 16 * ks + 8 * (m & 1) + (lane & 7), c = 2 * np + (m >> 1);
+        ldsm_x4_t(bf, vbase + slab_off(key, c));
+        mma16816(o[2 * np], pa[ks], bf[0], bf[1]);
+        mma16816(o[2 * np + 1], pa[ks], bf[2], bf[3]);
+      }
+    }
+    __syncwarp();                                // stage st is free for chunk t + kStages
+    ++piece_chunks;
   }
-  p.o[b * p.o_sb + (int64_t)p.head[j] * p.o_sh + d] = __float2bfloat16_rn(acc / L);
+  cp_async_wait<0>();
+  if (cur.id >= 0) flush();
 }
 
 namespace {
 int n_gathered_chunks(int topk, int sink) { return (topk + sink + kChunk - 1) / kChunk; }
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+size_t ticket_bytes(int B, int n_heads) { return align256((size_t)B * n_heads * sizeof(int)); }
 }  // namespace
 
 size_t decode_attn_ws_bytes(int B, int L, int n_heads, int topk, int window) {
   // `window` bounds every head's window; the sink (at most kMaxSink tokens)
-  // shares the selected list's chunks.
+  // shares the selected list's chunks. A segment is split into at most as
+  // many pieces as it has chunks.
   const int w = window < L ? window : L;
   const int n_wc = (w + kChunk - 1) / kChunk;
   const int n_gc = topk > 0 ? n_gathered_chunks(topk, kMaxSink) : 0;
-  return (size_t)B * n_heads * (n_wc + n_gc) * kPartStride * sizeof(float);
+  return kHeaderBytes + ticket_bytes(B, n_heads) +
+         (size_t)B * n_heads * (n_wc + n_gc) * kPartStride * sizeof(float);
 }
 
 cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
@@ -360,8 +497,8 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
   p.k = static_cast<const __nv_bfloat16*>(kc); p.k_sb = k_sb; p.k_sn = k_sn; p.k_sh = k_sh;
   p.v = static_cast<const __nv_bfloat16*>(vc); p.v_sb = v_sb; p.v_sn = v_sn; p.v_sh = v_sh;
   p.o = static_cast<__nv_bfloat16*>(o); p.o_sb = o_sb; p.o_sh = o_sh;
-  p.B = B; p.L = L; p.q_pos = q_pos; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv;
-  if (p.G > kMaxGroup) return cudaErrorInvalidValue;
+  p.B = B; p.G = Hq / Hkv;
+  if (p.G > kMaxGroup || Hkv > kMaxGroup) return cudaErrorInvalidValue;
   p.idx = idx; p.topk = n_ret > 0 ? topk : 0; p.sink = sink;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.whi = q_pos + 1 < L ? q_pos + 1 : L;
@@ -369,38 +506,56 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
   p.n_ret = n_ret;
   int wlo_union = p.whi;
   for (int r = 0; r < n_ret; ++r) {
-    p.head[r] = ret_heads[r]; p.ret_row[r] = r; p.ret_list[r] = r;
+    p.head[r] = ret_heads[r];
     p.wlo[r] = q_pos - ret_window + 1 > 0 ? q_pos - ret_window + 1 : 0;
     wlo_union = p.wlo[r] < wlo_union ? p.wlo[r] : wlo_union;
   }
   for (int s = 0; s < n_swa; ++s) {
     const int j = n_ret + s;
-    p.head[j] = swa_heads[s]; p.ret_row[j] = -1;
+    p.head[j] = swa_heads[s];
     p.wlo[j] = q_pos - swa_window + 1 > 0 ? q_pos - swa_window + 1 : 0;
     wlo_union = p.wlo[j] < wlo_union ? p.wlo[j] : wlo_union;
+  }
+  // active groups and their rows, in call-head order
+  int group_to_ag[kMaxGroup];
+  for (int g = 0; g < kMaxGroup; ++g) group_to_ag[g] = -1;
+  p.n_ag = 0;
+  for (int j = 0; j < p.n_heads; ++j) {
+    const int g = p.head[j] / p.G;
+    if (group_to_ag[g] < 0) {
+      group_to_ag[g] = p.n_ag;
+      p.ag_kv[p.n_ag] = g;
+      p.ag_n[p.n_ag] = 0;
+      ++p.n_ag;
+    }
+    const int a = group_to_ag[g];
+    if (p.ag_n[a] >= kMaxGroup) return cudaErrorInvalidValue;
+    p.ag_rows[a][p.ag_n[a]++] = j;
+    p.ag_of[j] = a;
   }
   p.wlo_union = wlo_union;
   p.n_wc = (p.whi - wlo_union + kChunk - 1) / kChunk;
   p.n_gc = n_ret > 0 ? n_gathered_chunks(p.topk, sink) : 0;
-  p.max_splits = p.n_wc + p.n_gc;
-  if (Hkv > kMaxGroup) return cudaErrorInvalidValue;
-  p.n_window_items = B * Hkv * p.n_wc;
-  p.part = static_cast<float*>(ws);
-  const int n_items = p.n_window_items + B * n_ret * p.n_gc;
+  p.max_slots = p.n_wc + p.n_gc;
+  p.n_win_chunks = B * p.n_ag * p.n_wc;
+  p.n_gat_chunks = B * n_ret * p.n_gc;
+  char* base = static_cast<char*>(ws);
+  p.ticket = reinterpret_cast<int*>(base + kHeaderBytes);
+  p.part = reinterpret_cast<float*>(base + kHeaderBytes + ticket_bytes(B, p.n_heads));
+  cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes + ticket_bytes(B, p.n_heads), stream);
+  if (e != cudaSuccess) return e;
+  if (p.n_win_chunks == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int most = p.n_win_chunks > p.n_gat_chunks ? p.n_win_chunks : p.n_gat_chunks;
+  const int grid = most < sms ? most : sms;
   const size_t smem = sizeof(Smem);
-  cudaError_t e = cudaFuncSetAttribute(decode_attn_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  e = cudaFuncSetAttribute(decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  decode_attn_partial_kernel<<<n_items, kThreads, smem, stream>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  dim3 g2(p.n_heads, B);
-  const size_t msmem = (size_t)p.max_splits * sizeof(float);
-  if (msmem > 48 * 1024) {
-    e = cudaFuncSetAttribute(decode_attn_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
-    if (e != cudaSuccess) return e;
-  }
-  decode_attn_merge_kernel<<<g2, RTP_D, msmem, stream>>>(p);
+  decode_attn_kernel<<<grid, kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -422,7 +577,7 @@ cudaError_t launch_decode_attn(const void* q, int64_t q_sb, int64_t q_sh,
 }
 
 // ---------------------------------------------------------------------------
-// Allocation-free variant: the split-K partials live in a fixed device array.
+// Allocation-free variant: the workspace is a fixed device array.
 // ---------------------------------------------------------------------------
 // Every GPU that loads the library holds this array until the process exits.
 // Host code must not pass `g_decode_scratch` itself to a kernel (on the host
@@ -460,8 +615,8 @@ cudaError_t launch_decode_attn_noalloc(const void* q, int64_t q_sb, int64_t q_sh
                                        int B, int L, int q_pos, int Hq, int Hkv,
                                        const int32_t* heads, int n_heads, const int32_t* idx, int topk,
                                        int window, int sink, float scale, cudaStream_t stream) {
-  // Every partial the merge reads is written by the same call's partial
-  // kernel, so nothing in the array has to start at zero.
+  // The call clears the array's status word and tickets on the stream; every
+  // partial the kernel reads is written by the same call.
   void* scratch = nullptr;
   cudaError_t e = decode_scratch_address(&scratch);
   if (e != cudaSuccess) return e;

@@ -271,6 +271,30 @@ def run_ours(args, rank, world):
         flush.zero_()
         decode_step(new_events(4))
     torch.cuda.synchronize()
+    # The decode step runs as one CUDA graph (the way a serving loop replays
+    # it): one host launch per step, every kernel of the step inside. Each
+    # call is also captured on its own for the per-kernel breakdown.
+    g_step = step.graph(qd, kc, vc, kindex, Pd, od)
+    d_calls = [
+        lambda: rtp.index_project(qd.unsqueeze(1), Pd, step.ret, step.kv_ret,
+                                  out=step.qt.view(Bd, len(step.ret), 1, R)),
+        lambda: rtp.select_decode(step.qt, kindex, step.kv_ret, step.topk, step.idx, step.ws_sel),
+        lambda: rtp.decode_attn_hybrid(qd, kc, vc, od, step.ret, step.idx, step.ret_window, step.swa_heads,
+                                       step.window, step.sink, step.scale, step.ws_att),
+    ]
+    g_calls = []
+    for fn in d_calls:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        g_calls.append(g)
+    for _ in range(args.warmup):
+        flush.zero_()
+        g_step.replay()
+        for g in g_calls:
+            flush.zero_()
+            g.replay()
+    torch.cuda.synchronize()
 
     # ---- timed region
     clocks = ClockSampler(torch.cuda.current_device())
@@ -284,8 +308,10 @@ def run_ours(args, rank, world):
         prefill_step(e)
         pev.append(e)
         flush.zero_()                       # L2 flush between timed decode steps (not timed)
-        e = new_events(4)
-        decode_step(e)
+        e = new_events(2)
+        e[0].record(stream)
+        g_step.replay()
+        e[1].record(stream)
         dev_ev.append(e)
         flush.zero_()
     torch.cuda.synchronize()
@@ -293,6 +319,21 @@ def run_ours(args, rank, world):
     clk = clocks.stop() if rank == 0 else None
     if layer.device_status() != 0:
         raise RuntimeError("a prefill kernel reported a timed-out wait")
+    if rtp.workspace_status(step.ws_att) != 0:
+        raise RuntimeError("the decode attention reported an error status")
+    # per-call breakdown of the decode step (after the timed region)
+    call_ev = []
+    for _ in range(max(args.steps, 3)):
+        row = []
+        for g in g_calls:
+            flush.zero_()
+            e = new_events(2)
+            e[0].record(stream)
+            g.replay()
+            e[1].record(stream)
+            row.append(e)
+        call_ev.append(row)
+    torch.cuda.synchronize()
 
     def per_call(evs, names):
         tot = {n: 0.0 for n in names}
@@ -302,9 +343,9 @@ def run_ours(args, rank, world):
         return {n: t / len(evs) for n, t in tot.items()}
 
     p_ms = per_call(pev, names_p)
-    d_ms = per_call(dev_ev, names_d)
+    d_ms = {n: sum(r[i][0].elapsed_time(r[i][1]) for r in call_ev) / len(call_ev) for i, n in enumerate(names_d)}
     p_step_ms = sum(p_ms.values())
-    d_step_ms = sum(d_ms.values())
+    d_step_ms = sum(e[0].elapsed_time(e[1]) for e in dev_ev) / len(dev_ev)
     p_step_ms = max_over_ranks(p_step_ms, world)
     d_step_ms = max_over_ranks(d_step_ms, world)
 
@@ -369,7 +410,7 @@ def run_ours(args, rank, world):
     # ---- end to end through the API with host buffers (rank-local, fewer steps)
     e2e = None
     if args.e2e:
-        e2e = run_e2e(args, pcfg, layer, q, k, v, P, o, qd, od, step, kc, vc, kindex, Pd, world, stream)
+        e2e = run_e2e(args, pcfg, layer, q, k, v, P, o, qd, od, g_step, world, stream)
 
     line = {
         "metric": "hybrid-attn prefill tok/s @1M & decode tok/s @128K per layer; % of roofline",
@@ -397,7 +438,7 @@ def run_ours(args, rank, world):
     return line
 
 
-def run_e2e(args, pcfg, layer, q, k, v, P, o, qd, od, step, kc, vc, kindex, Pd, world, stream):
+def run_e2e(args, pcfg, layer, q, k, v, P, o, qd, od, g_step, world, stream):
     """Same metric through the public API with host buffers: every step copies
     its inputs from pinned host memory and reads the result back."""
     import long_context_hybrid_b200 as rtp
@@ -420,7 +461,7 @@ def run_e2e(args, pcfg, layer, q, k, v, P, o, qd, od, step, kc, vc, kindex, Pd, 
 
     def dstep():
         qd.copy_(hqd, non_blocking=True)
-        step(qd, kc, vc, kindex, Pd, od)
+        g_step.replay()                     # DecodeStep.graph: the step captured on qd / od
         hod.copy_(od, non_blocking=True)
 
     steps = max(1, min(args.steps, 2))

@@ -260,18 +260,17 @@ RTP_API rtp_status rtp_decode_attn_hybrid(const void* q, const void* kc, rtp_str
  *   cudaMalloc/cudaFree (both may synchronise the device) on every step.
  *
  *   Arguments, layouts and results are those of rtp_sparse_attn_decode. The
- *   split-K partials, the per-head tickets and the status word go to a fixed
- *   array inside the library, 4 MiB per GPU, held by every GPU that loads the
- *   library until the process exits. A call whose workspace would not fit
- *   (about 512 + 4 * B * Hr + B * Hr * (ceil(window/128) +
- *   ceil((topk+64)/128)) * 528 bytes > 4 MiB) returns RTP_ERR_WORKSPACE and
- *   launches nothing. The first call on a device looks up the array's device
+ *   split-K partials and the status word go to a fixed array inside the
+ *   library, 4 MiB per GPU, held by every GPU that loads the library until
+ *   the process exits. A call whose workspace would not fit (about 256 +
+ *   4 * B * Hr * (ceil(window/64) + ceil((topk+64)/64)) * 528 bytes > 4 MiB)
+ *   returns RTP_ERR_WORKSPACE and launches nothing. The first call on a device looks up the array's device
  *   address (with that device current) and caches it; make that first call
  *   before any stream capture. Every call shares the one array, so calls
  *   whose work may overlap on the GPU (different streams, or concurrent host
  *   threads) race on it and must be serialised by the caller. Nothing in the
- *   array needs to start at zero: each call clears its status word and
- *   tickets on the stream and writes every partial it reads.
+ *   array needs to start at zero: each call writes every partial it reads
+ *   and its status word.
  */
 RTP_API rtp_status rtp_sparse_attn_decode_noalloc(const void* q, const void* kc, rtp_strides ks,
                                                   const void* vc, rtp_strides vs, void* o,

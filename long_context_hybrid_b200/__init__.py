@@ -325,6 +325,19 @@ class DecodeStep:
                            self.swa_heads, self.window, self.sink, self.scale, self.ws_att, stream=stream)
         return o
 
+    def graph(self, q, kc, vc, kindex, P, o) -> "torch.cuda.CUDAGraph":
+        """Captures one step on these buffers into a CUDA graph.
+
+        ``graph.replay()`` then runs the whole step (projection, selection,
+        attention: every kernel, one launch from the host) reading the query
+        currently in ``q`` and writing ``o``; write each new query into ``q``
+        (and append to the cache in place) before replaying. Run the step once
+        eagerly before capturing, so that every kernel attribute is set."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self(q, kc, vc, kindex, P, o)
+        return g
+
 
 __all__ = ["lib", "RtpError", "index_project", "select_prefill", "select_decode",
            "sparse_attn_prefill", "sparse_attn_decode", "swa", "decode_attn_hybrid", "PrefillLayer", "DecodeStep",

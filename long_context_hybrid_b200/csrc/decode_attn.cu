@@ -8,25 +8,25 @@
 //
 // The work is HBM-bound (512 bytes of K and V per attended token), so the
 // design goal is to read every K/V row once and keep enough bytes in flight:
-//   * the work is two lists of 128-key chunks in segments: a window segment
+//   * the work is two lists of 64-key chunks in segments: a window segment
 //     per (sequence, KV group) covers the union of the window, with every
 //     listed query head of the group as one row of a 16 x 128 query tile
 //     (grouped heads share the chunk's K/V; each row masks keys outside its
 //     own window); a gathered segment per (sequence, retrieval head) covers
 //     its sink tokens and selected list (entries inside the window or below
 //     `sink` are masked: those keys come from elsewhere);
-//   * one persistent CTA per SM takes a contiguous run of each list, so both
-//     kinds of chunk are spread evenly. Each of its four warps owns 32 keys of
-//     every chunk: it copies its own K and V rows with 16-byte cp.async
-//     (zero-filled where masked) three chunks ahead into a private ring of
-//     256-byte rows whose 16-byte pieces are XOR-swizzled (conflict-free
-//     ldmatrix), and computes S = Q K^T and O += P V with bf16 mma.sync (fp32
-//     accumulate) and an online softmax carried across the run's chunks of a
-//     segment. The warps never wait for one another inside a segment;
-//   * where a run leaves a segment the four warps combine their states and
-//     write one partial per head (running max in the log2 domain, sum,
-//     o[128]); the CTA that completes a head's chunk count (an atomic ticket)
-//     merges that head's partials and writes its output.
+//   * two persistent CTAs per SM each take a contiguous run of each list, so
+//     both kinds of chunk are spread evenly. Each of a CTA's four warps owns 16
+//     keys of every chunk: it copies its own K and V rows with 16-byte cp.async
+//     (zero-filled where masked) two chunks ahead into a private three-stage
+//     ring of 256-byte rows whose 16-byte pieces are XOR-swizzled
+//     (conflict-free ldmatrix), and computes S = Q K^T and O += P V with bf16
+//     mma.sync (fp32 accumulate) and an online softmax carried across the
+//     run's chunks of a segment. The warps never wait for one another;
+//   * where a run leaves a segment each warp writes its partial of every head
+//     of the segment (running max in the log2 domain, sum, o[128]); a second
+//     kernel, one CTA per head, merges each head's partials and writes its
+//     output.
 #include <mutex>
 
 #include "rtp_common.cuh"
@@ -37,14 +37,16 @@ namespace rtp {
 namespace {
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-constexpr int kChunk = 128;                   // keys per chunk
-constexpr int kKeys = kChunk / kWarps;        // keys per warp and chunk (32)
+constexpr int kCtasPerSm = 2;
+constexpr int kChunk = 64;                    // keys per chunk
+constexpr int kKeys = kChunk / kWarps;        // keys per warp and chunk (16)
 constexpr int kStages = 3;
 constexpr int kRowBytes = RTP_D * 2;          // 256
 constexpr int kSlab = kKeys * kRowBytes;      // one warp's K (or V) rows of one chunk
 constexpr int kPartStride = 4 + RTP_D;        // m, l, 2 pad, o[128] (16-byte aligned rows)
 constexpr int kPartO = 4;
 constexpr int kMaxGroup = 16;                 // query heads per KV group packed in one MMA tile
+constexpr int kMergeBatch = 16;               // partials read at once by a merging warp
 constexpr size_t kHeaderBytes = 256;          // status word (cleared by every call)
 
 struct DecodeParams {
@@ -64,7 +66,6 @@ struct DecodeParams {
   int n_win_chunks;                  // B * n_ag * n_wc
   int n_gat_chunks;                  // B * n_ret * n_gc
   float* part;                       // [B, n_heads, max_slots, kPartStride]
-  int* ticket;                       // [B, n_heads] chunks accounted for
   int head[kMaxHeads];               // query head of each call head
   int wlo[kMaxHeads];                // first position of each call head's window
   int ag_of[kMaxHeads];              // active-group index of each call head
@@ -75,11 +76,7 @@ struct DecodeParams {
 
 struct Smem {
   unsigned char ring[kWarps][kStages][2][kSlab];   // [warp][stage][K, V]
-  float comb[2][kMaxGroup][RTP_D];                 // cross-warp combine buffer
-  float cm[kWarps][kMaxGroup], cl[kWarps][kMaxGroup];
   int pos[kWarps][kStages][kKeys];
-  int todo[kMaxGroup];                             // heads completed by the current flush
-  int n_todo;
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t* r, uint32_t addr) {
@@ -134,50 +131,68 @@ __device__ __forceinline__ int piece_of(int cta, int x_first, int s0, int n, int
   return n_ctas <= n ? cta - cta_of(s0, n, n_ctas) : x_first - s0;
 }
 
-// Segment of the t-th chunk of a CTA: its window run, then its gathered run.
-struct Seg {
-  int id;        // segment index (window segments first)
-  int b;
+// Walks a CTA's chunks: its window run, then its gathered run. Segments:
+// window (sequence-major, then active group), gathered (sequence-major, then
+// retrieval head).
+struct Cursor {
+  int left_w;    // window chunks left after this one (-1: in the gathered run)
+  int x;         // chunk index in its list
+  int local;     // chunk index in its segment
+  int sg;        // segment index in its list
+  int b, a;      // sequence; active group (window) or retrieval head (gathered)
   int gathered;
-  int a;         // active group (window) or retrieval head (gathered)
-  int s0, len;   // first chunk and chunk count of the segment in its list
-  int x;         // the chunk's index in its list
-};
-__device__ __forceinline__ Seg seg_of(const DecodeParams& p, int x, bool gathered) {
-  Seg s;
-  s.x = x;
-  s.gathered = gathered;
-  if (!gathered) {
-    const int sg = x / p.n_wc;
-    s.id = sg; s.b = sg / p.n_ag; s.a = sg - s.b * p.n_ag;
-    s.s0 = sg * p.n_wc; s.len = p.n_wc;
-  } else {
-    const int sg = x / p.n_gc;
-    s.id = p.B * p.n_ag + sg; s.b = sg / p.n_ret; s.a = sg - s.b * p.n_ret;
-    s.s0 = sg * p.n_gc; s.len = p.n_gc;
+  __device__ int id(const DecodeParams& p) const { return gathered ? p.B * p.n_ag + sg : sg; }
+  __device__ int s0() const { return x - local; }
+  __device__ void at(const DecodeParams& p, int x_, int gathered_) {
+    x = x_;
+    gathered = gathered_;
+    const int len = gathered ? p.n_gc : p.n_wc, A = gathered ? p.n_ret : p.n_ag;
+    sg = x / len; local = x - sg * len;
+    b = sg / A; a = sg - b * A;
   }
-  return s;
-}
+  __device__ void next(const DecodeParams& p, int g0) {
+    if (left_w == 0) {
+      left_w = -1;
+      if (p.n_gat_chunks > 0) at(p, g0, 1);
+      return;
+    }
+    if (left_w > 0) --left_w;
+    ++x;
+    const int len = gathered ? p.n_gc : p.n_wc, A = gathered ? p.n_ret : p.n_ag;
+    if (++local == len) {
+      local = 0; ++sg;
+      if (++a == A) { a = 0; ++b; }
+    }
+  }
+};
 
-// Key position of slot `s` (0..127) of a chunk (-1: masked for every row).
-__device__ __forceinline__ int slot_pos(const DecodeParams& p, const Seg& sg, int s) {
-  const int local = sg.x - sg.s0;
-  if (!sg.gathered) {
-    const int u = p.wlo_union + local * kChunk + s;
+// Key position of slot `s` (0..kChunk-1) of the cursor's chunk (-1: masked
+// for every row), in two steps so that the selected-list read can be issued
+// a chunk early: slot_fetch reads what the position depends on, slot_pos
+// turns it into the position.
+__device__ __forceinline__ int slot_fetch(const DecodeParams& p, const Cursor& c, int s) {
+  if (!c.gathered) return 0;
+  const int j = c.a;                          // retrieval heads are call heads 0..n_ret-1
+  const int n_sink = min(p.sink, p.wlo[j]);
+  const int e = c.local * kChunk + s;         // virtual list: sink tokens, then the selected entries
+  if (e < n_sink || e - n_sink >= p.topk) return -1;
+  return __ldg(p.idx + ((size_t)c.b * p.n_ret + j) * p.topk + (e - n_sink));
+}
+__device__ __forceinline__ int slot_pos(const DecodeParams& p, const Cursor& c, int s, int fetched) {
+  if (!c.gathered) {
+    const int u = p.wlo_union + c.local * kChunk + s;
     return u < p.whi ? u : -1;
   }
-  const int j = sg.a;                         // retrieval heads are call heads 0..n_ret-1
-  const int wlo = p.wlo[j];
+  const int wlo = p.wlo[c.a];
   const int n_sink = min(p.sink, wlo);
-  const int e = local * kChunk + s;           // virtual list: sink tokens, then the selected entries
+  const int e = c.local * kChunk + s;
   if (e < n_sink) return e;
   if (e - n_sink >= p.topk) return -1;
-  const int u = __ldg(p.idx + ((size_t)sg.b * p.n_ret + j) * p.topk + (e - n_sink));
-  return (u >= p.sink && u < wlo) ? u : -1;
+  return (fetched >= p.sink && fetched < wlo) ? fetched : -1;
 }
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 decode_attn_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
@@ -189,29 +204,39 @@ decode_attn_kernel(const DecodeParams p) {
   const int g0 = p.n_gat_chunks ? run_start(blockIdx.x, p.n_gat_chunks, n_ctas) : 0;
   const int n_g = p.n_gat_chunks ? run_start(blockIdx.x + 1, p.n_gat_chunks, n_ctas) - g0 : 0;
   const int n_t = n_w + n_g;                  // this CTA's chunks: window run, then gathered run
-  auto seg_at = [&](int t) { return t < n_w ? seg_of(p, w0 + t, false) : seg_of(p, g0 + t - n_w, true); };
+  if (n_t == 0) return;
+  Cursor first;
+  first.left_w = n_w > 0 ? n_w - 1 : -1;
+  first.at(p, n_w > 0 ? w0 : g0, n_w > 0 ? 0 : 1);
 
-  // this warp's ring and its copies of chunk t into stage t % kStages
+  // this warp's ring and its copies of a chunk into stage st
   const uint32_t ring = su32(sm.ring[warp]);
+  Cursor icur = first;                        // next chunk to copy
+  const int my_slot = warp * kKeys + (lane & (kKeys - 1));
+  int fetched = slot_fetch(p, icur, my_slot);  // for the next chunk to copy
   auto issue = [&](int t) {
     if (t < n_t) {
-      const Seg sg = seg_at(t);
       const int st = t % kStages;
-      const int pos = slot_pos(p, sg, warp * kKeys + lane);   // lane owns row `lane`
-      sm.pos[warp][st][lane] = pos;
-      const int g = sg.gathered ? p.head[sg.a] / p.G : p.ag_kv[sg.a];
-      const __nv_bfloat16* kb = p.k + (int64_t)sg.b * p.k_sb + (int64_t)g * p.k_sh;
-      const __nv_bfloat16* vb = p.v + (int64_t)sg.b * p.v_sb + (int64_t)g * p.v_sh;
+      const int g = icur.gathered ? p.head[icur.a] / p.G : p.ag_kv[icur.a];
+      // lane r < kKeys owns row r: its position and its K/V row addresses
+      const int pos = slot_pos(p, icur, my_slot, fetched);
+      if (lane < kKeys) sm.pos[warp][st][lane] = pos;
+      const int64_t u = pos >= 0 ? pos : 0;
+      const char* krow = reinterpret_cast<const char*>(p.k + (int64_t)icur.b * p.k_sb + (int64_t)g * p.k_sh + u * p.k_sn);
+      const char* vrow = reinterpret_cast<const char*>(p.v + (int64_t)icur.b * p.v_sb + (int64_t)g * p.v_sh + u * p.v_sn);
       const uint32_t kdst = ring + (uint32_t)(st * 2) * kSlab, vdst = kdst + kSlab;
       const int c = lane & 15;
 #pragma unroll
       for (int i = 0; i < kKeys / 2; ++i) {
         const int r = 2 * i + (lane >> 4);
-        const int pr = __shfl_sync(0xffffffffu, pos, r);
-        const int64_t u = pr >= 0 ? pr : 0;
-        cp_async16(kdst + slab_off(r, c), kb + u * p.k_sn + c * 8, pr >= 0);
-        cp_async16(vdst + slab_off(r, c), vb + u * p.v_sn + c * 8, pr >= 0);
+        const bool ok = __shfl_sync(0xffffffffu, pos, r) >= 0;
+        const char* ks = reinterpret_cast<const char*>(__shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(krow), r));
+        const char* vs = reinterpret_cast<const char*>(__shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(vrow), r));
+        cp_async16(kdst + slab_off(r, c), ks + c * 16, ok);
+        cp_async16(vdst + slab_off(r, c), vs + c * 16, ok);
       }
+      icur.next(p, g0);
+      if (t + 1 < n_t) fetched = slot_fetch(p, icur, my_slot);
     }
     cp_async_commit();                        // one group per chunk, empty past the run
   };
@@ -220,156 +245,59 @@ decode_attn_kernel(const DecodeParams p) {
   float o[16][4];
   float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
   int ja = -1, jb = -1, lo_a = 0, lo_b = 0;
-  Seg cur;
-  cur.id = -1;
-  int piece_chunks = 0;
+  Cursor cur = first;                         // chunk being computed
+  int cur_id = -1, piece_b = 0, piece_a = 0, piece_x = 0, piece_s0 = 0, piece_gathered = 0, piece_chunks = 0;
 
-  // Combines the four warps' states, writes one partial per row of the
-  // segment and merges every head this piece completes.
+  // Writes this warp's partial of every row of the segment (its keys of the
+  // run's chunks in the segment).
   auto flush = [&]() {
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-    // two rounds: warps 2,3 -> 0,1, then warp 1 -> 0
-#pragma unroll 1
-    for (int round = 0; round < 2; ++round) {
-      const int src_lo = round == 0 ? 2 : 1, n_src = round == 0 ? 2 : 1;
-      if (warp >= src_lo && warp < src_lo + n_src) {
-        const int slot = warp - src_lo;
-        if (tq == 0) {
-          sm.cm[slot][gq] = m_a; sm.cm[slot][gq + 8] = m_b;
-          sm.cl[slot][gq] = l_a; sm.cl[slot][gq + 8] = l_b;
-        }
+    const int n_list = piece_gathered ? p.n_gat_chunks : p.n_win_chunks;
+    int piece = piece_of((int)blockIdx.x, piece_x, piece_s0, n_list, n_ctas);
+    if (piece_gathered)
+      piece += n_pieces((piece_b * p.n_ag + p.ag_of[piece_a]) * p.n_wc, p.n_wc, p.n_win_chunks, n_ctas);
+    const int kslot = piece * kWarps + warp;
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-          const int col = nt * 8 + 2 * tq;
-          *reinterpret_cast<float2*>(&sm.comb[slot][gq][col]) = make_float2(o[nt][0], o[nt][1]);
-          *reinterpret_cast<float2*>(&sm.comb[slot][gq + 8][col]) = make_float2(o[nt][2], o[nt][3]);
-        }
+    for (int half = 0; half < 2; ++half) {
+      const int j = half ? jb : ja;
+      if (j < 0) continue;
+      float* part = p.part + (((size_t)piece_b * p.n_heads + j) * p.max_slots + kslot) * kPartStride;
+      if (tq == 0) { part[0] = half ? m_b : m_a; part[1] = half ? l_b : l_a; }
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        const int col = nt * 8 + 2 * tq;
+        *reinterpret_cast<float2*>(part + kPartO + col) = make_float2(o[nt][half * 2], o[nt][half * 2 + 1]);
       }
-      __syncthreads();
-      if (warp < n_src) {
-        const int slot = warp;
-        const float mpa = sm.cm[slot][gq], mpb = sm.cm[slot][gq + 8];
-        const float Ma = fmaxf(m_a, mpa), Mb = fmaxf(m_b, mpb);
-        const float fa = m_a == -INFINITY ? 0.f : exp2f(m_a - Ma), fpa = mpa == -INFINITY ? 0.f : exp2f(mpa - Ma);
-        const float fb = m_b == -INFINITY ? 0.f : exp2f(m_b - Mb), fpb = mpb == -INFINITY ? 0.f : exp2f(mpb - Mb);
-        l_a = l_a * fa + sm.cl[slot][gq] * fpa;
-        l_b = l_b * fb + sm.cl[slot][gq + 8] * fpb;
-        m_a = Ma; m_b = Mb;
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-          const int col = nt * 8 + 2 * tq;
-          const float2 pa = *reinterpret_cast<const float2*>(&sm.comb[slot][gq][col]);
-          const float2 pb = *reinterpret_cast<const float2*>(&sm.comb[slot][gq + 8][col]);
-          o[nt][0] = o[nt][0] * fa + pa.x * fpa; o[nt][1] = o[nt][1] * fa + pa.y * fpa;
-          o[nt][2] = o[nt][2] * fb + pb.x * fpb; o[nt][3] = o[nt][3] * fb + pb.y * fpb;
-        }
-      }
-      __syncthreads();
-    }
-    if (warp == 0) {
-      // warp 0 holds the piece's state: one partial per row, then the tickets
-      const int n_list = cur.gathered ? p.n_gat_chunks : p.n_win_chunks;
-      int kslot = piece_of((int)blockIdx.x, cur.x, cur.s0, n_list, n_ctas);   // cur.x: the piece's first chunk
-      if (cur.gathered)
-        kslot += n_pieces((cur.b * p.n_ag + p.ag_of[cur.a]) * p.n_wc, p.n_wc, p.n_win_chunks, n_ctas);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int j = half ? jb : ja;
-        if (j < 0) continue;
-        float* part = p.part + (((size_t)cur.b * p.n_heads + j) * p.max_slots + kslot) * kPartStride;
-        if (tq == 0) { part[0] = half ? m_b : m_a; part[1] = half ? l_b : l_a; }
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-          const int col = nt * 8 + 2 * tq;
-          *reinterpret_cast<float2*>(part + kPartO + col) = make_float2(o[nt][half * 2], o[nt][half * 2 + 1]);
-        }
-      }
-      __threadfence();
-      __syncwarp();
-      // lane r (< 16) accounts row r's chunks; the heads it completes are merged below
-      int jr = -1;
-      if (lane < kMaxGroup)
-        jr = cur.gathered ? (lane == 0 ? cur.a : -1) : (lane < p.ag_n[cur.a] ? p.ag_rows[cur.a][lane] : -1);
-      bool done = false;
-      if (jr >= 0) {
-        const int total = p.n_wc + (jr < p.n_ret ? p.n_gc : 0);
-        done = atomicAdd(p.ticket + (size_t)cur.b * p.n_heads + jr, piece_chunks) + piece_chunks == total;
-      }
-      const unsigned todo = __ballot_sync(0xffffffffu, done);
-      if (done) sm.todo[__popc(todo & ((1u << lane) - 1u))] = jr;
-      if (lane == 0) sm.n_todo = __popc(todo);
-      if (todo) __threadfence();
-    }
-    __syncthreads();
-    // every warp merges its share of the completed heads
-    const int n_todo = sm.n_todo;
-    for (int i = warp; i < n_todo; i += kWarps) {
-      const int j = sm.todo[i];
-      // this head's pieces: its window segment's, then its gathered segment's
-      int n = n_pieces((cur.b * p.n_ag + p.ag_of[j]) * p.n_wc, p.n_wc, p.n_win_chunks, n_ctas);
-      if (j < p.n_ret) n += n_pieces((cur.b * p.n_ret + j) * p.n_gc, p.n_gc, p.n_gat_chunks, n_ctas);
-      const float* part = p.part + ((size_t)cur.b * p.n_heads + j) * p.max_slots * kPartStride;
-      float M = -INFINITY;
-      for (int s = lane; s < n; s += 32) M = fmaxf(M, __ldcg(part + s * kPartStride));
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-      float Lsum = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s0 = 0; s0 < n; s0 += 32) {
-        // lane s holds piece s0 + s's weight
-        float w = 0.f;
-        if (s0 + lane < n) {
-          const float ms = __ldcg(part + (s0 + lane) * kPartStride);
-          if (ms != -INFINITY) {
-            w = exp2f(ms - M);
-            Lsum += w * __ldcg(part + (s0 + lane) * kPartStride + 1);
-          }
-        }
-        const int cnt = min(32, n - s0);
-#pragma unroll 4
-        for (int s = 0; s < cnt; ++s) {
-          const float ws = __shfl_sync(0xffffffffu, w, s);
-          const float4 v4 = __ldcg(reinterpret_cast<const float4*>(part + (s0 + s) * kPartStride + kPartO) + lane);
-          acc.x += ws * v4.x; acc.y += ws * v4.y; acc.z += ws * v4.z; acc.w += ws * v4.w;
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, off);
-      const float inv = 1.f / Lsum;
-      __nv_bfloat16* dst = p.o + (int64_t)cur.b * p.o_sb + (int64_t)p.head[j] * p.o_sh + lane * 4;
-      uint2 packed;
-      packed.x = pack2(acc.x * inv, acc.y * inv);
-      packed.y = pack2(acc.z * inv, acc.w * inv);
-      *reinterpret_cast<uint2*>(dst) = packed;
     }
   };
 
   // prologue: the first kStages - 1 chunks in flight
 #pragma unroll
   for (int t = 0; t < kStages - 1; ++t) issue(t);
-  for (int t = 0; t < n_t; ++t) {
+  for (int t = 0; t < n_t; ++t, cur.next(p, g0)) {
     issue(t + kStages - 1);
-    const Seg sg = seg_at(t);
-    if (sg.id != cur.id) {
-      if (cur.id >= 0) flush();
-      cur = sg;
+    const int id = cur.id(p);
+    if (id != cur_id) {
+      if (cur_id >= 0) flush();
+      cur_id = id;
+      piece_b = cur.b; piece_a = cur.a; piece_x = cur.x; piece_s0 = cur.s0(); piece_gathered = cur.gathered;
       piece_chunks = 0;
       // rows of the tile: the group's heads (window) or the one retrieval head
-      if (sg.gathered) {
-        ja = gq == 0 ? sg.a : -1;
+      if (cur.gathered) {
+        ja = gq == 0 ? cur.a : -1;
         jb = -1;
       } else {
-        ja = gq < p.ag_n[sg.a] ? p.ag_rows[sg.a][gq] : -1;
-        jb = gq + 8 < p.ag_n[sg.a] ? p.ag_rows[sg.a][gq + 8] : -1;
+        ja = gq < p.ag_n[cur.a] ? p.ag_rows[cur.a][gq] : -1;
+        jb = gq + 8 < p.ag_n[cur.a] ? p.ag_rows[cur.a][gq + 8] : -1;
       }
-      lo_a = ja >= 0 ? (sg.gathered ? 0 : p.wlo[ja]) : 0x7fffffff;
-      lo_b = jb >= 0 ? (sg.gathered ? 0 : p.wlo[jb]) : 0x7fffffff;
+      lo_a = ja >= 0 ? (cur.gathered ? 0 : p.wlo[ja]) : 0x7fffffff;
+      lo_b = jb >= 0 ? (cur.gathered ? 0 : p.wlo[jb]) : 0x7fffffff;
       // query fragments straight from global memory (A operand, 16 x 128)
-      const __nv_bfloat16* qra = p.q + (int64_t)sg.b * p.q_sb + (int64_t)(ja >= 0 ? p.head[ja] : 0) * p.q_sh;
-      const __nv_bfloat16* qrb = p.q + (int64_t)sg.b * p.q_sb + (int64_t)(jb >= 0 ? p.head[jb] : 0) * p.q_sh;
+      const __nv_bfloat16* qra = p.q + (int64_t)cur.b * p.q_sb + (int64_t)(ja >= 0 ? p.head[ja] : 0) * p.q_sh;
+      const __nv_bfloat16* qrb = p.q + (int64_t)cur.b * p.q_sb + (int64_t)(jb >= 0 ? p.head[jb] : 0) * p.q_sh;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const int c = kk * 16 + 2 * tq;
@@ -389,28 +317,27 @@ decode_attn_kernel(const DecodeParams p) {
     __syncwarp();                                // ... and every lane's
     const int st = t % kStages;
     const uint32_t kbase = ring + (uint32_t)(st * 2) * kSlab, vbase = kbase + kSlab;
-    // S = Q K^T (16 rows x this warp's 32 keys)
-    float sacc[4][4];
+    // S = Q K^T (16 rows x this warp's 16 keys: two n-tiles per ldmatrix.x4)
+    float sacc[2][4];
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+    {
+      const int m = lane >> 3;
+      const int key = 8 * (m >> 1) + (lane & 7);
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-      for (int np = 0; np < 2; ++np) {          // two n-tiles per ldmatrix.x4
+      for (int kk = 0; kk < 8; ++kk) {
         uint32_t bf[4];
-        const int m = lane >> 3;
-        const int key = 8 * (2 * np + (m >> 1)) + (lane & 7), c = kk * 2 + (m & 1);
-        ldsm_x4(bf, kbase + slab_off(key, c));
-        mma16816(sacc[2 * np], qa[kk], bf[0], bf[1]);
-        mma16816(sacc[2 * np + 1], qa[kk], bf[2], bf[3]);
+        ldsm_x4(bf, kbase + slab_off(key, kk * 2 + (m & 1)));
+        mma16816(sacc[0], qa[kk], bf[0], bf[1]);
+        mma16816(sacc[1], qa[kk], bf[2], bf[3]);
       }
     }
     // mask, online softmax (rows gq and gq + 8)
     float mx_a = -INFINITY, mx_b = -INFINITY;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int pos = sm.pos[warp][st][nt * 8 + 2 * tq + e];
@@ -425,51 +352,120 @@ decode_attn_kernel(const DecodeParams p) {
     mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
     mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
     mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-    const float na = fmaxf(m_a, mx_a), nb = fmaxf(m_b, mx_b);
-    const float ra = na == -INFINITY ? 1.f : (m_a == -INFINITY ? 0.f : exp2f(m_a - na));
-    const float rb = nb == -INFINITY ? 1.f : (m_b == -INFINITY ? 0.f : exp2f(m_b - nb));
-    const float base_a = na == -INFINITY ? 0.f : na, base_b = nb == -INFINITY ? 0.f : nb;
-    m_a = na; m_b = nb;
-    l_a *= ra; l_b *= rb;
+    // the running max only moves up: rescale O and l when it does
+    if (mx_a > m_a || mx_b > m_b) {
+      const float na = fmaxf(m_a, mx_a), nb = fmaxf(m_b, mx_b);
+      const float ra = m_a == -INFINITY ? 0.f : exp2f(m_a - na);
+      const float rb = m_b == -INFINITY ? 0.f : exp2f(m_b - nb);
+      m_a = na; m_b = nb;
+      l_a *= ra; l_b *= rb;
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      o[nt][0] *= ra; o[nt][1] *= ra;
-      o[nt][2] *= rb; o[nt][3] *= rb;
+      for (int nt = 0; nt < 16; ++nt) {
+        o[nt][0] *= ra; o[nt][1] *= ra;
+        o[nt][2] *= rb; o[nt][3] *= rb;
+      }
     }
-    uint32_t pa[2][4];                          // A fragments of P for the two 16-key steps
+    const float base_a = m_a == -INFINITY ? 0.f : m_a, base_b = m_b == -INFINITY ? 0.f : m_b;
+    uint32_t pa[4];                             // A fragment of P (16 rows x 16 keys)
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
+    for (int nt = 0; nt < 2; ++nt) {
       const float e0 = exp2f(sacc[nt][0] - base_a), e1 = exp2f(sacc[nt][1] - base_a);
       const float e2 = exp2f(sacc[nt][2] - base_b), e3 = exp2f(sacc[nt][3] - base_b);
       l_a += e0 + e1;
       l_b += e2 + e3;
-      pa[nt >> 1][(nt & 1) * 2 + 0] = pack2(e0, e1);
-      pa[nt >> 1][(nt & 1) * 2 + 1] = pack2(e2, e3);
+      pa[nt * 2 + 0] = pack2(e0, e1);
+      pa[nt * 2 + 1] = pack2(e2, e3);
     }
     // O += P V (16 rows x 128 dims)
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
+    {
+      const int m = lane >> 3;
+      const int key = 8 * (m & 1) + (lane & 7);
 #pragma unroll
       for (int np = 0; np < 8; ++np) {
         uint32_t bf[4];
-        const int m = lane >> 3;
-        const int key = 16 * ks + 8 * (m & 1) + (lane & 7), c = 2 * np + (m >> 1);
-        ldsm_x4_t(bf, vbase + slab_off(key, c));
-        mma16816(o[2 * np], pa[ks], bf[0], bf[1]);
-        mma16816(o[2 * np + 1], pa[ks], bf[2], bf[3]);
+        ldsm_x4_t(bf, vbase + slab_off(key, 2 * np + (m >> 1)));
+        mma16816(o[2 * np], pa, bf[0], bf[1]);
+        mma16816(o[2 * np + 1], pa, bf[2], bf[3]);
       }
     }
     __syncwarp();                                // stage st is free for chunk t + kStages
     ++piece_chunks;
   }
   cp_async_wait<0>();
-  if (cur.id >= 0) flush();
+  if (cur_id >= 0) flush();
+}
+
+// One CTA per (sequence, call head): combines the head's partials (kWarps
+// per piece of its window segment, then of its gathered segment) and writes
+// o. Warp w takes every kWarps-th partial, reading up to kMergeBatch of them
+// with all loads in flight; the four warps then combine through shared memory.
+__global__ void __launch_bounds__(128)
+decode_merge_kernel(const DecodeParams p, int n_ctas, int* status) {
+  __shared__ float wm[4], wl[4];
+  __shared__ float4 wo[4][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+  const int b = blockIdx.x / p.n_heads, j = blockIdx.x - b * p.n_heads;
+  int n = n_pieces((b * p.n_ag + p.ag_of[j]) * p.n_wc, p.n_wc, p.n_win_chunks, n_ctas);
+  if (j < p.n_ret) n += n_pieces((b * p.n_ret + j) * p.n_gc, p.n_gc, p.n_gat_chunks, n_ctas);
+  n *= kWarps;
+  const float* part = p.part + ((size_t)b * p.n_heads + j) * p.max_slots * kPartStride;
+  float M = -INFINITY, Lsum = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = warp; s0 < n; s0 += 4 * kMergeBatch) {
+    float ms[kMergeBatch], ls[kMergeBatch];
+    float4 os[kMergeBatch];
+#pragma unroll
+    for (int s = 0; s < kMergeBatch; ++s) {
+      const int slot = s0 + 4 * s;
+      if (slot < n) {
+        const float* ps = part + (size_t)slot * kPartStride;
+        ms[s] = ps[0];
+        ls[s] = ps[1];
+        os[s] = reinterpret_cast<const float4*>(ps + kPartO)[lane];
+      } else {
+        ms[s] = -INFINITY; ls[s] = 0.f; os[s] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    float Mb = M;
+#pragma unroll
+    for (int s = 0; s < kMergeBatch; ++s) Mb = fmaxf(Mb, ms[s]);
+    if (Mb == -INFINITY) continue;
+    const float r = M == -INFINITY ? 0.f : exp2f(M - Mb);
+    Lsum *= r; acc.x *= r; acc.y *= r; acc.z *= r; acc.w *= r;
+#pragma unroll
+    for (int s = 0; s < kMergeBatch; ++s) {
+      const float wt = ms[s] == -INFINITY ? 0.f : exp2f(ms[s] - Mb);
+      Lsum += wt * ls[s];
+      acc.x += wt * os[s].x; acc.y += wt * os[s].y; acc.z += wt * os[s].z; acc.w += wt * os[s].w;
+    }
+    M = Mb;
+  }
+  if (lane == 0) { wm[warp] = M; wl[warp] = Lsum; }
+  wo[warp][lane] = acc;
+  __syncthreads();
+  if (warp != 0) return;
+  const float Mt = fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3]));
+  float Lt = 0.f;
+  float4 at = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const float f = wm[w] == -INFINITY ? 0.f : exp2f(wm[w] - Mt);
+    Lt += f * wl[w];
+    const float4 v = wo[w][lane];
+    at.x += f * v.x; at.y += f * v.y; at.z += f * v.z; at.w += f * v.w;
+  }
+  const float inv = 1.f / Lt;
+  __nv_bfloat16* dst = p.o + (int64_t)b * p.o_sb + (int64_t)p.head[j] * p.o_sh + lane * 4;
+  uint2 packed;
+  packed.x = pack2(at.x * inv, at.y * inv);
+  packed.y = pack2(at.z * inv, at.w * inv);
+  *reinterpret_cast<uint2*>(dst) = packed;
 }
 
 namespace {
 int n_gathered_chunks(int topk, int sink) { return (topk + sink + kChunk - 1) / kChunk; }
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-size_t ticket_bytes(int B, int n_heads) { return align256((size_t)B * n_heads * sizeof(int)); }
 }  // namespace
 
 size_t decode_attn_ws_bytes(int B, int L, int n_heads, int topk, int window) {
@@ -479,8 +475,8 @@ size_t decode_attn_ws_bytes(int B, int L, int n_heads, int topk, int window) {
   const int w = window < L ? window : L;
   const int n_wc = (w + kChunk - 1) / kChunk;
   const int n_gc = topk > 0 ? n_gathered_chunks(topk, kMaxSink) : 0;
-  return kHeaderBytes + ticket_bytes(B, n_heads) +
-         (size_t)B * n_heads * (n_wc + n_gc) * kPartStride * sizeof(float);
+  return kHeaderBytes +
+         (size_t)B * n_heads * kWarps * (n_wc + n_gc) * kPartStride * sizeof(float);
 }
 
 cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
@@ -536,14 +532,13 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
   p.wlo_union = wlo_union;
   p.n_wc = (p.whi - wlo_union + kChunk - 1) / kChunk;
   p.n_gc = n_ret > 0 ? n_gathered_chunks(p.topk, sink) : 0;
-  p.max_slots = p.n_wc + p.n_gc;
+  p.max_slots = kWarps * (p.n_wc + p.n_gc);
   p.n_win_chunks = B * p.n_ag * p.n_wc;
   p.n_gat_chunks = B * n_ret * p.n_gc;
   char* base = static_cast<char*>(ws);
-  p.ticket = reinterpret_cast<int*>(base + kHeaderBytes);
-  p.part = reinterpret_cast<float*>(base + kHeaderBytes + ticket_bytes(B, p.n_heads));
-  cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes + ticket_bytes(B, p.n_heads), stream);
-  if (e != cudaSuccess) return e;
+  p.part = reinterpret_cast<float*>(base + kHeaderBytes);
+  int* status = reinterpret_cast<int*>(base);
+  cudaError_t e;
   if (p.n_win_chunks == 0) return cudaSuccess;
   int dev = 0, sms = 148;
   e = cudaGetDevice(&dev);
@@ -551,11 +546,14 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const int most = p.n_win_chunks > p.n_gat_chunks ? p.n_win_chunks : p.n_gat_chunks;
-  const int grid = most < sms ? most : sms;
+  const int grid = most < kCtasPerSm * sms ? most : kCtasPerSm * sms;
   const size_t smem = sizeof(Smem);
   e = cudaFuncSetAttribute(decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   decode_attn_kernel<<<grid, kThreads, smem, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_merge_kernel<<<B * p.n_heads, 128, 0, stream>>>(p, grid, status);
   return cudaGetLastError();
 }
 
@@ -615,8 +613,8 @@ cudaError_t launch_decode_attn_noalloc(const void* q, int64_t q_sb, int64_t q_sh
                                        int B, int L, int q_pos, int Hq, int Hkv,
                                        const int32_t* heads, int n_heads, const int32_t* idx, int topk,
                                        int window, int sink, float scale, cudaStream_t stream) {
-  // The call clears the array's status word and tickets on the stream; every
-  // partial the kernel reads is written by the same call.
+  // Every partial the merge reads is written by the same call, and the merge
+  // writes the status word.
   void* scratch = nullptr;
   cudaError_t e = decode_scratch_address(&scratch);
   if (e != cudaSuccess) return e;

@@ -359,6 +359,20 @@ def test_e2e_decode_reduced():
             outs.append(_f64(o[b, h].cpu()))
             refs.append(res["out"][h])
     assert_attn_close(np.stack(outs), np.stack(refs), "decode")
+    # the same step captured as a CUDA graph and replayed with a new query
+    o_eager = o.clone()
+    g = step.graph(q, kc, vc, kindex, P, o)
+    o.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_eager), "graph replay differs from the eager step"
+    q2 = synth.make_decode(cfg, device=DEV, B=B, L=L, seed=cfg.seed + 1)["q"]
+    q.copy_(q2)
+    g.replay()
+    o2 = torch.zeros_like(o)
+    step(q2, kc, vc, kindex, P, o2)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2), "graph replay with a new query differs from the eager step"
 
 
 @pytest.mark.parametrize("L,ret_window,swa_window,topk", [(6000, 512, 256, 300), (6000, 256, 1024, 129),

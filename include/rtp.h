@@ -165,7 +165,8 @@ RTP_API rtp_status rtp_select_prefill(const void* qt, const void* kt, int B, int
  *   idx      int32 [B, Hr, topk] device out: ascending token indices;
  *            min(k, L) of them, the rest -1.
  *   ws       workspace of rtp_workspace_size_select_decode() bytes.
- *   r = 16, 1 <= topk <= 4096, L >= 1.
+ *   r = 16, 1 <= topk <= 4096, L >= 1; Hkv <= 16 and at most 16 retrieval
+ *   heads per KV group (RTP_ERR_UNSUPPORTED otherwise).
  */
 RTP_API size_t rtp_workspace_size_select_decode(int B, int L, int Hr, int topk);
 RTP_API rtp_status rtp_select_decode(const float* qt, const void* kindex, int B, int L, int Hr, int Hkv,

@@ -133,6 +133,12 @@ rtp_status rtp_select_decode(const float* qt, const void* kindex, int B, int L, 
   if (!aligned16(qt) || !aligned16(kindex) || !aligned16(idx)) return RTP_ERR_INVALID_ARG;
   for (int j = 0; j < Hr; ++j)
     if (kv_of[j] < 0 || kv_of[j] >= Hkv) return RTP_ERR_INVALID_ARG;
+  if (Hkv > 16) return RTP_ERR_UNSUPPORTED;
+  for (int g = 0; g < Hkv; ++g) {
+    int c = 0;
+    for (int j = 0; j < Hr; ++j) c += kv_of[j] == g;
+    if (c > 16) return RTP_ERR_UNSUPPORTED;
+  }
   const size_t need = select_decode_ws_bytes(B, L, Hr, topk);
   if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
   rtp_status st = check_device();

@@ -4,21 +4,25 @@
 // 16-d indexer is the scout). Exact ties rank the smaller token first.
 //
 // Two kernels:
-//   scan    one pass over the key index; a KV group's index is read once for
-//           all retrieval heads of that group (grouped-query heads share
-//           keys). It writes every score (fp32, to the workspace, sized to stay
-//           in L2) and a histogram of the top 11 bits of each score's
-//           order-preserving key.
-//   filter  several CTAs per (sequence, head), each over a slice of the
-//           L2-resident scores. From the histogram every CTA knows the bin
-//           holding the k-th score: it marks the scores above that bin in a
-//           per-row bitmap (every 32-token word is owned by one CTA, so plain
-//           stores) and appends the bin's members to a candidate list. The
-//           last CTA of a row to finish settles the bin by a radix search over
-//           the candidates' remaining bits (exact ties: smallest token first),
-//           sets their bits and compacts the bitmap into the ascending index
-//           list. If the candidates overflow their list it runs a full radix
-//           select over the row instead.
+//   scan    one pass over the key index by as many CTAs as fit on the GPU, each
+//           a contiguous run of the (sequence, KV group) token ranges laid end
+//           to end; a group's index is read once for all its retrieval heads
+//           (grouped-query heads share keys), with evict-first loads. It
+//           writes every score (fp32, to the workspace; they stay in L2) and
+//           a histogram of the top 11 bits of each score's order-preserving
+//           key.
+//   filter  one wave of CTAs, several per (sequence, head), each over a slice
+//           of the scores. From the histogram every CTA knows the bin holding
+//           the k-th score (as float bounds): it marks the scores above that
+//           bin in a per-row bitmap (every 32-token word is owned by one CTA,
+//           so plain stores) and appends the bin's members to the row's
+//           candidate list through a shared buffer. The last CTA of a row to
+//           finish loads the candidates into shared memory, settles the bin by
+//           a radix search over their remaining bits (exact ties: smallest
+//           token first), sets their bits and compacts the bitmap into the
+//           ascending index list. Larger candidate lists are searched in
+//           global memory; if they overflow the list, a full radix select over
+//           the row runs instead.
 #include "rtp_common.cuh"
 #include "rtp_internal.h"
 
@@ -26,27 +30,37 @@ namespace rtp {
 
 namespace {
 constexpr int kScanThreads = 256;
-constexpr int kScanTokensPerThread = 16;
 constexpr int kScanBatch = 8;
-constexpr int kScanTokens = kScanThreads * kScanTokensPerThread;   // 4096 per CTA
+constexpr int kMaxGroups = 16;                                      // KV groups
+constexpr int kMaxHeadsPerGroup = 16;                               // retrieval heads of one group
 constexpr int kBins = 2048;                                        // top 11 bits
 constexpr int kFiltThreads = 512;
 constexpr int kFiltStep = kFiltThreads * 16;                       // scores per CTA step
 constexpr int kMaxTopk = 4096;
+constexpr int kLocCap = 2048;                                      // shared slots for a CTA's candidates
+constexpr int kSmemCand = 4096;                                    // shared slots for a row's candidates
+constexpr int kSmemWords = 4096;                                   // shared bitmap words (rows up to 128K)
 
 // Per-row bookkeeping of the filter kernel (zeroed with the histogram).
 struct RowState {
-  int n_cand;
-  int ticket;
+  int n_cand;      // filter: candidates appended
+  int ticket;      // filter: CTAs done
   int pad[2];
 };
 
 // Candidate-list capacity per row: an eighth of the row, at least 8192.
 __host__ __device__ inline int cand_cap(int L) { return L / 8 > 8192 ? L / 8 : 8192; }
 
+// Smallest float whose order-preserving key (f2key) is >= K: a score x has
+// f2key(x) >= K iff x >= key_floor_float(K) (for non-NaN x; -0 and +0 share
+// a key and compare equal).
+__device__ __forceinline__ float key_floor_float(uint32_t K) {
+  return __uint_as_float((K & 0x80000000u) ? (K & 0x7fffffffu) : ~K);
+}
+
 struct DecodeWs {
   float* scores;          // [B, Hr, L]
-  uint32_t* hist;         // [B, Hr, kBins]
+  uint32_t* hist;         // [B, Hr, kBins]: top 11 key bits of every score
   RowState* state;        // [B, Hr]      (zeroed together with hist)
   uint32_t* bitmap;       // [B, Hr, ceil(L / 32)]
   uint2* cand;            // [B, Hr, cand_cap(L)] (key, token)
@@ -77,8 +91,8 @@ DecodeWs decode_ws_layout(void* base, int B, int L, int Hr) {
 
 // Bin (top 11 key bits) of the k-th largest score of a row from its histogram,
 // and how many scores lie in higher bins. All threads get the result.
-template <int NT>
-__device__ void kth_bin(const uint32_t* __restrict__ h, int k, TopkSmem<NT>& sm, uint32_t& bin, int& above) {
+template <int NT, class SM>
+__device__ void kth_bin(const uint32_t* __restrict__ h, int k, SM& sm, uint32_t& bin, int& above) {
   const int tid = threadIdx.x;
   constexpr int per = kBins / NT;
   int local = 0;
@@ -105,70 +119,126 @@ __device__ void kth_bin(const uint32_t* __restrict__ h, int k, TopkSmem<NT>& sm,
 }
 }  // namespace
 
+// Retrieval heads served by each KV group (call-head indices), and the
+// groups serving at least one (the active groups) in order.
+struct GroupHeads {
+  int n[kMaxGroups];
+  int j[kMaxGroups][kMaxHeadsPerGroup];
+  int n_ag;
+  int ag[kMaxGroups];
+};
+
+
+// Persistent scan: the CTAs split the tokens of every (sequence, active
+// group) pair, laid end to end, into contiguous equal runs. Over each piece
+// of a pair a CTA scores the tokens for the group's retrieval heads and
+// histograms the top 11 key bits in shared memory, then adds the histogram to
+// the row's. MAXJ > 0: the group's q~ rows sit in
+// registers (at most MAXJ heads per group); MAXJ == 0: any number, read from
+// shared memory. Each thread keeps the loads of BATCH tokens in flight.
+template <int MAXJ, int BATCH>
 __global__ void __launch_bounds__(kScanThreads)
-decode_scan_kernel(const float* __restrict__ qt, const uint4* __restrict__ kindex, int L, int Hr, int Hkv,
-                   const HeadList hl, float* __restrict__ scores, uint32_t* __restrict__ ghist) {
-  extern __shared__ uint32_t shist[];                  // [n_j][kBins]
-  const int b = blockIdx.z, g = blockIdx.y;
-  __shared__ float qs[kMaxHeads][RTP_R];
-  __shared__ int js[kMaxHeads];
-  __shared__ int nj;
-  if (threadIdx.x == 0) {
-    int c = 0;
-    for (int j = 0; j < hl.n; ++j)
-      if (hl.kv[j] == g) js[c++] = j;
-    nj = c;
-  }
-  __syncthreads();
-  const int n = nj;
-  if (n == 0) return;
-  for (int e = threadIdx.x; e < n * RTP_R; e += kScanThreads)
-    qs[e / RTP_R][e % RTP_R] = qt[((size_t)b * Hr + js[e / RTP_R]) * RTP_R + e % RTP_R];
-  for (int e = threadIdx.x; e < n * kBins; e += kScanThreads) shist[e] = 0u;
-  __syncthreads();
-  const uint4* krow = kindex + ((size_t)b * Hkv + g) * (size_t)L * 2;
-  const int base = blockIdx.x * kScanTokens;
-  // batches of kScanBatch tokens per thread: all their loads are issued
-  // before any score is computed (32 bytes per token in flight)
+decode_scan_kernel(const float* __restrict__ qt, const uint4* __restrict__ kindex, int B, int L, int Hr, int Hkv,
+                   const GroupHeads gh, const DecodeWs w) {
+  extern __shared__ uint32_t shist[];                  // [heads of the group][kBins]
+  __shared__ float qs[MAXJ > 0 ? 1 : kMaxHeadsPerGroup][RTP_R];
+  const int64_t total = (int64_t)B * gh.n_ag * L;
+  const int64_t x0 = total * blockIdx.x / gridDim.x, x1 = total * (blockIdx.x + 1) / gridDim.x;
+  constexpr int QJ = MAXJ > 0 ? MAXJ : 1;
+  for (int64_t x = x0; x < x1;) {
+    const int seg = (int)(x / L);
+    const int u0 = (int)(x - (int64_t)seg * L);
+    const int64_t rem = x1 - x;
+    const int u1 = rem < (int64_t)(L - u0) ? u0 + (int)rem : L;
+    const int b = seg / gh.n_ag, g = gh.ag[seg - b * gh.n_ag];
+    const int n = gh.n[g];
+    float q[QJ][RTP_R];
+    float* srow[QJ];
+    if constexpr (MAXJ > 0) {
+#pragma unroll
+      for (int jj = 0; jj < MAXJ; ++jj) {
+        const int j = jj < n ? gh.j[g][jj] : gh.j[g][0];
+#pragma unroll
+        for (int c = 0; c < RTP_R; ++c) q[jj][c] = __ldg(qt + ((size_t)b * Hr + j) * RTP_R + c);
+        srow[jj] = w.scores + ((size_t)b * Hr + j) * L;
+      }
+    } else {
+      for (int e = threadIdx.x; e < n * RTP_R; e += kScanThreads)
+        qs[e / RTP_R][e % RTP_R] = qt[((size_t)b * Hr + gh.j[g][e / RTP_R]) * RTP_R + e % RTP_R];
+    }
+    for (int e = threadIdx.x; e < n * kBins; e += kScanThreads) shist[e] = 0u;
+    __syncthreads();
+    const uint4* krow = kindex + ((size_t)b * Hkv + g) * (size_t)L * 2;
 #pragma unroll 1
-  for (int s0 = 0; s0 < kScanTokensPerThread; s0 += kScanBatch) {
-    uint4 lo[kScanBatch], hi[kScanBatch];
+    for (int base = u0; base < u1; base += kScanThreads * BATCH) {
+      uint4 lo[BATCH], hi[BATCH];
 #pragma unroll
-    for (int t = 0; t < kScanBatch; ++t) {
-      const int u = base + (s0 + t) * kScanThreads + threadIdx.x;
-      if (u < L) {
-        lo[t] = __ldg(krow + (size_t)u * 2);
-        hi[t] = __ldg(krow + (size_t)u * 2 + 1);
+      for (int t = 0; t < BATCH; ++t) {
+        const int u = base + t * kScanThreads + threadIdx.x;
+        if (u < u1) {
+          // read once: evict-first, so that the scores stay in L2 for the filter
+          lo[t] = __ldcs(krow + (size_t)u * 2);
+          hi[t] = __ldcs(krow + (size_t)u * 2 + 1);
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < BATCH; ++t) {
+        const int u = base + t * kScanThreads + threadIdx.x;
+        if (u >= u1) break;
+        const float k[16] = {bf16_lo(lo[t].x), bf16_hi(lo[t].x), bf16_lo(lo[t].y), bf16_hi(lo[t].y),
+                             bf16_lo(lo[t].z), bf16_hi(lo[t].z), bf16_lo(lo[t].w), bf16_hi(lo[t].w),
+                             bf16_lo(hi[t].x), bf16_hi(hi[t].x), bf16_lo(hi[t].y), bf16_hi(hi[t].y),
+                             bf16_lo(hi[t].z), bf16_hi(hi[t].z), bf16_lo(hi[t].w), bf16_hi(hi[t].w)};
+        if constexpr (MAXJ > 0) {
+#pragma unroll
+          for (int jj = 0; jj < MAXJ; ++jj) {
+            if (jj >= n) break;
+            float acc = 0.f;
+#pragma unroll
+            for (int c = 0; c < RTP_R; ++c) acc = fmaf(q[jj][c], k[c], acc);
+            srow[jj][u] = acc;
+            atomicAdd(&shist[jj * kBins + (f2key(acc) >> 21)], 1u);
+          }
+        } else {
+          for (int jj = 0; jj < n; ++jj) {
+            float acc = 0.f;
+#pragma unroll
+            for (int c = 0; c < RTP_R; ++c) acc = fmaf(qs[jj][c], k[c], acc);
+            w.scores[((size_t)b * Hr + gh.j[g][jj]) * L + u] = acc;
+            atomicAdd(&shist[jj * kBins + (f2key(acc) >> 21)], 1u);
+          }
+        }
       }
     }
-#pragma unroll
-    for (int t = 0; t < kScanBatch; ++t) {
-      const int u = base + (s0 + t) * kScanThreads + threadIdx.x;
-      if (u >= L) break;
-      const float k[16] = {bf16_lo(lo[t].x), bf16_hi(lo[t].x), bf16_lo(lo[t].y), bf16_hi(lo[t].y),
-                           bf16_lo(lo[t].z), bf16_hi(lo[t].z), bf16_lo(lo[t].w), bf16_hi(lo[t].w),
-                           bf16_lo(hi[t].x), bf16_hi(hi[t].x), bf16_lo(hi[t].y), bf16_hi(hi[t].y),
-                           bf16_lo(hi[t].z), bf16_hi(hi[t].z), bf16_lo(hi[t].w), bf16_hi(hi[t].w)};
-      for (int jj = 0; jj < n; ++jj) {
-        float acc = 0.f;
-#pragma unroll
-        for (int c = 0; c < RTP_R; ++c) acc = fmaf(qs[jj][c], k[c], acc);
-        scores[((size_t)b * Hr + js[jj]) * L + u] = acc;
-        atomicAdd(&shist[jj * kBins + (f2key(acc) >> 21)], 1u);
-      }
+    __syncthreads();
+    for (int e = threadIdx.x; e < n * kBins; e += kScanThreads) {
+      const uint32_t c = shist[e];
+      if (c) atomicAdd(&w.hist[((size_t)b * Hr + gh.j[g][e / kBins]) * kBins + (e % kBins)], c);
     }
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < n * kBins; e += kScanThreads) {
-    const uint32_t c = shist[e];
-    if (c) atomicAdd(&ghist[((size_t)b * Hr + js[e / kBins]) * kBins + (e % kBins)], c);
+    x += u1 - u0;
   }
 }
 
-__global__ void __launch_bounds__(kFiltThreads)
+struct FiltSmem {
+  TopkSmem<kFiltThreads> tk;
+  union {
+    uint2 loc[kLocCap];                         // phase A: this CTA's candidates
+    uint2 all[kSmemCand];                       // phase B: the row's candidates
+  } cbuf;
+  uint32_t bits[kSmemWords];                    // phase B: the row's bitmap
+  uint2 fin[32];                                // phase B: the k-th score's 22-bit bin
+  int s_last, n_loc, s_base, n_fin;
+};
+
+__global__ void __launch_bounds__(kFiltThreads, 2)
 decode_filter_kernel(const DecodeWs w, int L, int Hr, int topk, int slice, int n_split, int32_t* __restrict__ idx) {
-  __shared__ TopkSmem<kFiltThreads> sm;
-  __shared__ int s_last;
+  extern __shared__ __align__(16) unsigned char filt_smem[];
+  FiltSmem& fs = *reinterpret_cast<FiltSmem*>(filt_smem);
+  TopkSmem<kFiltThreads>& sm = fs.tk;
+  uint2* loc = fs.cbuf.loc;
+  int& s_last = fs.s_last;
+  int& n_loc = fs.n_loc;
+  int& s_base = fs.s_base;
   const int part = blockIdx.x, j = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const size_t row = (size_t)b * Hr + j;
@@ -186,59 +256,92 @@ decode_filter_kernel(const DecodeWs w, int L, int Hr, int topk, int slice, int n
   uint32_t d1;
   int above1;
   kth_bin<kFiltThreads>(w.hist + row * kBins, topk, sm, d1, above1);
+  if (tid == 0) n_loc = 0;
+  __syncthreads();
 
-  // 1. this CTA's slice: bits for the scores above bin d1, candidates inside it.
-  //    A lane takes 16 consecutive scores; lanes 2m, 2m+1 share one bitmap word.
+  // A. this CTA's slice, two steps of 512 scores per warp at a time (all
+  //    loads in flight together): bits for the scores above bin d1; the
+  //    bin's members go to a shared buffer, then to the row's candidate list
+  //    with one reservation. A lane takes 16 consecutive scores; lanes 2m,
+  //    2m+1 share one bitmap word.
   const int lo = part * slice, hi = min(L, lo + slice);
   const bool vec = (L & 3) == 0;
-  for (int wbase = lo + warp * 512; wbase < hi; wbase += kFiltStep) {
-    const int base = wbase + lane * 16;
-    float x[16];
-    if (vec && base + 16 <= hi) {
+  // bin d1 as float bounds: a score is in the bin iff lo_f <= x < hi_f
+  // (no score lies above the top bin: hi_f is then NaN)
+  const float lo_f = key_floor_float(d1 << 21);
+  const float hi_f = d1 < 2047u ? key_floor_float((d1 + 1u) << 21) : __int_as_float(0x7fc00000);
+  for (int wb0 = lo + warp * 512; wb0 < hi; wb0 += 2 * kFiltStep) {
+    float x[2][16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(s + base) + q);
-        x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
-      }
-    } else {
+    for (int h = 0; h < 2; ++h) {
+      const int base = wb0 + h * kFiltStep + lane * 16;
+      if (vec && base + 16 <= hi) {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) x[e] = base + e < hi ? __ldg(s + base + e) : 0.f;
-    }
-    uint32_t bits = 0, cbits = 0;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const uint32_t d = f2key(x[e]) >> 21;
-      const bool valid = base + e < hi;
-      bits |= (valid && d > d1) ? 1u << e : 0u;
-      cbits |= (valid && d == d1) ? 1u << e : 0u;
-    }
-    // candidates: one global atomic per warp, lanes write their own in order
-    const int nc = __popc(cbits);
-    int incl = nc;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const int wtot = __shfl_sync(0xffffffffu, incl, 31);
-    if (wtot) {
-      int cbase = 0;
-      if (lane == 31) cbase = atomicAdd(&w.state[row].n_cand, wtot);
-      cbase = __shfl_sync(0xffffffffu, cbase, 31);
-      int pos = cbase + incl - nc;
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        if ((cbits >> e) & 1u) {
-          if (pos < cap) cand[pos] = make_uint2(f2key(x[e]), (uint32_t)(base + e));
-          ++pos;
+        for (int q = 0; q < 4; ++q) {
+          const float4 v = __ldg(reinterpret_cast<const float4*>(s + base) + q);
+          x[h][4 * q] = v.x; x[h][4 * q + 1] = v.y; x[h][4 * q + 2] = v.z; x[h][4 * q + 3] = v.w;
         }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[h][e] = base + e < hi ? __ldg(s + base + e) : 0.f;
+      }
     }
-    uint32_t word = bits << ((lane & 1) * 16);
-    word |= __shfl_xor_sync(0xffffffffu, word, 1);
-    if (!(lane & 1) && base < hi) bm[base >> 5] = word;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int base = wb0 + h * kFiltStep + lane * 16;
+      uint32_t bits = 0, cbits = 0;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const bool above = x[h][e] >= hi_f, in_bin = x[h][e] >= lo_f;
+        bits |= above ? 1u << e : 0u;
+        cbits |= (in_bin && !above) ? 1u << e : 0u;
+      }
+      if (base + 16 > hi) {
+        const uint32_t valid = base >= hi ? 0u : (1u << (hi - base)) - 1u;
+        bits &= valid;
+        cbits &= valid;
+      }
+      if (__any_sync(0xffffffffu, cbits != 0)) {
+        const int nc = __popc(cbits);
+        int incl = nc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        int cbase = 0;
+        if (lane == 31) cbase = atomicAdd(&n_loc, incl);
+        cbase = __shfl_sync(0xffffffffu, cbase, 31);
+        int pos = cbase + incl - nc;
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          if ((cbits >> e) & 1u) {
+            const uint32_t key = f2key(x[h][e]);
+            if (pos < kLocCap) loc[pos] = make_uint2(key, (uint32_t)(base + e));
+            else {
+              // the shared buffer is full: straight to the row's list
+              const int gp = atomicAdd(&w.state[row].n_cand, 1);
+              if (gp < cap) cand[gp] = make_uint2(key, (uint32_t)(base + e));
+            }
+            ++pos;
+          }
+      }
+      uint32_t word = bits << ((lane & 1) * 16);
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      if (!(lane & 1) && base < hi) bm[base >> 5] = word;
+    }
+  }
+  __syncthreads();
+  {
+    const int n_l = min(n_loc, kLocCap);
+    if (tid == 0 && n_l > 0) s_base = atomicAdd(&w.state[row].n_cand, n_l);
+    __syncthreads();
+    const int gb = s_base;
+    for (int x = tid; x < n_l; x += kFiltThreads)
+      if (gb + x < cap) cand[gb + x] = loc[x];
   }
 
-  // 2. the last CTA of the row settles bin d1 and writes the list
+  // B. the last CTA of the row settles the bin and writes the list
   __threadfence();
   __syncthreads();
   if (tid == 0) s_last = atomicAdd(&w.state[row].ticket, 1) == n_split - 1;
@@ -252,42 +355,131 @@ decode_filter_kernel(const DecodeWs w, int L, int Hr, int topk, int slice, int n
     block_topk_ascending<kFiltThreads>(key_of, L, topk, out, sm);
     return;
   }
-  const uint2* cc = cand;
   int need = topk - above1;
-  auto ckey = [cc](int x) { return __ldcg(&cc[x].x); };
-  const uint32_t thr = block_radix_threshold<kFiltThreads>(ckey, n_cand, need, sm, 1, d1 << 21, 0x7FFu << 21);
-  // keys equal to the threshold: the `need` smallest tokens among them
-  int n_eq = 0;
-  for (int x = tid; x < n_cand; x += kFiltThreads) n_eq += __ldcg(&cc[x].x) == thr;
-  int eq_tot;
-  block_exclusive_scan<kFiltThreads>(n_eq, eq_tot, sm.scan);
-  uint32_t tie_thr = 0;   // on ~token: larger means smaller token
-  if (need < eq_tot) {
-    int need2 = need;
-    auto tkey = [cc, thr](int x) {
-      const uint2 e = __ldcg(cc + x);
-      return e.x == thr ? ~e.y : 0u;
-    };
-    tie_thr = block_radix_threshold<kFiltThreads>(tkey, n_cand, need2, sm);
+  const uint2* cc = cand;
+  // the row's bitmap (when it fits) and candidates (when they fit) into
+  // shared memory, all loads of a thread in flight together
+  const bool sbits = W <= kSmemWords, scand = n_cand <= kSmemCand;
+  uint2* cs = fs.cbuf.all;
+  {
+    const int nw = sbits ? W : 0, nc = scand ? n_cand : 0;
+    for (int x0 = 0; x0 < max(nw, nc); x0 += kFiltThreads * 8) {
+      uint32_t wv[8];
+      uint2 e[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int x = x0 + t * kFiltThreads + tid;
+        wv[t] = x < nw ? __ldcg(bm + x) : 0u;
+        e[t] = x < nc ? __ldcg(cc + x) : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int x = x0 + t * kFiltThreads + tid;
+        if (x < nw) fs.bits[x] = wv[t];
+        if (x < nc) cs[x] = e[t];
+      }
+    }
   }
+  if (tid == 0) fs.n_fin = 0;
+  __syncthreads();
+  auto take = [&](uint32_t tok) {
+    if (sbits) atomicOr(&fs.bits[tok >> 5], 1u << (tok & 31));
+    else atomicOr(bm + (tok >> 5), 1u << (tok & 31));
+  };
+  // the bin's members, from shared memory when they fit
+  auto ckey = [&](int x) { return scand ? cs[x].x : __ldcg(&cc[x].x); };
+  auto ctok = [&](int x) { return scand ? cs[x].y : __ldcg(&cc[x].y); };
+  // pass 1: key bits 20..10 of the members -> the k-th score's 22-bit bin
+  for (int x = tid; x < kBins; x += kFiltThreads) sm.hist[x] = 0u;
+  __syncthreads();
+  for (int x = tid; x < n_cand; x += kFiltThreads) atomicAdd(&sm.hist[(ckey(x) >> 10) & 2047u], 1u);
+  __syncthreads();
+  uint32_t d2;
+  int above2;
+  {
+    constexpr int per = kBins / kFiltThreads;
+    int local = 0;
+    uint32_t c[per];
+#pragma unroll
+    for (int q = 0; q < per; ++q) {
+      c[q] = sm.hist[kBins - 1 - (tid * per + q)];
+      local += c[q];
+    }
+    int tot;
+    const int ab = block_exclusive_scan<kFiltThreads>(local, tot, sm.scan);
+    if (ab < need && ab + local >= need) {
+      int run = ab;
+#pragma unroll
+      for (int q = 0; q < per; ++q) {
+        if (run + (int)c[q] >= need) { sm.digit = kBins - 1 - (tid * per + q); sm.above = run; break; }
+        run += c[q];
+      }
+    }
+    __syncthreads();
+    d2 = (uint32_t)sm.digit;
+    above2 = sm.above;
+  }
+  const uint32_t pre22 = (d1 << 11) | d2;
+  need -= above2;
+  // members above the 22-bit bin are taken; the bin's own are gathered
   for (int x = tid; x < n_cand; x += kFiltThreads) {
-    const uint2 e = __ldcg(cc + x);
-    if (e.x > thr || (e.x == thr && ~e.y >= tie_thr)) atomicOr(bm + (e.y >> 5), 1u << (e.y & 31));
+    const uint32_t k = ckey(x), d = k >> 10;
+    if (d > pre22) take(ctok(x));
+    else if (d == pre22) {
+      const int p = atomicAdd(&fs.n_fin, 1);
+      if (p < 32) fs.fin[p] = make_uint2(k, ctok(x));
+    }
   }
   __syncthreads();
-  // 3. ordered compaction of the bitmap: ascending token indices
+  const int m = fs.n_fin;
+  if (m <= 32) {
+    // one warp ranks the bin's members: by key, then smaller token first
+    if (warp == 0 && lane < m) {
+      const uint2 me = fs.fin[lane];
+      int rank = 0;
+      for (int y = 0; y < m; ++y) {
+        const uint2 o = fs.fin[y];
+        rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+      }
+      if (rank < need) take(me.y);
+    }
+  } else {
+    // a crowded bin: radix over the last 10 bits, then the smallest tokens
+    // among keys equal to the threshold
+    const uint32_t thr = block_radix_threshold<kFiltThreads>(ckey, n_cand, need, sm, 2, pre22 << 10,
+                                                              0x3FFFFFu << 10);
+    int n_eq = 0;
+    for (int x = tid; x < n_cand; x += kFiltThreads) n_eq += ckey(x) == thr;
+    int eq_tot;
+    block_exclusive_scan<kFiltThreads>(n_eq, eq_tot, sm.scan);
+    uint32_t tie_thr = 0;   // on ~token: larger means smaller token
+    if (need < eq_tot) {
+      int need2 = need;
+      auto tkey = [&](int x) { return ckey(x) == thr ? ~ctok(x) : 0u; };
+      tie_thr = block_radix_threshold<kFiltThreads>(tkey, n_cand, need2, sm);
+    }
+    for (int x = tid; x < n_cand; x += kFiltThreads) {
+      const uint32_t k = ckey(x);
+      if ((k >> 10) != pre22) continue;
+      if (k > thr || (k == thr && ~ctok(x) >= tie_thr)) take(ctok(x));
+    }
+  }
+  __syncthreads();
+  // 3. ordered compaction of the bitmap: ascending token indices (a thread
+  //    holds `per` consecutive words)
   const int per = (W + kFiltThreads - 1) / kFiltThreads;
+  auto word = [&](int wi) { return sbits ? fs.bits[wi] : __ldcg(bm + wi); };
   int cnt = 0;
   for (int q = 0; q < per; ++q) {
     const int wi = tid * per + q;
-    if (wi < W) cnt += __popc(__ldcg(bm + wi));
+    if (wi < W) cnt += __popc(word(wi));
   }
   int tot;
   int pos = block_exclusive_scan<kFiltThreads>(cnt, tot, sm.scan);
   for (int q = 0; q < per; ++q) {
     const int wi = tid * per + q;
     if (wi >= W) break;
-    uint32_t v = __ldcg(bm + wi);
+    uint32_t v = word(wi);
     while (v) {
       const int bit = __ffs(v) - 1;
       v &= v - 1;
@@ -305,38 +497,64 @@ size_t select_decode_ws_bytes(int B, int L, int Hr, int topk) {
 cudaError_t launch_select_decode(const float* qt, const void* kindex, int B, int L, int Hr, int Hkv,
                                  const int32_t* kv_of, int topk, int32_t* idx, void* ws, cudaStream_t stream) {
   if (topk > kMaxTopk) return cudaErrorInvalidValue;
-  HeadList hl;
-  hl.n = Hr;
+  if (Hkv > kMaxGroups) return cudaErrorInvalidValue;
+  GroupHeads gh;
   int max_nj = 0;
+  gh.n_ag = 0;
   for (int g = 0; g < Hkv; ++g) {
     int c = 0;
-    for (int j = 0; j < Hr; ++j) c += (kv_of[j] == g);
+    for (int j = 0; j < Hr; ++j)
+      if (kv_of[j] == g) {
+        if (c >= kMaxHeadsPerGroup) return cudaErrorInvalidValue;
+        gh.j[g][c++] = j;
+      }
+    gh.n[g] = c;
+    if (c > 0) gh.ag[gh.n_ag++] = g;
     max_nj = c > max_nj ? c : max_nj;
   }
-  for (int j = 0; j < Hr; ++j) { hl.head[j] = j; hl.kv[j] = kv_of[j]; }
   const DecodeWs w = decode_ws_layout(ws, B, L, Hr);
   cudaError_t e = cudaMemsetAsync(w.hist, 0, w.zero_bytes, stream);
   if (e != cudaSuccess) return e;
-  const size_t scan_smem = (size_t)max_nj * kBins * sizeof(uint32_t);
-  if (scan_smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(decode_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
-    if (e != cudaSuccess) return e;
-  }
-  dim3 g1((L + kScanTokens - 1) / kScanTokens, Hkv, B);
-  decode_scan_kernel<<<g1, kScanThreads, scan_smem, stream>>>(qt, static_cast<const uint4*>(kindex), L, Hr, Hkv,
-                                                              hl, w.scores, w.hist);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  // about two CTAs per SM over all rows; slices are whole CTA steps
   int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  // scan: as many CTAs as fit on the GPU at once, each a contiguous run
+  const size_t scan_smem = (size_t)max_nj * kBins * sizeof(uint32_t);
+  const int64_t total = (int64_t)B * gh.n_ag * L;
+  auto scan = [&](auto kernel) -> cudaError_t {
+    cudaError_t e2 = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
+    if (e2 != cudaSuccess) return e2;
+    int per_sm = 0;
+    e2 = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kScanThreads, scan_smem);
+    if (e2 != cudaSuccess) return e2;
+    int64_t grid = (int64_t)(per_sm > 0 ? per_sm : 1) * sms;
+    const int64_t min_tokens = kScanThreads * kScanBatch;   // at least one batch of tokens per CTA
+    if (grid * min_tokens > total) grid = (total + min_tokens - 1) / min_tokens;
+    kernel<<<(int)grid, kScanThreads, scan_smem, stream>>>(qt, static_cast<const uint4*>(kindex), B, L, Hr, Hkv, gh,
+                                                           w);
+    return cudaGetLastError();
+  };
+  if (max_nj <= 1) e = scan(decode_scan_kernel<1, kScanBatch>);
+  else if (max_nj <= 2) e = scan(decode_scan_kernel<2, kScanBatch>);
+  else if (max_nj <= 4) e = scan(decode_scan_kernel<4, kScanBatch>);
+  else e = scan(decode_scan_kernel<0, kScanBatch>);
+  if (e != cudaSuccess) return e;
+  // filter: one wave of CTAs over all rows; slices are whole CTA steps
+  e = cudaFuncSetAttribute(decode_filter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(FiltSmem));
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_filter_kernel, kFiltThreads, sizeof(FiltSmem));
+  if (e != cudaSuccess) return e;
   const int rows = B * Hr;
-  int n_split = (2 * sms + rows - 1) / rows;
+  int n_split = (per_sm > 0 ? per_sm : 1) * sms / rows;
+  if (n_split < 1) n_split = 1;
   int slice = (L + n_split - 1) / n_split;
   slice = (slice + 511) / 512 * 512;
   n_split = (L + slice - 1) / slice;
   dim3 g2(n_split, Hr, B);
-  decode_filter_kernel<<<g2, kFiltThreads, 0, stream>>>(w, L, Hr, topk, slice, n_split, idx);
+  decode_filter_kernel<<<g2, kFiltThreads, sizeof(FiltSmem), stream>>>(w, L, Hr, topk, slice, n_split, idx);
   return cudaGetLastError();
 }
 

@@ -79,6 +79,10 @@ def test_rejects_bad_arguments_without_launching(L):
     assert L.rtp_select_decode(fake, fake, 1, 1000, 1, 1, 16, _heads([0]), 8, fake, None, 0, None) == WS
     assert L.rtp_select_decode(fake, fake, 1, 1000, 1, 1, 16, _heads([0]), 8, fake, fake, 10, None) == WS
     assert L.rtp_select_decode(fake, fake, 1, 1000, 1, 1, 16, _heads([0]), 5000, fake, fake, 1 << 30, None) == UNSUP
+    # more than 16 KV groups, or more than 16 retrieval heads on one group
+    assert L.rtp_select_decode(fake, fake, 1, 1000, 1, 17, 16, _heads([0]), 8, fake, fake, 1 << 30, None) == UNSUP
+    assert L.rtp_select_decode(fake, fake, 1, 1000, 17, 2, 16, _heads([0] * 17), 8, fake, fake, 1 << 30,
+                               None) == UNSUP
     # sparse prefill: bad window / scale / GQA ratio
     qs = S(64 * 8 * 128, 8 * 128, 128)
     ks = S(64 * 2 * 128, 2 * 128, 128)

@@ -108,9 +108,11 @@ def test_select_decode_matches_oracle(L, topk):
             assert ok, f"b{b} j{j}: {msg}"
 
 
-def test_select_decode_ties_pick_lowest_index():
-    """All keys equal: the lowest k indices must be chosen."""
-    L, topk = 3000, 100
+@pytest.mark.parametrize("L", [1500, 3000, 6000])
+def test_select_decode_ties_pick_lowest_index(L):
+    """All keys equal: the lowest k indices must be chosen (the tied bin fits
+    in shared memory at L = 1500; it does not at 3000 and 6000)."""
+    topk = 100
     kindex = torch.ones(1, 1, L, 16, dtype=torch.bfloat16)
     qt = torch.ones(1, 1, 16)
     idx = rtp.select_decode(qt.to(DEV), kindex.to(DEV), [0], topk).cpu().numpy()

@@ -202,6 +202,10 @@ def decode_bytes(cfg, idx: torch.Tensor, L: int, B: int) -> dict:
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+# Nominal dense peaks of one B200 (context beside the measured ones)
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 7700.0
+
 # DRAM bytes per launch (read + write) from one-pass ncu counters of the
 # current kernels at full size (profiles/traffic_prefill_1m.md and
 # profiles/decode_128k_b8.md); None where no capture of the current kernel
@@ -266,16 +270,20 @@ def run_ours(args, rank, world):
             rtp.swa(q, k, v, o, layer.swa_heads, layer.window, 0, layer.scale, ws=layer.ws_swa)
         ev[5].record(stream)
 
+    # the decode step's three calls on their own (per-kernel breakdown only;
+    # the step itself is one rtp_decode_step call, DecodeStep)
+    b_qt = torch.empty(Bd, len(step.ret), R, dtype=torch.float32, device=dev)
+    b_idx = torch.empty_like(step.idx)
+    b_ws_sel = torch.empty(rtp.lib().rtp_workspace_size_select_decode(Bd, L, len(step.ret), step.topk),
+                           dtype=torch.uint8, device=dev)
+    b_ws_att = torch.empty(rtp.lib().rtp_workspace_size_decode_attn_hybrid(
+        Bd, L, dcfg.Hq, step.topk, max(step.window, step.ret_window)), dtype=torch.uint8, device=dev)
+    b_od = torch.empty_like(od)
+
     def decode_step(ev):
         ev[0].record(stream)
-        rtp.index_project(qd.unsqueeze(1), Pd, step.ret, step.kv_ret,
-                          out=step.qt.view(Bd, len(step.ret), 1, R))
+        step(qd, kc, vc, kindex, Pd, od)
         ev[1].record(stream)
-        rtp.select_decode(step.qt, kindex, step.kv_ret, step.topk, step.idx, step.ws_sel)
-        ev[2].record(stream)
-        rtp.decode_attn_hybrid(qd, kc, vc, od, step.ret, step.idx, step.ret_window, step.swa_heads,
-                               step.window, step.sink, step.scale, step.ws_att)
-        ev[3].record(stream)
 
     def new_events(n):
         return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
@@ -284,19 +292,21 @@ def run_ours(args, rank, world):
     for _ in range(args.warmup):
         prefill_step(new_events(6))
         flush.zero_()
-        decode_step(new_events(4))
+        decode_step(new_events(2))
     torch.cuda.synchronize()
     # The decode step runs as one CUDA graph (the way a serving loop replays
     # it): one host launch per step, every kernel of the step inside. Each
     # call is also captured on its own for the per-kernel breakdown.
     g_step = step.graph(qd, kc, vc, kindex, Pd, od)
     d_calls = [
-        lambda: rtp.index_project(qd.unsqueeze(1), Pd, step.ret, step.kv_ret,
-                                  out=step.qt.view(Bd, len(step.ret), 1, R)),
-        lambda: rtp.select_decode(step.qt, kindex, step.kv_ret, step.topk, step.idx, step.ws_sel),
-        lambda: rtp.decode_attn_hybrid(qd, kc, vc, od, step.ret, step.idx, step.ret_window, step.swa_heads,
-                                       step.window, step.sink, step.scale, step.ws_att),
+        lambda: rtp.index_project(qd.unsqueeze(1), Pd, step.ret, step.kv_ret, out=b_qt.view(Bd, len(step.ret), 1, R)),
+        lambda: rtp.select_decode(b_qt, kindex, step.kv_ret, step.topk, b_idx, b_ws_sel),
+        lambda: rtp.decode_attn_hybrid(qd, kc, vc, b_od, step.ret, b_idx, step.ret_window, step.swa_heads,
+                                       step.window, step.sink, step.scale, b_ws_att),
     ]
+    for fn in d_calls:                      # once eagerly before capture
+        fn()
+    torch.cuda.synchronize()
     g_calls = []
     for fn in d_calls:
         g = torch.cuda.CUDAGraph()
@@ -334,7 +344,7 @@ def run_ours(args, rank, world):
     clk = clocks.stop() if rank == 0 else None
     if layer.device_status() != 0:
         raise RuntimeError("a prefill kernel reported a timed-out wait")
-    if rtp.workspace_status(step.ws_att) != 0:
+    if rtp.workspace_status(step.ws) != 0:
         raise RuntimeError("the decode attention reported an error status")
     # per-call breakdown of the decode step (after the timed region)
     call_ev = []
@@ -361,6 +371,10 @@ def run_ours(args, rank, world):
     d_ms = {n: sum(r[i][0].elapsed_time(r[i][1]) for r in call_ev) / len(call_ev) for i, n in enumerate(names_d)}
     p_step_ms = sum(p_ms.values())
     d_step_ms = sum(e[0].elapsed_time(e[1]) for e in dev_ev) / len(dev_ev)
+    p_steps = [e[0].elapsed_time(e[5]) for e in pev]
+    d_steps = [e[0].elapsed_time(e[1]) for e in dev_ev]
+    step_stats = {"prefill_ms_median": round(statistics.median(p_steps), 3), "prefill_ms_min": round(min(p_steps), 3),
+                  "decode_ms_median": round(statistics.median(d_steps), 4), "decode_ms_min": round(min(d_steps), 4)}
     p_step_ms = max_over_ranks(p_step_ms, world)
     d_step_ms = max_over_ranks(d_step_ms, world)
 
@@ -405,6 +419,9 @@ def run_ours(args, rank, world):
                     "work_per_launch": dw["bytes"]}
     selected_flops = sum(work[n]["flops"] for n in ("swa_prefill", "sparse_attn_prefill", "select_prefill"))
     layer_frac = selected_flops / (p_step_ms / 1e3) / 1e12 / tflops_peak
+    att_ms = p_ms["swa_prefill"] + p_ms["sparse_attn_prefill"]
+    att_frac = (work["swa_prefill"]["flops"] + work["sparse_attn_prefill"]["flops"]) / max(att_ms / 1e3, 1e-12) \
+        / 1e12 / tflops_peak
 
     db = decode_bytes(dcfg, step.idx, L, Bd)
     d_kern = {}
@@ -421,7 +438,7 @@ def run_ours(args, rank, world):
     value = total_tokens / (p_step_ms / 1e3)
     d_value = Bd * world / (d_step_ms / 1e3)
     launches_p = 5 if (layer.ret and layer.swa_heads) else 3
-    launches = launches_p + 5   # decode: project, scan, top-k, attention partials, merge
+    launches = launches_p + 5   # decode: projection, scan, filter, attention, merge
 
     # ---- end to end through the API with host buffers (rank-local, fewer steps)
     e2e = None
@@ -440,11 +457,17 @@ def run_ours(args, rank, world):
                    "decode_topk": dcfg.topk, "parallelism": f"independent layer per GPU x{world}",
                    "l2": "inputs larger than L2 (prefill Q/K/V 10 GiB); L2 flushed between decode steps"},
         "roofline": roofline,
+        "roofline_nominal": {"peak_tflops": NOMINAL_BF16_TFLOPS, "peak_gbs": NOMINAL_HBM_GBS,
+                             "frac": round(roofline["achieved"] / (NOMINAL_BF16_TFLOPS if roofline["unit"] == "TFLOP/s"
+                                                                   else NOMINAL_HBM_GBS), 4)},
+        "step_stats": step_stats,
         "layer_frac_of_tensor_peak": round(layer_frac, 4),
+        "attention_frac_of_tensor_peak": round(att_frac, 4),
         "kernels_prefill": kernels,
         "decode": {"value": round(d_value, 1), "unit": "tok/s", "ms_per_step": round(d_step_ms, 4),
                    "roofline": {"bound": "hbm", "achieved": round(d_ach, 1), "peak": peaks["hbm_gbs"],
                                 "unit": "GB/s", "frac": round(d_ach / peaks["hbm_gbs"], 4),
+                                "frac_nominal": round(d_ach / NOMINAL_HBM_GBS, 4),
                                 "traffic": MEASURED_TRAFFIC.get((dcfg.name, "step")), "bytes_per_step": db},
                    "kernels": d_kern},
         "gpu_launches": launches * args.steps,

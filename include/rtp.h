@@ -252,6 +252,36 @@ RTP_API rtp_status rtp_decode_attn_hybrid(const void* q, const void* kc, rtp_str
                                           rtp_stream_t stream);
 
 /*
+ * rtp_decode_step - one decode step of a layer in one call: the retrieval
+ * heads' query index q~ = q . P (fp32, as rtp_index_project), their token
+ * top-k over the key index (as rtp_select_decode, written to idx), and the
+ * attention of the retrieval and streaming heads (as rtp_decode_attn_hybrid).
+ *   Sources: the 128K decode workload statement (selection over the whole
+ *   cache unioned with the window and token 0); RTPurboV2 article (streaming
+ *   heads SWA). The paper defines the steps, not this grouping: it exists so
+ *   that the library knows the order of its own kernels and can start the
+ *   attention's window reads while the selection finishes.
+ *   q        bf16 [B, Hq, 128] device, contiguous (the new token's queries).
+ *   P        bf16 [Hkv, 128, 16] device (projector per KV head).
+ *   kindex   bf16 [B, Hkv, L, 16] device, contiguous (key index of the cache,
+ *            including the new token at L - 1).
+ *   kc, vc   bf16 [B, L, Hkv, 128] device with element strides ks, vs.
+ *   o        bf16 [B, Hq, 128] device out: rows of the listed heads.
+ *   ret_heads/swa_heads  host int32 lists (Hr or n_swa may be 0, not both).
+ *   idx      int32 [B, Hr, topk] device out (the selected tokens, ascending).
+ *   ws       rtp_workspace_size_decode_step(B, L, Hq, Hr, topk,
+ *            max(ret_window, swa_window)) bytes, 256-byte aligned; its first
+ *            word is the status word read by rtp_workspace_status.
+ *   Limits as in the three calls it combines. Asynchronous on `stream`.
+ */
+RTP_API size_t rtp_workspace_size_decode_step(int B, int L, int Hq, int Hr, int topk, int window);
+RTP_API rtp_status rtp_decode_step(const void* q, const void* P, const void* kindex, const void* kc, rtp_strides ks,
+                                   const void* vc, rtp_strides vs, void* o, int B, int L, int Hq, int Hkv,
+                                   const int32_t* ret_heads, int Hr, int topk, int ret_window, int sink,
+                                   const int32_t* swa_heads, int n_swa, int swa_window, float scale, int32_t* idx,
+                                   void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
  * rtp_sparse_attn_decode_noalloc - rtp_sparse_attn_decode without a workspace
  * argument and without allocating anything.
  *   The method's sources have no counterpart of this call: it exists for

@@ -56,6 +56,9 @@ _SIGNATURES = {
     "rtp_workspace_size_decode_attn_hybrid": (_SZ, [_I, _I, _I, _I, _I]),
     "rtp_decode_attn_hybrid": (_I, [_P, _P, Strides, _P, Strides, _P, _I, _I, _I, _I, _c_i32p, _I, _P, _I,
                                     _I, _I, _c_i32p, _I, _I, _F, _P, _SZ, _P]),
+    "rtp_workspace_size_decode_step": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "rtp_decode_step": (_I, [_P, _P, _P, _P, Strides, _P, Strides, _P, _I, _I, _I, _I, _c_i32p, _I, _I, _I, _I,
+                             _c_i32p, _I, _I, _F, _P, _P, _SZ, _P]),
     "rtp_workspace_size_swa": (_SZ, [_I, _I, _I, _I, _I]),
     "rtp_swa": (_I, [_P, Strides, _P, Strides, _P, Strides, _P, Strides, _I, _I, _I, _I, _I, _I,
                      _c_i32p, _I, _I, _F, _P, _SZ, _P]),
@@ -229,6 +232,27 @@ def decode_attn_hybrid(q, kc, vc, o, ret_heads: Sequence[int], idx, ret_window: 
     return o
 
 
+def decode_step(q, P, kindex, kc, vc, o, ret_heads: Sequence[int], idx, ret_window: int,
+                swa_heads: Sequence[int], swa_window: int, topk: int, sink: int = 1,
+                scale: Optional[float] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """One decode step in one call: q~ projection, top-k selection into idx and
+    the attention of retrieval and streaming heads. q/o [B,Hq,D], P [Hkv,D,r],
+    kindex [B,Hkv,L,r], kc/vc [B,L,Hkv,D], idx [B,Hr,topk] int32 (written)."""
+    B, Hq, D = q.shape
+    L, Hkv = kc.shape[1], kc.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    wmax = max(ret_window if ret_heads else 0, swa_window if swa_heads else 0)
+    need = lib().rtp_workspace_size_decode_step(B, L, Hq, len(ret_heads), topk, wmax)
+    buf, nbytes = _ws(need, q.device, ws)
+    _check(lib().rtp_decode_step(q.data_ptr(), P.data_ptr() if ret_heads else None,
+                                 kindex.data_ptr() if ret_heads else None, kc.data_ptr(), _strides4(kc),
+                                 vc.data_ptr(), _strides4(vc), o.data_ptr(), B, L, Hq, Hkv, _i32(ret_heads),
+                                 len(ret_heads), topk, ret_window, sink, _i32(swa_heads), len(swa_heads),
+                                 swa_window, scale, idx.data_ptr() if ret_heads else None, _wsptr(buf), nbytes,
+                                 _stream(stream)), "rtp_decode_step")
+    return o
+
+
 def swa(q, k, v, o, heads: Sequence[int], window: int, q_pos0: int = 0,
         scale: Optional[float] = None, ws: Optional[torch.Tensor] = None, stream=None):
     """Streaming-head sliding-window attention. q/o [B,Nq,Hq,D], k/v [B,Nk,Hkv,D]."""
@@ -306,23 +330,15 @@ class DecodeStep:
         self.window, self.ret_window, self.topk, self.sink = window, ret_window, topk, sink
         self.scale = 1.0 / math.sqrt(D_HEAD) if scale is None else scale
         self.kv_ret = [kv_of(h, Hq, Hkv) for h in self.ret]
-        if self.ret:
-            self.qt = torch.empty(B, len(self.ret), R_INDEX, dtype=torch.float32, device=device)
-            self.idx = torch.empty(B, len(self.ret), topk, dtype=torch.int32, device=device)
-            self.ws_sel = torch.empty(lib().rtp_workspace_size_select_decode(B, L, len(self.ret), topk),
-                                      dtype=torch.uint8, device=device)
+        self.idx = torch.empty(B, len(self.ret), topk, dtype=torch.int32, device=device) if self.ret else None
         wmax = max(ret_window if self.ret else 0, window if self.swa_heads else 0)
-        self.ws_att = torch.empty(lib().rtp_workspace_size_decode_attn_hybrid(B, L, Hq, topk if self.ret else 0,
-                                                                              wmax), dtype=torch.uint8, device=device)
+        self.ws = torch.empty(lib().rtp_workspace_size_decode_step(B, L, Hq, len(self.ret), topk, wmax),
+                              dtype=torch.uint8, device=device)
 
     def __call__(self, q, kc, vc, kindex, P, o, stream=None):
-        """q/o [B,Hq,D]; kc/vc [B,L,Hkv,D]; kindex [B,Hkv,L,r]."""
-        if self.ret:
-            index_project(q.unsqueeze(1), P, self.ret, self.kv_ret, out=self.qt.view(self.B, len(self.ret), 1, R_INDEX),
-                          stream=stream)
-            select_decode(self.qt, kindex, self.kv_ret, self.topk, self.idx, self.ws_sel, stream=stream)
-        decode_attn_hybrid(q, kc, vc, o, self.ret, self.idx if self.ret else None, self.ret_window,
-                           self.swa_heads, self.window, self.sink, self.scale, self.ws_att, stream=stream)
+        """q/o [B,Hq,D]; kc/vc [B,L,Hkv,D]; kindex [B,Hkv,L,r]; one rtp_decode_step call."""
+        decode_step(q, P, kindex, kc, vc, o, self.ret, self.idx, self.ret_window, self.swa_heads, self.window,
+                    self.topk, self.sink, self.scale, self.ws, stream=stream)
         return o
 
     def graph(self, q, kc, vc, kindex, P, o) -> "torch.cuda.CUDAGraph":

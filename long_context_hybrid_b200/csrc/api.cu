@@ -240,6 +240,76 @@ size_t rtp_workspace_size_decode_attn_hybrid(int B, int L, int Hq, int topk, int
   return decode_attn_ws_bytes(B, L, Hq, topk, window);
 }
 
+// Decode step workspace: [attention][q~ fp32 (256-aligned)][selection], the
+// attention part first so that its status word is at the start.
+namespace {
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+size_t step_qt_bytes(int B, int Hr) { return align256((size_t)B * Hr * RTP_R * sizeof(float)); }
+}  // namespace
+
+size_t rtp_workspace_size_decode_step(int B, int L, int Hq, int Hr, int topk, int window) {
+  if (B < 1 || L < 1 || Hq < 1 || Hr < 0 || window < 1) return 0;
+  size_t n = align256(decode_attn_ws_bytes(B, L, Hq, Hr > 0 ? topk : 0, window));
+  if (Hr > 0) n += step_qt_bytes(B, Hr) + align256(select_decode_ws_bytes(B, L, Hr, topk));
+  return n;
+}
+
+rtp_status rtp_decode_step(const void* q, const void* P, const void* kindex, const void* kc, rtp_strides ks,
+                           const void* vc, rtp_strides vs, void* o, int B, int L, int Hq, int Hkv,
+                           const int32_t* ret_heads, int Hr, int topk, int ret_window, int sink,
+                           const int32_t* swa_heads, int n_swa, int swa_window, float scale, int32_t* idx,
+                           void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  if (!q || !kc || !vc || !o) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return RTP_ERR_INVALID_ARG;
+  if (Hr < 0 || n_swa < 0 || Hr + n_swa < 1 || Hr + n_swa > kMaxHeads) return RTP_ERR_INVALID_ARG;
+  if (Hq / Hkv > 16 || Hkv > 16) return RTP_ERR_UNSUPPORTED;
+  if (Hr > 0) {
+    if (!P || !kindex || !idx || !ret_heads || topk < 1 || ret_window < 1) return RTP_ERR_INVALID_ARG;
+    if (topk > 4096) return RTP_ERR_UNSUPPORTED;
+    if (!aligned16(P) || !aligned16(kindex) || !aligned16(idx)) return RTP_ERR_INVALID_ARG;
+  }
+  if (n_swa > 0 && swa_window < 1) return RTP_ERR_INVALID_ARG;
+  if (sink < 0 || sink > kMaxSink || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
+  if (!stride_ok(ks) || !stride_ok(vs)) return RTP_ERR_INVALID_ARG;
+  int32_t all[kMaxHeads];
+  for (int i = 0; i < Hr; ++i) all[i] = ret_heads[i];
+  for (int i = 0; i < n_swa; ++i) all[Hr + i] = swa_heads ? swa_heads[i] : -1;
+  rtp_status st = check_heads(all, Hr + n_swa, Hq);
+  if (st != RTP_OK) return st;
+  const int G = Hq / Hkv;
+  int32_t kv_of[kMaxHeads];
+  for (int i = 0; i < Hr; ++i) kv_of[i] = ret_heads[i] / G;
+  for (int g = 0; g < Hkv; ++g) {
+    int c = 0;
+    for (int i = 0; i < Hr; ++i) c += kv_of[i] == g;
+    if (c > 16) return RTP_ERR_UNSUPPORTED;
+  }
+  const int wmax = (Hr > 0 && ret_window > swa_window) || n_swa == 0 ? ret_window : swa_window;
+  const size_t need = rtp_workspace_size_decode_step(B, L, Hq, Hr, topk, wmax);
+  if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
+  if ((st = check_device()) != RTP_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* base = static_cast<char*>(ws);
+  char* ws_att = base;
+  if (Hr > 0) {
+    float* qt = reinterpret_cast<float*>(base + align256(decode_attn_ws_bytes(B, L, Hq, topk, wmax)));
+    void* ws_sel = reinterpret_cast<char*>(qt) + step_qt_bytes(B, Hr);
+    // q~ = q . P for the retrieval heads (fp32, unrounded), then the top-k
+    cudaError_t e = launch_project(q, (int64_t)Hq * RTP_D, (int64_t)Hq * RTP_D, RTP_D, B, 1, P, ret_heads, kv_of, Hr,
+                                   qt, 1, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    e = launch_select_decode(qt, kindex, B, L, Hr, Hkv, kv_of, topk, idx, ws_sel, s);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  // The kernel before the attention is the selection's filter (or nothing of
+  // this call): it writes only idx, so the attention may read q, K and V early.
+  return from_cuda(launch_decode_hybrid(q, (int64_t)Hq * RTP_D, RTP_D, kc, ks.b, ks.n, ks.h, vc, vs.b, vs.n, vs.h,
+                                        o, (int64_t)Hq * RTP_D, RTP_D, B, L, L - 1, Hq, Hkv, ret_heads, Hr, idx, topk,
+                                        ret_window, sink, swa_heads, n_swa, swa_window, scale, ws_att, s,
+                                        /*early_start=*/Hr > 0));
+}
+
 rtp_status rtp_decode_attn_hybrid(const void* q, const void* kc, rtp_strides ks, const void* vc, rtp_strides vs,
                                   void* o, int B, int L, int Hq, int Hkv,
                                   const int32_t* ret_heads, int Hr, const int32_t* idx, int topk, int ret_window,

@@ -66,6 +66,7 @@ struct DecodeParams {
   int n_win_chunks;                  // B * n_ag * n_wc
   int n_gat_chunks;                  // B * n_ret * n_gc
   float* part;                       // [B, n_heads, max_slots, kPartStride]
+  int early_start;                   // window chunks may be read before the previous kernel ends
   int head[kMaxHeads];               // query head of each call head
   int wlo[kMaxHeads];                // first position of each call head's window
   int ag_of[kMaxHeads];              // active-group index of each call head
@@ -170,8 +171,12 @@ struct Cursor {
 // for every row), in two steps so that the selected-list read can be issued
 // a chunk early: slot_fetch reads what the position depends on, slot_pos
 // turns it into the position.
-__device__ __forceinline__ int slot_fetch(const DecodeParams& p, const Cursor& c, int s) {
+__device__ __forceinline__ int slot_fetch(const DecodeParams& p, const Cursor& c, int s, bool& dep_done) {
   if (!c.gathered) return 0;
+  if (!dep_done) {
+    pdl_wait();                               // the selected lists come from the previous kernel
+    dep_done = true;
+  }
   const int j = c.a;                          // retrieval heads are call heads 0..n_ret-1
   const int n_sink = min(p.sink, p.wlo[j]);
   const int e = c.local * kChunk + s;         // virtual list: sink tokens, then the selected entries
@@ -196,6 +201,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 decode_attn_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  pdl_trigger();                              // the merge may launch; it waits for this grid
+  // Unless the caller knows that the previous kernel on the stream writes
+  // none of q, K, V (only the selected lists), wait for it before any read.
+  if (!p.early_start) pdl_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, tq = lane & 3;
   const int n_ctas = gridDim.x;
@@ -213,7 +222,8 @@ decode_attn_kernel(const DecodeParams p) {
   const uint32_t ring = su32(sm.ring[warp]);
   Cursor icur = first;                        // next chunk to copy
   const int my_slot = warp * kKeys + (lane & (kKeys - 1));
-  int fetched = slot_fetch(p, icur, my_slot);  // for the next chunk to copy
+  bool dep_done = false;
+  int fetched = slot_fetch(p, icur, my_slot, dep_done);  // for the next chunk to copy
   auto issue = [&](int t) {
     if (t < n_t) {
       const int st = t % kStages;
@@ -236,7 +246,7 @@ decode_attn_kernel(const DecodeParams p) {
         cp_async16(vdst + slab_off(r, c), vs + c * 16, ok);
       }
       icur.next(p, g0);
-      if (t + 1 < n_t) fetched = slot_fetch(p, icur, my_slot);
+      if (t + 1 < n_t) fetched = slot_fetch(p, icur, my_slot, dep_done);
     }
     cp_async_commit();                        // one group per chunk, empty past the run
   };
@@ -404,6 +414,7 @@ decode_merge_kernel(const DecodeParams p, int n_ctas, int* status) {
   __shared__ float wm[4], wl[4];
   __shared__ float4 wo[4][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait();                                 // the partials are complete
   if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
   const int b = blockIdx.x / p.n_heads, j = blockIdx.x - b * p.n_heads;
   int n = n_pieces((b * p.n_ag + p.ag_of[j]) * p.n_wc, p.n_wc, p.n_win_chunks, n_ctas);
@@ -487,8 +498,9 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
                                  const int32_t* ret_heads, int n_ret, const int32_t* idx, int topk,
                                  int ret_window, int sink,
                                  const int32_t* swa_heads, int n_swa, int swa_window,
-                                 float scale, void* ws, cudaStream_t stream) {
+                                 float scale, void* ws, cudaStream_t stream, bool early_start) {
   DecodeParams p;
+  p.early_start = early_start ? 1 : 0;
   p.q = static_cast<const __nv_bfloat16*>(q); p.q_sb = q_sb; p.q_sh = q_sh;
   p.k = static_cast<const __nv_bfloat16*>(kc); p.k_sb = k_sb; p.k_sn = k_sn; p.k_sh = k_sh;
   p.v = static_cast<const __nv_bfloat16*>(vc); p.v_sb = v_sb; p.v_sn = v_sn; p.v_sh = v_sh;
@@ -550,10 +562,12 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
   const size_t smem = sizeof(Smem);
   e = cudaFuncSetAttribute(decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  decode_attn_kernel<<<grid, kThreads, smem, stream>>>(p);
-  e = cudaGetLastError();
+  // both kernels may start while their predecessor runs (with early_start the
+  // attention streams its window chunks before it waits for the selected lists)
+  e = launch_pdl(decode_attn_kernel, dim3(grid), dim3(kThreads), smem, stream, p);
   if (e != cudaSuccess) return e;
-  decode_merge_kernel<<<B * p.n_heads, 128, 0, stream>>>(p, grid, status);
+  e = launch_pdl(decode_merge_kernel, dim3(B * p.n_heads), dim3(128), 0, stream, p, grid, status);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -19,6 +19,14 @@ struct HeadList {
   int kv[kMaxHeads];     // its KV head
 };
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start before the previous kernel of the stream has
+// finished; pdl_wait() blocks the calling thread until that kernel has
+// completed and its writes are visible (a no-op for a normal launch), and
+// pdl_trigger() lets the next such kernel launch before this one ends.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 

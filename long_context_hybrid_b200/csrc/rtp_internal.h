@@ -7,6 +7,25 @@
 
 namespace rtp {
 
+// Launches `kernel` with programmatic stream serialisation: it may begin
+// while the previous kernel on the stream is still running, and must call
+// pdl_wait() before reading anything that kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 struct HeadList;
 
 cudaError_t launch_project(const void* x, int64_t sb, int64_t sn, int64_t sh, int B, int N,
@@ -47,7 +66,7 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
                                  const int32_t* ret_heads, int n_ret, const int32_t* idx, int topk,
                                  int ret_window, int sink,
                                  const int32_t* swa_heads, int n_swa, int swa_window,
-                                 float scale, void* ws, cudaStream_t stream);
+                                 float scale, void* ws, cudaStream_t stream, bool early_start = false);
 
 // Same as launch_decode_attn for retrieval heads, with the partials in a
 // library-owned static device array of kNoAllocScratchBytes.

@@ -140,6 +140,7 @@ template <int MAXJ, int BATCH>
 __global__ void __launch_bounds__(kScanThreads)
 decode_scan_kernel(const float* __restrict__ qt, const uint4* __restrict__ kindex, int B, int L, int Hr, int Hkv,
                    const GroupHeads gh, const DecodeWs w) {
+  pdl_trigger();                                       // the filter may launch and wait for this grid
   extern __shared__ uint32_t shist[];                  // [heads of the group][kBins]
   __shared__ float qs[MAXJ > 0 ? 1 : kMaxHeadsPerGroup][RTP_R];
   const int64_t total = (int64_t)B * gh.n_ag * L;
@@ -243,6 +244,8 @@ decode_filter_kernel(const DecodeWs w, int L, int Hr, int topk, int slice, int n
   const int lane = tid & 31, warp = tid >> 5;
   const size_t row = (size_t)b * Hr + j;
   int32_t* out = idx + row * topk;
+  pdl_trigger();          // the attention may launch: it waits for this grid before reading idx
+  pdl_wait();             // the scan's scores and histogram are complete
   if (L <= topk) {
     if (part == 0)
       for (int i = tid; i < topk; i += kFiltThreads) out[i] = i < L ? i : -1;
@@ -554,8 +557,8 @@ cudaError_t launch_select_decode(const float* qt, const void* kindex, int B, int
   slice = (slice + 511) / 512 * 512;
   n_split = (L + slice - 1) / slice;
   dim3 g2(n_split, Hr, B);
-  decode_filter_kernel<<<g2, kFiltThreads, sizeof(FiltSmem), stream>>>(w, L, Hr, topk, slice, n_split, idx);
-  return cudaGetLastError();
+  return launch_pdl(decode_filter_kernel, g2, dim3(kFiltThreads), sizeof(FiltSmem), stream, w, L, Hr, topk, slice,
+                    n_split, idx);
 }
 
 }  // namespace rtp

@@ -103,6 +103,22 @@ def test_rejects_bad_arguments_without_launching(L):
     # decode sparse attention: idx null
     assert L.rtp_sparse_attn_decode(fake, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, None,
                                     16, 64, 1, ctypes.c_float(0.1), fake, 1 << 20, None) == INVALID
+    # fused decode step: retrieval heads need P, the index and idx; workspace checked; sink bound
+    f = ctypes.c_float(0.1)
+    assert L.rtp_decode_step(fake, None, fake, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, 16, 64, 1,
+                             _heads([1]), 1, 64, f, fake, fake, 1 << 24, None) == INVALID
+    assert L.rtp_decode_step(fake, fake, fake, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, 16, 64, 1,
+                             _heads([1]), 1, 64, f, fake, None, 0, None) == WS
+    assert L.rtp_decode_step(fake, fake, fake, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, 16, 64, 65,
+                             _heads([1]), 1, 64, f, fake, fake, 1 << 24, None) == INVALID
+    assert L.rtp_decode_step(fake, fake, fake, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, 5000, 64, 1,
+                             _heads([1]), 1, 64, f, fake, fake, 1 << 30, None) == UNSUP
+    # its workspace holds the three calls' workspaces
+    B, Lc, Hq, Hr, k, w = 4, 20000, 32, 5, 2048, 4096
+    whole = L.rtp_workspace_size_decode_step(B, Lc, Hq, Hr, k, w)
+    parts = (L.rtp_workspace_size_decode_attn_hybrid(B, Lc, Hq, k, w)
+             + L.rtp_workspace_size_select_decode(B, Lc, Hr, k) + B * Hr * 16 * 4)
+    assert parts <= whole <= parts + 3 * 256
 
 
 def test_binding_raises_without_library(tmp_path, monkeypatch):

@@ -377,6 +377,31 @@ def test_e2e_decode_reduced():
     assert torch.equal(o, o2), "graph replay with a new query differs from the eager step"
 
 
+def test_decode_step_equals_the_three_calls():
+    """rtp_decode_step (projection, selection and attention in one call, the
+    attention starting before the selection ends) gives bit for bit what the
+    three calls give one after another."""
+    cfg = synth.DECODE_128K
+    B, L = 3, 20000
+    data = synth.make_decode(cfg, device=DEV, B=B, L=L, seed=cfg.seed + 5)
+    q, kc, vc, P = data["q"], data["kc"], data["vc"], data["P"]
+    kindex = rtp.index_project(kc, P, list(range(cfg.Hkv)), list(range(cfg.Hkv)))
+    ret = list(cfg.ret_heads)
+    swa_heads = [h for h in range(cfg.Hq) if h not in ret]
+    kv_ret = [rtp.kv_of(h, cfg.Hq, cfg.Hkv) for h in ret]
+    for window in (8192, 1000):
+        o1 = torch.zeros(B, cfg.Hq, 128, dtype=torch.bfloat16, device=DEV)
+        idx1 = torch.empty(B, len(ret), cfg.topk, dtype=torch.int32, device=DEV)
+        rtp.decode_step(q, P, kindex, kc, vc, o1, ret, idx1, window, swa_heads, window, cfg.topk, sink=1)
+        qt = rtp.index_project(q.unsqueeze(1), P, ret, kv_ret, out_dtype=torch.float32).view(B, len(ret), 16)
+        idx2 = rtp.select_decode(qt, kindex, kv_ret, cfg.topk)
+        o2 = torch.zeros_like(o1)
+        rtp.decode_attn_hybrid(q, kc, vc, o2, ret, idx2, window, swa_heads, window, 1)
+        torch.cuda.synchronize()
+        assert torch.equal(idx1, idx2)
+        assert torch.equal(o1, o2)
+
+
 @pytest.mark.parametrize("L,ret_window,swa_window,topk", [(6000, 512, 256, 300), (6000, 256, 1024, 129),
                                                           (700, 4096, 4096, 100), (20000, 8192, 8192, 2048)])
 def test_decode_attn_hybrid_matches_oracle(L, ret_window, swa_window, topk):

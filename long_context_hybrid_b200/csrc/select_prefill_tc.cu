@@ -4,8 +4,8 @@
 // key block j <= i, the max of q~_t . k~_u over the causal pairs of the two
 // 64-token blocks; each query block keeps its top-k key blocks (RTPurbo digest:
 // the 16-d indexer picks the candidates). The token score matrix never leaves
-// the SM: every 128 x 256 score tile lives in TMEM only until its block maxima
-// are taken.
+// the SM: every 128 x 256 score tile lives in TMEM only until the epilogue has
+// copied it into registers.
 //
 // One CTA handles query blocks 2t and 2t+1 (128 query rows) of one retrieval
 // head, longest key ranges first. Warp roles (384 threads):
@@ -14,12 +14,17 @@
 //                swizzle);
 //   warp 1       TMEM owner and MMA issuer: one tcgen05.mma M=128 N=256 K=16
 //                per key tile into one of two TMEM score buffers;
-//   warps 4..11  two epilogue warpgroups, one per score buffer: thread r reads
-//                row r of the tile, takes the causal max of each 64-column
-//                block (3-input max), reduces over the 32 rows of its warp
-//                (redux.sync), and folds the result into the block-score array
-//                of its query block with a shared-memory atomic max on
-//                order-preserving integer keys.
+//   warps 4..11  epilogue: every warp takes part in every tile. Warp w reads
+//                rows 32*(w%4).. and the 128 columns of key blocks 2*(w/4-1)
+//                and the next with one tcgen05.ld, releases the buffer to the
+//                MMA warp at once, and reduces each 64-column block of its
+//                row to one value with a tree of 3-input maxima. The per-row
+//                maxima are staged in shared memory (32 rows x 32 values per
+//                warp); every 16 tiles lane l folds column l over the 32 rows
+//                and merges it into the block-score array of its query block
+//                with a shared-memory atomic max on order-preserving keys.
+//                Tiles that reach the diagonal block take a per-block path
+//                with the causal mask and a warp reduction.
 // Finally all threads run the exact radix top-k of each of the two block-score
 // arrays (ties to the smaller block) and write ascending lists.
 #include "rtp_common.cuh"
@@ -32,11 +37,14 @@ using namespace sm100;
 namespace {
 
 constexpr int kThreads = 384;
+constexpr int kBpw = 2;                            // 64-key blocks per epilogue warp per tile
 constexpr int kKStages = 4;
 constexpr int kChunkKeys = 256;                    // 4 key blocks per MMA
 constexpr uint32_t kQOff = 0;                      // 128 rows x 32 B
 constexpr uint32_t kKOff = 4096;                   // stage s at +s*8192 (256 rows x 32 B)
-constexpr uint32_t kScoreOff = kKOff + kKStages * 8192u;
+constexpr int kStageChunks = 32 / kBpw;            // tiles per flush of the staged row maxima
+constexpr uint32_t kStgOff = kKOff + kKStages * 8192u;  // per epilogue warp: 32 rows x 33 floats
+constexpr uint32_t kScoreOff = kStgOff + 8u * 32u * 33u * 4u;
 constexpr int kStatusTimeout = 4;
 
 struct SelBars {
@@ -53,6 +61,43 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
+}
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) { asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory"); }
+__device__ __forceinline__ float lds_f32(uint32_t a) { float v; asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory"); return v; }
+// max of 64 scores: a tree of 3-input maxima (32 instructions, depth 4)
+__device__ __forceinline__ float tree_max64(const uint32_t* u) {
+  float a[22], c[8];
+#pragma unroll
+  for (int x = 0; x < 21; ++x)
+    a[x] = max3f(__uint_as_float(u[3 * x]), __uint_as_float(u[3 * x + 1]), __uint_as_float(u[3 * x + 2]));
+  a[21] = __uint_as_float(u[63]);
+#pragma unroll
+  for (int x = 0; x < 7; ++x) c[x] = max3f(a[3 * x], a[3 * x + 1], a[3 * x + 2]);
+  c[7] = a[21];
+  return max3f(max3f(c[0], c[1], c[2]), max3f(c[3], c[4], c[5]), fmaxf(c[6], c[7]));
+}
+__device__ __forceinline__ bool try_wait_nohint(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Bounded wait without a suspend hint (the epilogue's per-tile handshake).
+__device__ __forceinline__ bool wait_tile(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (try_wait_nohint(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (try_wait_nohint(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > kWaitLimitCycles) { *abort_flag = 1; return false; }
+    }
+  }
 }
 __device__ __forceinline__ float warp_max(float v) {
   float r;
@@ -113,7 +158,7 @@ prefill_select_tc_kernel(const SelectTcParams p, const __grid_constant__ CUtenso
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&bars.s_full[s]), 1);
-      mbar_init(smem_u32(&bars.s_free[s]), 128);
+      mbar_init(smem_u32(&bars.s_free[s]), 8);     // one arrive per epilogue warp
     }
     mbar_init(smem_u32(&bars.fin), 1);
     bars.abort = 0;
@@ -169,50 +214,110 @@ prefill_select_tc_kernel(const SelectTcParams p, const __grid_constant__ CUtenso
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int wg = (warp - 4) >> 2;                 // 0 or 1: which score buffer
-    const int r = tid - 128 - wg * 128;             // row 0..127 of the tile
-    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16) + wg * 256u;
-    const bool in_a = r < 64;
-    const int my_last = in_a ? qa : last_blk;       // key blocks this row's query block may see
-    const int rq = in_a ? r : r - 64;               // row within its query block
+    const int wu = __shfl_sync(0xffffffffu, warp, 0);   // warp index, uniform across the warp
+    const int quad = wu & 3;                            // TMEM lane quarter = rows 32*quad ..
+    const int b_lo = ((wu - 4) >> 2) * kBpw;            // first of this warp's blocks in a tile
+    const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(b_lo * 64);
+    const bool in_a = quad < 2;
     const int my_q = in_a ? qa : qb;
+    const int my_last = in_a ? qa : last_blk;
+    const int rq = (quad & 1) * 32 + lane;              // row within its query block
+    const bool rows_valid = in_a || has_b;
     uint32_t* dst = in_a ? sA : sB;
-    for (int c = wg; c < n_chunks; c += 2) {
-      bool w = mbar_wait(smem_u32(&bars.s_full[wg]), (c >> 1) & 1, abort_flag);
+    const int n_fast = qa >> 2;                         // tiles whose 4 blocks all precede block qa
+    bool live = true;
+    int c = 0;
+    const uint32_t stg = sb + kStgOff + (uint32_t)((wu - 4) * (32 * 33) * 4);   // shared address
+    int n_stg = 0, c_stg = 0;
+    // lane l folds staged column l (tile c_stg + l / kBpw, block b_lo + l % kBpw) over the warp's 32 rows
+    auto flush = [&](int n_tiles) {
+      __syncwarp();
+      if (lane < n_tiles * kBpw) {
+        const uint32_t col = stg + lane * 4u;
+        float x[11];
+#pragma unroll
+        for (int r = 0; r < 10; ++r)
+          x[r] = max3f(lds_f32(col + (3 * r) * 132), lds_f32(col + (3 * r + 1) * 132), lds_f32(col + (3 * r + 2) * 132));
+        x[10] = fmaxf(lds_f32(col + 30 * 132), lds_f32(col + 31 * 132));
+        const float m = max3f(max3f(x[0], x[1], x[2]), max3f(x[3], x[4], x[5]), max3f(max3f(x[6], x[7], x[8]), x[9], x[10]));
+        const int kb = (c_stg + lane / kBpw) * 4 + b_lo + lane % kBpw;
+        if (rows_valid) atomicMax(&dst[kb], f2key(m));
+      }
+      __syncwarp();
+    };
+    // two tiles (both score buffers) per iteration: constant TMEM offsets, one parity
+    for (; c + 1 < n_fast; c += 2) {
+      const uint32_t par = (c >> 1) & 1;
+#pragma unroll
+      for (int buf = 0; buf < 2; ++buf) {
+        const bool w = wait_tile(smem_u32(&bars.s_full[buf]), par, abort_flag);
+        if (!__all_sync(0xffffffffu, w)) { live = false; break; }
+        tc_fence_after();
+        uint32_t v[128];
+        tmem_ld128(taddr + buf * 256u, v);
+        tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars.s_free[buf]));
+        const uint32_t a = stg + (uint32_t)(lane * 33 + (n_stg + buf) * 2) * 4u;
+        sts_f32(a, tree_max64(v));
+        sts_f32(a + 4, tree_max64(v + 64));
+      }
+      if (!live) break;
+      n_stg += 2;
+      if (n_stg == kStageChunks) {
+        flush(kStageChunks);
+        n_stg = 0;
+        c_stg = c + 2;
+      }
+    }
+    for (; live && c < n_fast; ++c) {
+      const int buf = c & 1;
+      const bool w = wait_tile(smem_u32(&bars.s_full[buf]), (c >> 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, w)) { live = false; break; }
+      tc_fence_after();
+      uint32_t v[128];
+      tmem_ld128(taddr + buf * 256u, v);
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars.s_free[buf]));
+#pragma unroll
+      for (int bb = 0; bb < kBpw; ++bb) sts_f32(stg + (uint32_t)(lane * 33 + n_stg * kBpw + bb) * 4u, tree_max64(v + 64 * bb));
+      if (++n_stg == kStageChunks) {
+        flush(kStageChunks);
+        n_stg = 0;
+        c_stg = c + 1;
+      }
+    }
+    if (live && n_stg > 0) flush(n_stg);
+    for (; live && c < n_chunks; ++c) {
+      const int buf = c & 1;
+      const bool w = wait_tile(smem_u32(&bars.s_full[buf]), (c >> 1) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after();
+      uint32_t v[128];
+      tmem_ld128(taddr + buf * 256u, v);
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars.s_free[buf]));
 #pragma unroll
-      for (int bi = 0; bi < 4; ++bi) {
-        const int kb = c * 4 + bi;
-        if (kb > last_blk) break;                   // warp-uniform: same for the whole CTA
-        uint32_t v[64];
-        tmem_ld32(lane_base + bi * 64u, v);
-        tmem_ld32(lane_base + bi * 64u + 32u, v + 32);
-        tc_wait_ld();
+      for (int bb = 0; bb < kBpw; ++bb) {
+        const int kb = c * 4 + b_lo + bb;
+        const uint32_t* u = v + 64 * bb;
         float m = -INFINITY;
         if (kb < my_q) {
-          // 64 -> 1 in a tree of 3-input maxima (32 instructions, depth 4)
-          float a[22], c[8];
-#pragma unroll
-          for (int x = 0; x < 21; ++x)
-            a[x] = max3f(__uint_as_float(v[3 * x]), __uint_as_float(v[3 * x + 1]), __uint_as_float(v[3 * x + 2]));
-          a[21] = __uint_as_float(v[63]);
-#pragma unroll
-          for (int x = 0; x < 7; ++x) c[x] = max3f(a[3 * x], a[3 * x + 1], a[3 * x + 2]);
-          c[7] = a[21];
-          m = max3f(max3f(c[0], c[1], c[2]), max3f(c[3], c[4], c[5]), fmaxf(c[6], c[7]));
+          m = tree_max64(u);
         } else if (kb == my_q) {
           // diagonal block: key column x is causal for this row iff x <= rq
 #pragma unroll
           for (int x = 0; x < 64; ++x)
-            if (x <= rq) m = fmaxf(m, __uint_as_float(v[x]));
+            if (x <= rq) m = fmaxf(m, __uint_as_float(u[x]));
         }
-        if (!has_b && !in_a) m = -INFINITY;         // rows of a query block past the end
-        const float wm = warp_max(m);
-        if (lane == 0 && kb <= my_last && wm != -INFINITY) atomicMax(&dst[kb], f2key(wm));
+        const float wmax = warp_max(m);
+        if (lane == 0 && rows_valid && kb <= my_last && wmax != -INFINITY) atomicMax(&dst[kb], f2key(wmax));
       }
-      tc_fence_before();
-      mbar_arrive(smem_u32(&bars.s_free[wg]));
     }
   }
 

@@ -12,8 +12,9 @@
 //   warp 0       TMA: the 128 x 16 query-index tile once, then 256 x 16
 //                key-index tiles (4 key blocks) into a 4-stage ring (32-byte
 //                swizzle);
-//   warp 1       TMEM owner and MMA issuer: one tcgen05.mma M=128 N=256 K=16
-//                per key tile into one of two TMEM score buffers;
+//   warp 1       TMEM owner; warps 1 and 2 issue the MMAs of the even and the
+//                odd key tiles: one tcgen05.mma M=128 N=256 K=16 per tile into
+//                TMEM score buffer 0 or 1;
 //   warps 4..11  epilogue: every warp takes part in every tile. Warp w reads
 //                rows 32*(w%4).. and the 128 columns of key blocks 2*(w/4-1)
 //                and the next with one tcgen05.ld, releases the buffer to the
@@ -160,7 +161,7 @@ prefill_select_tc_kernel(const SelectTcParams p, const __grid_constant__ CUtenso
       mbar_init(smem_u32(&bars.s_full[s]), 1);
       mbar_init(smem_u32(&bars.s_free[s]), 8);     // one arrive per epilogue warp
     }
-    mbar_init(smem_u32(&bars.fin), 1);
+    mbar_init(smem_u32(&bars.fin), 2);
     bars.abort = 0;
     fence_mbar_init();
   }
@@ -195,13 +196,17 @@ prefill_select_tc_kernel(const SelectTcParams p, const __grid_constant__ CUtenso
           wait_short(smem_u32(&bars.k_full[c % kKStages]), (c / kKStages) & 1);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
+    // Two issuers, one per score buffer: a tcgen05.mma and its commits take a
+    // few hundred cycles to issue on a scheduler whose epilogue warps keep the
+    // ALU busy, so one thread alone cannot keep both buffers full.
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false, false);
       bool ok = mbar_wait(smem_u32(&bars.q_full), 0, abort_flag);
       const uint64_t qdesc = desc_sw32(sb + kQOff);
-      for (int c = 0; ok && c < n_chunks; ++c) {
-        const int s = c % kKStages, buf = c & 1;
+      const int buf = warp - 1;
+      for (int c = buf; ok && c < n_chunks; c += 2) {
+        const int s = c % kKStages;
         if (!mbar_wait(smem_u32(&bars.k_full[s]), (c / kKStages) & 1, abort_flag)) break;
         if (c >= 2 && !mbar_wait(smem_u32(&bars.s_free[buf]), ((c >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();

@@ -211,6 +211,7 @@ NOMINAL_HBM_GBS = 7700.0
 # profiles/decode_128k_b8.md); None where no capture of the current kernel
 # exists. Reset an entry whenever its kernel changes.
 MEASURED_TRAFFIC = {
+    ("prefill_1m", "select_prefill"): 316478208 + 73203200,
     ("prefill_1m", "sparse_attn_prefill"): 112003927552 + 1351792128,
     ("prefill_1m", "swa_prefill"): 21796575744 + 7232377088,
     # decode step: scan + filter + attention + merge (cold cache, as the bench

@@ -11,12 +11,15 @@
 //           writes every score (fp32, to the workspace; they stay in L2) and
 //           a histogram of the top 11 bits of each score's order-preserving
 //           key.
-//   filter  one wave of CTAs, several per (sequence, head), each over a slice
-//           of the scores. From the histogram every CTA knows the bin holding
-//           the k-th score (as float bounds): it marks the scores above that
-//           bin in a per-row bitmap (every 32-token word is owned by one CTA,
-//           so plain stores) and appends the bin's members to the row's
-//           candidate list through a shared buffer. The last CTA of a row to
+//   filter  about one CTA per SM, several per (sequence, head), each over a
+//           slice of the scores (the SMs keep room for the attention kernel
+//           launched behind it, which streams the window meanwhile). From the
+//           histogram every CTA knows the bin holding the k-th score (as float
+//           bounds): it marks the scores above that bin in a per-row bitmap
+//           (every 32-token word is owned by one CTA, so plain stores) and the
+//           bin's members in a shared bitmap; the members are then compacted,
+//           their keys read back, and appended to the row's candidate list
+//           through a shared buffer. The last CTA of a row to
 //           finish loads the candidates into shared memory, settles the bin by
 //           a radix search over their remaining bits (exact ties: smallest
 //           token first), sets their bits and compacts the bitmap into the
@@ -37,7 +40,7 @@ constexpr int kBins = 2048;                                        // top 11 bit
 constexpr int kFiltThreads = 512;
 constexpr int kFiltStep = kFiltThreads * 16;                       // scores per CTA step
 constexpr int kMaxTopk = 4096;
-constexpr int kLocCap = 2048;                                      // shared slots for a CTA's candidates
+constexpr int kLocCap = 4096;                                      // shared slots for a CTA's candidates
 constexpr int kSmemCand = 4096;                                    // shared slots for a row's candidates
 constexpr int kSmemWords = 4096;                                   // shared bitmap words (rows up to 128K)
 
@@ -263,12 +266,15 @@ decode_filter_kernel(const DecodeWs w, int L, int Hr, int topk, int slice, int n
   __syncthreads();
 
   // A. this CTA's slice, two steps of 512 scores per warp at a time (all
-  //    loads in flight together): bits for the scores above bin d1; the
-  //    bin's members go to a shared buffer, then to the row's candidate list
-  //    with one reservation. A lane takes 16 consecutive scores; lanes 2m,
-  //    2m+1 share one bitmap word.
+  //    loads in flight together): the row's bitmap words for the scores above
+  //    bin d1, and a shared bitmap of the bin's members. A lane takes 16
+  //    consecutive scores; lanes 2m, 2m+1 share one bitmap word. Then the
+  //    members' tokens are compacted into a shared buffer (in token order),
+  //    their keys read back with all loads in flight, and the buffer goes to
+  //    the row's candidate list with one reservation.
   const int lo = part * slice, hi = min(L, lo + slice);
   const bool vec = (L & 3) == 0;
+  uint32_t* ibits = fs.bits;                    // phase A: the bin's members of this slice (phase B reuses it)
   // bin d1 as float bounds: a score is in the bin iff lo_f <= x < hi_f
   // (no score lies above the top bin: hi_f is then NaN)
   const float lo_f = key_floor_float(d1 << 21);
@@ -304,34 +310,62 @@ decode_filter_kernel(const DecodeWs w, int L, int Hr, int topk, int slice, int n
         bits &= valid;
         cbits &= valid;
       }
-      if (__any_sync(0xffffffffu, cbits != 0)) {
-        const int nc = __popc(cbits);
-        int incl = nc;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        int cbase = 0;
-        if (lane == 31) cbase = atomicAdd(&n_loc, incl);
-        cbase = __shfl_sync(0xffffffffu, cbase, 31);
-        int pos = cbase + incl - nc;
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if ((cbits >> e) & 1u) {
-            const uint32_t key = f2key(x[h][e]);
-            if (pos < kLocCap) loc[pos] = make_uint2(key, (uint32_t)(base + e));
-            else {
-              // the shared buffer is full: straight to the row's list
-              const int gp = atomicAdd(&w.state[row].n_cand, 1);
-              if (gp < cap) cand[gp] = make_uint2(key, (uint32_t)(base + e));
-            }
-            ++pos;
-          }
-      }
-      uint32_t word = bits << ((lane & 1) * 16);
+      uint32_t word = bits << ((lane & 1) * 16), cword = cbits << ((lane & 1) * 16);
       word |= __shfl_xor_sync(0xffffffffu, word, 1);
-      if (!(lane & 1) && base < hi) bm[base >> 5] = word;
+      cword |= __shfl_xor_sync(0xffffffffu, cword, 1);
+      if (!(lane & 1) && base < hi) {
+        bm[base >> 5] = word;
+        ibits[(base - lo) >> 5] = cword;
+      }
+    }
+  }
+  __syncthreads();
+  {
+    // members' tokens, word by word (the loop bound is warp-uniform: the
+    // lanes exchange counts)
+    const int n_words = (hi - lo + 31) >> 5;
+    for (int wbase = warp * 32; wbase < n_words; wbase += kFiltThreads) {
+      const int wi = wbase + lane;
+      uint32_t cw = wi < n_words ? ibits[wi] : 0u;
+      const int nc = __popc(cw);
+      int incl = nc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int wtot = __shfl_sync(0xffffffffu, incl, 31);
+      int cbase = 0;
+      if (lane == 31 && wtot > 0) cbase = atomicAdd(&n_loc, wtot);
+      cbase = __shfl_sync(0xffffffffu, cbase, 31);
+      int pos = cbase + incl - nc;
+      while (cw) {
+        const int e = __ffs(cw) - 1;
+        cw &= cw - 1;
+        const uint32_t tok = (uint32_t)(lo + wi * 32 + e);
+        if (pos < kLocCap) loc[pos].y = tok;
+        else {
+          // the shared buffer is full: straight to the row's list
+          const int gp = atomicAdd(&w.state[row].n_cand, 1);
+          if (gp < cap) cand[gp] = make_uint2(f2key(__ldcg(s + tok)), tok);
+        }
+        ++pos;
+      }
+    }
+    __syncthreads();
+    // the members' keys, all loads of a thread in flight
+    const int n_l = min(n_loc, kLocCap);
+    constexpr int kPer = kLocCap / kFiltThreads;
+    float v[kPer];
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+      const int xx = tid + t * kFiltThreads;
+      v[t] = xx < n_l ? __ldcg(s + loc[xx].y) : 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+      const int xx = tid + t * kFiltThreads;
+      if (xx < n_l) loc[xx].x = f2key(v[t]);
     }
   }
   __syncthreads();
@@ -550,8 +584,14 @@ cudaError_t launch_select_decode(const float* qt, const void* kindex, int B, int
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_filter_kernel, kFiltThreads, sizeof(FiltSmem));
   if (e != cudaSuccess) return e;
+  // about one filter CTA per SM, so that the attention launched behind the
+  // filter finds room to start streaming the window while the filter runs;
+  // a slice fits the shared bitmap of its bin members
   const int rows = B * Hr;
-  int n_split = (per_sm > 0 ? per_sm : 1) * sms / rows;
+  (void)per_sm;
+  int n_split = sms / rows;
+  const int min_split = (L + kSmemWords * 32 - 1) / (kSmemWords * 32);
+  if (n_split < min_split) n_split = min_split;
   if (n_split < 1) n_split = 1;
   int slice = (L + n_split - 1) / n_split;
   slice = (slice + 511) / 512 * 512;

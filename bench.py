@@ -216,7 +216,7 @@ MEASURED_TRAFFIC = {
     ("prefill_1m", "swa_prefill"): 21796575744 + 7232377088,
     # decode step: scan + filter + attention + merge (cold cache, as the bench
     # flushes L2 before each step)
-    ("decode_128k_b8", "step"): 134314496 + 6625792 + 21372928 + 173754880 + 3980032 + 6119168,
+    ("decode_128k_b8", "step"): 134311936 + 6669824 + 21367296 + 173760768 + 3689216 + 6118912,
 }
 
 

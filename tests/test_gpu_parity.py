@@ -137,7 +137,10 @@ def test_select_decode_candidate_overflow_falls_back_exactly():
 # ---------------------------------------------------------------------------
 # Prefill selection
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("N,topk", [(1536, 5), (256, 8), (64, 1), (4096, 16)])
+# 192 and 2368: an odd number of query blocks (the last CTA has one); 9600:
+# more than 16 full key tiles per CTA, so the staged row maxima are folded
+# several times
+@pytest.mark.parametrize("N,topk", [(1536, 5), (256, 8), (64, 1), (4096, 16), (192, 2), (2368, 9), (9600, 20)])
 def test_select_prefill_matches_oracle(N, topk):
     B, Hkv, kv = 1, 2, [0, 1, 1]
     kt = _clustered_bf16((B, Hkv, N, 16), 20 + N)

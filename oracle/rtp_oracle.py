@@ -243,6 +243,93 @@ def attend_decode(q, kc, vc, keys_idx, scale: float) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# 8-bit key index
+# ---------------------------------------------------------------------------
+QGROUP = 64
+
+
+def quantize_index(kt, group: int = QGROUP):
+    """The 8-bit key index: symmetric int8 codes with one fp32 scale per group
+    of ``group`` consecutive tokens of one KV head (the "mixed-precision index
+    system" section of the Baidu article on layered long-context attention: an
+    8-bit quantised indexer; the pages fix no scheme, so this is the plain one).
+
+    ``kt`` [L, r] holds the bf16 index values; only the L // group full groups
+    are quantised (a partial last group stays in bf16). Per group, in fp32
+    arithmetic (so that both sides take every rounding decision alike):
+    amax = max |x|, s = amax / 127 (one fp32 division), and each code is x / s
+    (one fp32 division) rounded half to even and clamped to [-127, 127]; an
+    all-zero group gets s = 0 and zero codes. Returns (codes [n_full*group, r]
+    int8, scales [n_full] float32).
+    """
+    x = to_f64(kt).astype(np.float32)            # bf16 values are exact in fp32
+    n_full = x.shape[0] // group
+    r = x.shape[1]
+    codes = np.zeros((n_full * group, r), np.int8)
+    scales = np.zeros(n_full, np.float32)
+    for gi in range(n_full):
+        blk = x[gi * group:(gi + 1) * group]
+        amax = np.float32(np.abs(blk).max())
+        if amax == 0:
+            continue
+        s_g = np.float32(amax / np.float32(127.0))
+        q = np.rint(blk / s_g)                   # float32 / float32: one IEEE division each
+        codes[gi * group:(gi + 1) * group] = np.clip(q, -127, 127).astype(np.int8)
+        scales[gi] = s_g
+    return codes, scales
+
+
+def decode_scores_q8(qt, codes, scales, kt_tail, group: int = QGROUP) -> np.ndarray:
+    """Decode scores over an 8-bit index: score_u = s_g * sum_c qt_c code_{u,c}
+    for the tokens of full groups (g = u // group), and qt . kt[u] over the
+    bf16 rows of the partial last group (``kt_tail``). Exact in fp64."""
+    qt = to_f64(qt)
+    full = (codes.astype(np.float64) @ qt) * np.repeat(scales.astype(np.float64), group)
+    tail = to_f64(kt_tail) @ qt if len(kt_tail) else np.zeros(0)
+    return np.concatenate([full, tail])
+
+
+# ---------------------------------------------------------------------------
+# Static patterns on the same attention (presets)
+# ---------------------------------------------------------------------------
+def triangle_keys(t: int, N: int, sink_blocks: int, window_blocks: int, last_tokens: int,
+                  block: int = BLOCK) -> np.ndarray:
+    """Keys of query row t under the triangle-shaped mask (TriangleMix
+    interview, 36kr, paragraph on the triangle-shaped mask): rows of the last
+    Q-K region (t >= N - last_tokens) keep every causal key; every other row
+    keeps only the streaming region, the sink blocks and the local band of
+    blocks ending at its own block (block-granular, like the retrieval heads'
+    window), causal."""
+    if t >= N - last_tokens:
+        return np.arange(0, t + 1)
+    i = t // block
+    blocks = np.union1d(np.arange(0, min(sink_blocks, i + 1)), np.arange(max(0, i - window_blocks + 1), i + 1))
+    keys = np.concatenate([np.arange(j * block, (j + 1) * block) for j in blocks])
+    return keys[keys <= t]
+
+
+def triangle_rows(q, k, v, rows, sink_blocks: int, window_blocks: int, last_tokens: int,
+                  scale: float, block: int = BLOCK) -> np.ndarray:
+    """Triangle-mask attention of query rows ``rows`` of one head (q [N, D],
+    k/v [N, D] of its KV head), one row at a time."""
+    N = k.shape[0]
+    q64, k64, v64 = to_f64(q), to_f64(k), to_f64(v)
+    out = []
+    for t in rows:
+        keys = triangle_keys(int(t), N, sink_blocks, window_blocks, last_tokens, block)
+        out.append(attend(q64[t:t + 1], [t], k64[keys], v64[keys], keys, scale)[0])
+    return np.stack(out)
+
+
+def dense_decode(q, kc, vc, scale: float) -> np.ndarray:
+    """Full attention of one query (at the last position) over the whole
+    cache: the cross-attention of an output position in Orthros (Orthros
+    article, section on one attention with two working modes; the trained
+    Scale-Offset of its query is out of scope, so the query is used as is)."""
+    return attend_decode(q, kc, vc, np.arange(kc.shape[0]), scale)
+
+
+# ---------------------------------------------------------------------------
 # Whole-layer drivers
 # ---------------------------------------------------------------------------
 def kv_of(h: int, Hq: int, Hkv: int) -> int:
@@ -297,11 +384,13 @@ def prefill_layer(q, k, v, P, ret_heads, window: int, ret_window: int, topk: int
 
 
 def decode_layer(q, kc, vc, P, ret_heads, window: int, ret_window: int, topk: int,
-                 scale: float, sink: int = 1, heads=None):
+                 scale: float, sink: int = 1, heads=None, index_bits: int = 16):
     """One decode step for one sequence.
 
     ``q`` [Hq, D], ``kc``/``vc`` [L, Hkv, D], ``P`` [Hkv, D, r]. The key index
     is the bf16-rounded projection of the cache; the query index is unrounded.
+    ``index_bits`` = 8 scores over the 8-bit form of that index
+    (``quantize_index``; its partial last group stays bf16).
     Returns ``out`` {h: [D]}, ``sel``/``scores`` {h: ...}.
     """
     q, P = to_f64(q), to_f64(P)
@@ -317,7 +406,11 @@ def decode_layer(q, kc, vc, P, ret_heads, window: int, ret_window: int, topk: in
                 res["kt"][g] = project(kc[:, g, :], P[g])
             kt = res["kt"][g]
             qt = project(q[h], P[g], round_to_bf16=False)
-            sc = decode_scores(qt, kt)
+            if index_bits == 8:
+                codes, scales = quantize_index(kt)
+                sc = decode_scores_q8(qt, codes, scales, kt[len(codes):])
+            else:
+                sc = decode_scores(qt, kt)
             sel = topk_desc(sc, topk)
             res["sel"][h], res["scores"][h] = sel, sc
             idx = decode_attended(sel, L, ret_window, sink)
@@ -331,5 +424,6 @@ __all__ = [
     "BLOCK", "bf16_round", "to_f64", "project", "block_scores", "topk_desc", "select_prefill",
     "attended_blocks", "attend", "sparse_attn_prefill_block", "swa_rows", "decode_scores",
     "select_decode", "decode_attended", "attend_decode", "kv_of", "prefill_layer",
-    "decode_layer",
+    "decode_layer", "triangle_keys", "triangle_rows", "dense_decode", "QGROUP", "quantize_index",
+    "decode_scores_q8",
 ]

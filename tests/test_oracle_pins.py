@@ -427,3 +427,181 @@ def test_planted_mistakes_are_caught():
     g = json.load(open(os.path.join(GOLDEN, "block_select_hand.json")))
     wrong = np.unique(np.concatenate([np.array(g["selected"]["3"]), [0], np.arange(0, 1)]))
     assert list(wrong) != g["attended"]["3"]
+
+
+# ---------------------------------------------------------------------------
+# Static patterns: triangle-shaped mask, dense (full cross-attention) decode
+# ---------------------------------------------------------------------------
+def _ranges_to_keys(ranges):
+    return np.concatenate([np.arange(a, b + 1) for a, b in ranges])
+
+
+def _golden_triangle_ok(keys_fn):
+    g = json.load(open(os.path.join(GOLDEN, "triangle_mask_hand.json")))
+    for c in g["cases"]:
+        got = keys_fn(c["t"], g["N"], c["sink_blocks"], c["window_blocks"], c["last_tokens"], g["block"])
+        if not np.array_equal(np.asarray(got), _ranges_to_keys(c["ranges"])):
+            return False
+    return True
+
+
+def test_golden_triangle_key_sets():
+    assert _golden_triangle_ok(O.triangle_keys)
+
+
+def test_triangle_uniform_attention_averages_the_key_set():
+    """q = 0 makes every logit equal, so each output row is the plain mean of
+    the attended value rows: with v_u = e_u the row is 1/|set| on the set."""
+    g = json.load(open(os.path.join(GOLDEN, "triangle_mask_hand.json")))
+    N, D = g["N"], g["N"]
+    q = np.zeros((N, D))
+    k = _bf16_arr((N, D), 1, np.random.default_rng(30))
+    v = np.eye(N)
+    for c in g["cases"]:
+        o = O.triangle_rows(q, k, v, [c["t"]], c["sink_blocks"], c["window_blocks"], c["last_tokens"], 0.3)[0]
+        want = np.zeros(N)
+        keys = _ranges_to_keys(c["ranges"])
+        want[keys] = 1.0 / len(keys)
+        np.testing.assert_allclose(o, want, rtol=0, atol=1e-15)
+
+
+def test_triangle_whole_last_region_is_dense_causal():
+    rs = np.random.default_rng(31)
+    N, D = 256, 128
+    q, k, v = _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs)
+    scale = 1 / math.sqrt(D)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, None], torch.from_numpy(k)[None, None],
+        torch.from_numpy(v)[None, None], is_causal=True, scale=scale)[0, 0].numpy()
+    rows = np.arange(N)
+    np.testing.assert_allclose(O.triangle_rows(q, k, v, rows, 1, 1, N, scale), ref, rtol=0, atol=1e-12)
+    # no last region but a band covering every block: dense causal as well
+    np.testing.assert_allclose(O.triangle_rows(q, k, v, rows, 0, N // 64, 0, scale), ref, rtol=0, atol=1e-12)
+
+
+def test_triangle_matches_masked_sdpa():
+    rs = np.random.default_rng(32)
+    N, D, block = 384, 64, 64
+    q, k, v = _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs), _bf16_arr((N, D), 1, rs)
+    sink, wb, last = 1, 2, 128
+    t = np.arange(N)
+    kb, qb = t[None, :] // block, t[:, None] // block
+    # mask from the golden's wording: last rows see every causal key; others
+    # see sink blocks and the band of wb blocks ending at their own block
+    mask = (t[None, :] <= t[:, None]) & ((t[:, None] >= N - last) | (kb < sink) | (kb > qb - wb))
+    ref = _sdpa_masked(q, k, v, mask, 0.125)
+    np.testing.assert_allclose(O.triangle_rows(q, k, v, t, sink, wb, last, 0.125), ref, rtol=0, atol=1e-12)
+
+
+def test_dense_decode_is_full_attention():
+    rs = np.random.default_rng(33)
+    L, D = 700, 128
+    q, kc, vc = _bf16_arr((D,), 1, rs), _bf16_arr((L, D), 1, rs), _bf16_arr((L, D), 1, rs)
+    ref = _sdpa_masked(q[None], kc, vc, np.ones((1, L), bool), 1 / math.sqrt(D))[0]
+    np.testing.assert_allclose(O.dense_decode(q, kc, vc, 1 / math.sqrt(D)), ref, rtol=0, atol=1e-12)
+
+
+def test_planted_triangle_mistakes_are_caught():
+    def last_region_off_by_one(t, N, sink, wb, last, block):     # '>' instead of '>='
+        if t > N - last:
+            return np.arange(0, t + 1)
+        return O.triangle_keys(t, N, sink, wb, 0, block)
+
+    def band_without_own_block(t, N, sink, wb, last, block):     # band ends one block early
+        if t >= N - last:
+            return np.arange(0, t + 1)
+        i = t // block
+        blocks = np.union1d(np.arange(0, min(sink, i + 1)), np.arange(max(0, i - wb), i))
+        keys = np.concatenate([np.arange(j * block, (j + 1) * block) for j in blocks]) if len(blocks) else \
+            np.arange(0)
+        return keys[keys <= t]
+
+    assert not _golden_triangle_ok(last_region_off_by_one)
+    assert not _golden_triangle_ok(band_without_own_block)
+
+
+# ---------------------------------------------------------------------------
+# 8-bit key index
+# ---------------------------------------------------------------------------
+def _golden_q8_ok(quant):
+    import struct
+    g = json.load(open(os.path.join(GOLDEN, "index_q8_hand.json")))
+    kt = np.array(g["kt"])
+    codes, scales = quant(kt, g["group"])
+    if codes.tolist() != g["codes"]:
+        return False
+    hexes = [hex(struct.unpack("<I", struct.pack("<f", float(x)))[0]) for x in scales]
+    if [int(h, 16) for h in hexes] != [int(h, 16) for h in g["scales_f32_hex"]]:
+        return False
+    sc = O.decode_scores_q8(g["q"], codes, scales, kt[len(codes):], g["group"])
+    return all(sc[int(r)] == v for r, v in g["scores_by_row"].items()) and \
+        sc[2] / float(scales[1]) == g["score_row2_over_s1"]
+
+
+def test_golden_index_q8():
+    assert _golden_q8_ok(O.quantize_index)
+
+
+def test_index_q8_reconstruction_bound_and_extremes():
+    """Each code times its scale lies within half a step (s/2) of the bf16
+    value, plus what the fp32 division x / s may move the quotient by (half
+    an fp32 ulp of a quotient below 128: 2^-17 code units), and a group's
+    largest magnitude maps to +-127."""
+    rs = np.random.default_rng(40)
+    kt = O.bf16_round(rs.standard_normal((64 * 37 + 13, 16)) * rs.uniform(0.01, 30, (64 * 37 + 13, 1)))
+    codes, scales = O.quantize_index(kt)
+    assert codes.shape == (64 * 37, 16) and scales.shape == (37,)
+    rec = codes.astype(np.float64) * np.repeat(scales.astype(np.float64), 64)[:, None]
+    err = np.abs(rec - kt[:64 * 37])
+    assert np.all(err <= np.repeat(scales.astype(np.float64), 64)[:, None] * (0.5 + 2.0 ** -17))
+    for gi in range(37):
+        blk = codes[gi * 64:(gi + 1) * 64]
+        assert np.abs(blk).max() == 127
+
+
+def test_index_q8_scores_track_the_bf16_scores():
+    """The 8-bit scores differ from the bf16 ones by at most sum_c |q_c| (s/2
+    + the fp32 quotient rounding, 2^-17 s)."""
+    rs = np.random.default_rng(41)
+    kt = O.bf16_round(rs.standard_normal((4096, 16)))
+    q = rs.standard_normal(16)
+    codes, scales = O.quantize_index(kt)
+    sc8 = O.decode_scores_q8(q, codes, scales, kt[len(codes):])
+    sc16 = O.decode_scores(q, kt)
+    bound = np.abs(q).sum() * np.repeat(scales.astype(np.float64), 64) * (0.5 + 2.0 ** -17)
+    assert np.all(np.abs(sc8 - sc16) <= bound)
+
+
+def test_planted_q8_mistakes_are_caught():
+    def truncating(kt, group):                     # round toward zero instead of half to even
+        x = O.to_f64(kt).astype(np.float32)
+        n = x.shape[0] // group
+        codes = np.zeros((n * group, x.shape[1]), np.int8)
+        scales = np.zeros(n, np.float32)
+        for gi in range(n):
+            blk = x[gi * group:(gi + 1) * group]
+            a = np.float32(np.abs(blk).max())
+            if a == 0:
+                continue
+            s_g = np.float32(a / np.float32(127.0))
+            codes[gi * group:(gi + 1) * group] = np.clip(np.trunc(blk / s_g), -127, 127).astype(np.int8)
+            scales[gi] = s_g
+        return codes, scales
+
+    def scale_by_128(kt, group):                   # step amax/128: the largest value overflows
+        x = O.to_f64(kt).astype(np.float32)
+        n = x.shape[0] // group
+        codes = np.zeros((n * group, x.shape[1]), np.int8)
+        scales = np.zeros(n, np.float32)
+        for gi in range(n):
+            blk = x[gi * group:(gi + 1) * group]
+            a = np.float32(np.abs(blk).max())
+            if a == 0:
+                continue
+            s_g = np.float32(a / np.float32(128.0))
+            codes[gi * group:(gi + 1) * group] = np.clip(np.rint(blk / s_g), -127, 127).astype(np.int8)
+            scales[gi] = s_g
+        return codes, scales
+
+    assert not _golden_q8_ok(truncating)
+    assert not _golden_q8_ok(scale_by_128)

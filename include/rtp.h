@@ -83,26 +83,21 @@ RTP_API const char* rtp_status_string(rtp_status s);
 RTP_API int rtp_version(void);
 
 /*
- * rtp_workspace_status - device-side status of the last call that used `ws`.
- *   The prefill and decode attention calls keep a status word in the first
- *   bytes of their workspace: cleared on the stream before the launch, set to
- *   RTP_ERR_TIMEOUT by a CTA whose bounded wait ran out (the kernel then
- *   drains and returns instead of spinning). This call synchronises `stream`
- *   and returns RTP_OK or the recorded status.
+ * rtp_get_device_status - the device-side status of the last call that used
+ * the workspace `ws`.
+ *   The tensor-core prefill calls (rtp_select_prefill, rtp_sparse_attn_prefill
+ *   and rtp_swa with Nq > 1) keep a status word in the first bytes of their
+ *   workspace: cleared on the stream before their launch and set to
+ *   RTP_ERR_TIMEOUT by a thread block whose bounded wait ran out (that block
+ *   then drains its copies, frees its tensor memory and returns instead of
+ *   spinning). The decode calls keep the same word and always leave RTP_OK in
+ *   it: their kernels never wait on one another on the device.
+ *   This call synchronises `stream` (the word is read after every call queued
+ *   on it before), then writes the recorded status to *out (RTP_OK when the
+ *   word is zero). Returns RTP_ERR_INVALID_ARG for a NULL `ws` or `out`,
+ *   RTP_ERR_CUDA if the synchronisation or the read fails, else RTP_OK.
  */
-RTP_API rtp_status rtp_workspace_status(const void* ws, rtp_stream_t stream);
-
-/*
- * rtp_debug_prefill_timeout_probe - test hook for the bounded waits.
- *   Launches one CTA of the prefill attention kernel on a 128-token, one-head
- *   sliding-window problem whose producer deliberately never loads Q, so the
- *   CTA's waits run out (about 2 s), it drains its copies, frees its tensor
- *   memory and records RTP_ERR_TIMEOUT in the status word of `ws` (read it
- *   with rtp_workspace_status). q, k, v, o: bf16 [1, 128, 1, 128] device
- *   buffers (o is not written). The device stays usable afterwards.
- */
-RTP_API rtp_status rtp_debug_prefill_timeout_probe(const void* q, const void* k, const void* v, void* o, void* ws,
-                                                   size_t ws_bytes, rtp_stream_t stream);
+RTP_API rtp_status rtp_get_device_status(const void* ws, rtp_stream_t stream, rtp_status* out);
 
 /*
  * rtp_index_project - the low-rank indexer projection x~ = x . P.
@@ -126,6 +121,31 @@ RTP_API rtp_status rtp_index_project(const void* x, rtp_strides xs, int B, int N
                              void* out, rtp_dtype out_dtype, rtp_stream_t stream);
 
 /*
+ * rtp_index_append - keeps the decode key index in step with the KV cache:
+ * projects the keys of new tokens into their rows of the index.
+ *   Source: RTPurboV2 article, paragraph on the low-rank projector (keys
+ *   projected from D to r = 16) and the Qwen3-Coder-30B-A3B recipe (the
+ *   sparse indexer runs in the decode stage); the 128K decode workload
+ *   statement (a 16-d key index of shape [KV heads, context, 16] beside the
+ *   cache). The pages give no maintenance scheme; the plain reading is that
+ *   the index holds bf16(k . P_g) for every cached token, so every token that
+ *   enters the cache enters the index the same way.
+ *
+ *   k        bf16 [B, n_new, Hkv, D] device (strides ks): the keys of the new
+ *            tokens, every KV head (for the prefill -> decode handoff, the
+ *            whole prefill K with n_new = N and pos = 0; for a decode step,
+ *            the new token's row with n_new = 1 and pos = L - 1).
+ *   P        bf16 [Hkv, D, r] device, contiguous: KV head g uses P[g].
+ *   kindex   bf16 [B, Hkv, cap, r] device, contiguous, written at rows
+ *            pos .. pos + n_new - 1 of every (sequence, KV head) with the
+ *            bf16 rounding of the fp32 dot products (as rtp_index_project);
+ *            other rows are untouched.
+ *   r = 16, pos >= 0, pos + n_new <= cap, Hkv <= 128.
+ */
+RTP_API rtp_status rtp_index_append(const void* k, rtp_strides ks, int B, int n_new, int Hkv, const void* P, int r,
+                                    void* kindex, int64_t cap, int pos, rtp_stream_t stream);
+
+/*
  * rtp_select_prefill - per query block, the top-k key blocks by block score.
  *   Source: block score = max over the (query, key) pairs of a 64 x 64
  *   block pair of q~ . k~, each query block keeping its top-k causal key
@@ -135,20 +155,22 @@ RTP_API rtp_status rtp_index_project(const void* x, rtp_strides xs, int B, int N
  *   the smaller block first. The token score matrix is never materialised.
  *
  *   qt       bf16 [B, Hr, N, r] device, contiguous (projected retrieval-head queries).
- *   kt       bf16 [B, Hkv, N, r] device, contiguous (projected keys).
+ *   kt       bf16 [B, Hkv, kt_cap, r] device, contiguous (projected keys; rows
+ *            0 .. N-1 are read). kt_cap >= N: a key index kept with headroom
+ *            for decode (see rtp_index_append) serves as is.
  *   kv_of    host int32 [Hr]: KV head of each retrieval head.
  *   topk     k >= 1 selected blocks per query block.
  *   blocks   int32 [B, Hr, N/64, topk] device out: ascending block indices,
  *            min(k, i+1) of them, the rest -1.
  *   counts   int32 [B, Hr, N/64] device out: min(k, i+1).
  *   ws       workspace of rtp_workspace_size_select_prefill() bytes (the
- *            status word, see rtp_workspace_status).
+ *            status word, see rtp_get_device_status).
  *   N must be a multiple of 64, r = 16; the block scores of a query-block
  *   pair are kept on chip, which bounds N at about 1.4M tokens
  *   (RTP_ERR_UNSUPPORTED beyond).
  */
 RTP_API size_t rtp_workspace_size_select_prefill(int B, int N, int Hr, int topk);
-RTP_API rtp_status rtp_select_prefill(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
+RTP_API rtp_status rtp_select_prefill(const void* qt, const void* kt, int64_t kt_cap, int B, int N, int Hr, int Hkv,
                               int r, const int32_t* kv_of, int topk,
                               int32_t* blocks, int32_t* counts,
                               void* ws, size_t ws_bytes, rtp_stream_t stream);
@@ -160,18 +182,59 @@ RTP_API rtp_status rtp_select_prefill(const void* qt, const void* kt, int B, int
  *   Exact ties rank the smaller token first.
  *
  *   qt       fp32 [B, Hr, r] device (unrounded projected decode queries).
- *   kindex   bf16 [B, Hkv, L, r] device, contiguous (the key index).
+ *   kindex   bf16 [B, Hkv, kindex_cap, r] device, contiguous (the key index;
+ *            rows 0 .. L-1 are the cache's tokens). kindex_cap >= L.
  *   kv_of    host int32 [Hr].
  *   idx      int32 [B, Hr, topk] device out: ascending token indices;
  *            min(k, L) of them, the rest -1.
  *   ws       workspace of rtp_workspace_size_select_decode() bytes.
- *   r = 16, 1 <= topk <= 4096, L >= 1; Hkv <= 16 and at most 16 retrieval
+ *   r = 16, 1 <= topk <= 4194304 (topk >= L selects every token: the dense
+ *   preset of a full cross-attention decode), L >= 1; Hkv <= 16 and at most 16 retrieval
  *   heads per KV group (RTP_ERR_UNSUPPORTED otherwise).
  */
 RTP_API size_t rtp_workspace_size_select_decode(int B, int L, int Hr, int topk);
-RTP_API rtp_status rtp_select_decode(const float* qt, const void* kindex, int B, int L, int Hr, int Hkv,
+RTP_API rtp_status rtp_select_decode(const float* qt, const void* kindex, int64_t kindex_cap, int B, int L, int Hr,
+                                     int Hkv,
                              int r, const int32_t* kv_of, int topk, int32_t* idx,
                              void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * rtp_index_quantize - the 8-bit form of the decode key index.
+ *   Source: the Baidu developer article on layered long-context attention
+ *   ("深度解析：超长上下文注意力架构的分层优化策略"), section on the
+ *   mixed-precision index system: an 8-bit quantised indexer that cuts the
+ *   index storage (here the bytes the decode scan reads) with a small loss of
+ *   precision. The page fixes no scheme; this is the plain symmetric one.
+ *   Per group of 64 consecutive tokens of one (sequence, KV head): amax =
+ *   max |x| over its 64 x 16 bf16 values, s = amax / 127 and code =
+ *   round-half-even(x / s) clamped to [-127, 127], both divisions IEEE fp32;
+ *   an all-zero group gets s = 0 and zero codes.
+ *
+ *   kindex   bf16 [B, Hkv, cap, 16] device (the bf16 index, rtp_index_append).
+ *   kindex8  int8 [B, Hkv, cap, 16] device out: codes of the tokens of groups
+ *            g0 .. g1-1 (tokens 64 g0 .. 64 g1 - 1); other rows untouched.
+ *   kscale   fp32 [B, Hkv, ceil(cap / 64)] device out: the groups' scales.
+ *   0 <= g0 <= g1, 64 g1 <= cap. A decode loop quantises each group once it
+ *   is full (after appending token 64 g + 63); the partial last group is
+ *   scanned from the bf16 rows.
+ */
+RTP_API rtp_status rtp_index_quantize(const void* kindex, int64_t cap, int B, int Hkv, int g0, int g1, void* kindex8,
+                                      float* kscale, rtp_stream_t stream);
+
+/*
+ * rtp_select_decode_q8 - rtp_select_decode over the 8-bit key index.
+ *   Source: as rtp_index_quantize and rtp_select_decode. Tokens of the full
+ *   64-token groups, 0 .. 64 floor(L/64) - 1, are scored s * sum_c q~_c code_c
+ *   (fp32) from kindex8 / kscale, which must hold every full group
+ *   (rtp_index_quantize); the rest from the bf16 rows of kindex. Selection,
+ *   ties, outputs, limits and workspace as rtp_select_decode (same
+ *   rtp_workspace_size_select_decode). The scan reads 16 bytes per token
+ *   instead of 32.
+ */
+RTP_API rtp_status rtp_select_decode_q8(const float* qt, const void* kindex8, const float* kscale, const void* kindex,
+                                        int64_t kindex_cap, int B, int L, int Hr, int Hkv, int r,
+                                        const int32_t* kv_of, int topk, int32_t* idx, void* ws, size_t ws_bytes,
+                                        rtp_stream_t stream);
 
 /*
  * rtp_sparse_attn_prefill - exact attention of retrieval heads over their
@@ -194,7 +257,7 @@ RTP_API rtp_status rtp_select_decode(const float* qt, const void* kindex, int B,
  *   window_blocks >= 1, sink_blocks >= 0, scale > 0 (the softmax scale,
  *   1/sqrt(D) in the method's usual form).
  *   ws       at least rtp_workspace_size_sparse_attn_prefill() bytes (the
- *            status word, see rtp_workspace_status).
+ *            status word, see rtp_get_device_status).
  */
 RTP_API size_t rtp_workspace_size_sparse_attn_prefill(int B, int N, int Hr, int topk);
 RTP_API rtp_status rtp_sparse_attn_prefill(const void* q, rtp_strides qs, const void* k, rtp_strides ks,
@@ -203,6 +266,38 @@ RTP_API rtp_status rtp_sparse_attn_prefill(const void* q, rtp_strides qs, const 
                                    const int32_t* blocks, const int32_t* counts, int topk,
                                    int window_blocks, int sink_blocks, float scale,
                                    void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * rtp_triangle_prefill - prefill attention under the triangle-shaped mask of
+ * TriangleMix, a static pattern on the same kernels.
+ *   Source: the TriangleMix interview (36kr, "微软研究院杨玉庆：Agent 的注意力系统"),
+ *   paragraph on the triangle-shaped mask: deep layers skip the middle Q-K
+ *   region and keep only the streaming region (the first keys and the local
+ *   band) and the last Q-K region (the last queries against every key). The
+ *   page gives no sizes; this call takes them as arguments, with the sink and
+ *   the band block-granular as for the retrieval heads of
+ *   rtp_sparse_attn_prefill.
+ *   Query row t (block i = t / 64) attends the keys u <= t
+ *     - in blocks {0 .. sink_blocks-1} U {i-window_blocks+1 .. i}, for
+ *       t < N - last_tokens (the streaming region);
+ *     - all of them, for t >= N - last_tokens (the last Q-K region).
+ *   With last_tokens = N this is dense causal attention.
+ *
+ *   q, o     bf16 [B, N, Hq, D] device (strides qs, os); o written only for
+ *            the listed heads.
+ *   k, v     bf16 [B, N, Hkv, D] device (strides ks, vs).
+ *   heads    host int32 [n_heads].
+ *   N and last_tokens multiples of 64 (RTP_ERR_UNSUPPORTED otherwise),
+ *   0 <= last_tokens <= N, window_blocks >= 1, sink_blocks >= 0, scale > 0.
+ *   ws       rtp_workspace_size_triangle_prefill() bytes: the status word
+ *            (see rtp_get_device_status), shared by the call's two kernels.
+ */
+RTP_API size_t rtp_workspace_size_triangle_prefill(void);
+RTP_API rtp_status rtp_triangle_prefill(const void* q, rtp_strides qs, const void* k, rtp_strides ks,
+                                        const void* v, rtp_strides vs, void* o, rtp_strides os,
+                                        int B, int N, int Hq, int Hkv, const int32_t* heads, int n_heads,
+                                        int sink_blocks, int window_blocks, int last_tokens, float scale,
+                                        void* ws, size_t ws_bytes, rtp_stream_t stream);
 
 /*
  * rtp_sparse_attn_decode - one new query token per sequence attends, per
@@ -217,9 +312,10 @@ RTP_API rtp_status rtp_sparse_attn_prefill(const void* q, rtp_strides qs, const 
  *   kc, vc   bf16 [B, L, Hkv, D] device (strides ks, vs): the cache, whose
  *            last row (L-1) is the new token's own key/value.
  *   heads    host int32 [Hr]; idx int32 [B, Hr, topk] device: distinct
- *            token indices, -1 padded, as written by rtp_select_decode
- *            (entries in the window or below `sink` are skipped there,
- *            since those keys are attended anyway).
+ *            token indices first, then -1 padding, as written by
+ *            rtp_select_decode (entries in the window or below `sink` are
+ *            skipped there, since those keys are attended anyway; with
+ *            topk > L only the first L entries of a row are read).
  *   window >= 1, 0 <= sink <= 64, scale > 0; Hq / Hkv <= 16 and Hkv <= 16
  *   (the query heads of a KV group are packed into one 16-row tensor-core
  *   tile).
@@ -263,19 +359,24 @@ RTP_API rtp_status rtp_decode_attn_hybrid(const void* q, const void* kc, rtp_str
  *   attention's window reads while the selection finishes.
  *   q        bf16 [B, Hq, 128] device, contiguous (the new token's queries).
  *   P        bf16 [Hkv, 128, 16] device (projector per KV head).
- *   kindex   bf16 [B, Hkv, L, 16] device, contiguous (key index of the cache,
- *            including the new token at L - 1).
+ *   kindex   bf16 [B, Hkv, kindex_cap, 16] device, contiguous (key index of
+ *            the cache; rows 0 .. L-1 are read, the new token's at L - 1 included,
+ *            see rtp_index_append). kindex_cap >= L.
+ *   kindex8, kscale  NULL, or the 8-bit index of the same cache
+ *            (rtp_index_quantize): the selection then runs as
+ *            rtp_select_decode_q8 (both NULL or both set).
  *   kc, vc   bf16 [B, L, Hkv, 128] device with element strides ks, vs.
  *   o        bf16 [B, Hq, 128] device out: rows of the listed heads.
  *   ret_heads/swa_heads  host int32 lists (Hr or n_swa may be 0, not both).
  *   idx      int32 [B, Hr, topk] device out (the selected tokens, ascending).
  *   ws       rtp_workspace_size_decode_step(B, L, Hq, Hr, topk,
  *            max(ret_window, swa_window)) bytes, 256-byte aligned; its first
- *            word is the status word read by rtp_workspace_status.
+ *            word is the status word read by rtp_get_device_status.
  *   Limits as in the three calls it combines. Asynchronous on `stream`.
  */
 RTP_API size_t rtp_workspace_size_decode_step(int B, int L, int Hq, int Hr, int topk, int window);
-RTP_API rtp_status rtp_decode_step(const void* q, const void* P, const void* kindex, const void* kc, rtp_strides ks,
+RTP_API rtp_status rtp_decode_step(const void* q, const void* P, const void* kindex, int64_t kindex_cap,
+                                   const void* kindex8, const float* kscale, const void* kc, rtp_strides ks,
                                    const void* vc, rtp_strides vs, void* o, int B, int L, int Hq, int Hkv,
                                    const int32_t* ret_heads, int Hr, int topk, int ret_window, int sink,
                                    const int32_t* swa_heads, int n_swa, int swa_window, float scale, int32_t* idx,
@@ -291,17 +392,22 @@ RTP_API rtp_status rtp_decode_step(const void* q, const void* P, const void* kin
  *   cudaMalloc/cudaFree (both may synchronise the device) on every step.
  *
  *   Arguments, layouts and results are those of rtp_sparse_attn_decode. The
- *   split-K partials and the status word go to a fixed array inside the
- *   library, 4 MiB per GPU, held by every GPU that loads the library until
- *   the process exits. A call whose workspace would not fit (about 256 +
- *   4 * B * Hr * (ceil(window/64) + ceil((topk+64)/64)) * 528 bytes > 4 MiB)
- *   returns RTP_ERR_WORKSPACE and launches nothing. The first call on a device looks up the array's device
- *   address (with that device current) and caches it; make that first call
- *   before any stream capture. Every call shares the one array, so calls
- *   whose work may overlap on the GPU (different streams, or concurrent host
- *   threads) race on it and must be serialised by the caller. Nothing in the
- *   array needs to start at zero: each call writes every partial it reads
- *   and its status word.
+ *   split-K partials go to a fixed array inside the library, 4 MiB per GPU,
+ *   held by every GPU that loads the library until the process exits. A call
+ *   whose partials would not fit (about 256 + 4 * B * Hr * (ceil(window/64) +
+ *   ceil((topk+64)/64)) * 528 bytes > 4 MiB) returns RTP_ERR_WORKSPACE and
+ *   launches nothing.
+ *   The first call on a device looks up the array's device address (with that
+ *   device current) and caches it together with the device's current context;
+ *   a later call under a different context (for instance after
+ *   cudaDeviceReset) looks it up again. Make the first call on each device
+ *   before any stream capture. The call never calls cudaMalloc or cudaFree.
+ *   Every call shares the one array, so calls whose work may overlap on the
+ *   GPU (different streams, or concurrent host threads) race on it and must
+ *   be serialised by the caller. Nothing in the array needs to start at zero:
+ *   each call writes every partial it reads. The decode kernels have no
+ *   device-side waits, so there is no status word to read for this call:
+ *   errors come back in the return value.
  */
 RTP_API rtp_status rtp_sparse_attn_decode_noalloc(const void* q, const void* kc, rtp_strides ks,
                                                   const void* vc, rtp_strides vs, void* o,

@@ -37,19 +37,26 @@ _P = ctypes.c_void_p
 _I = ctypes.c_int
 _F = ctypes.c_float
 _SZ = ctypes.c_size_t
+_L = ctypes.c_int64
 
 _SIGNATURES = {
     "rtp_status_string": (ctypes.c_char_p, [_I]),
     "rtp_version": (_I, []),
-    "rtp_workspace_status": (_I, [_P, _P]),
+    "rtp_get_device_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int)]),
     "rtp_index_project": (_I, [_P, Strides, _I, _I, _I, _P, _I, _I, _c_i32p, _c_i32p, _I, _P, _I, _P]),
     "rtp_workspace_size_select_prefill": (_SZ, [_I, _I, _I, _I]),
-    "rtp_select_prefill": (_I, [_P, _P, _I, _I, _I, _I, _I, _c_i32p, _I, _P, _P, _P, _SZ, _P]),
+    "rtp_index_append": (_I, [_P, Strides, _I, _I, _I, _P, _I, _P, _L, _I, _P]),
+    "rtp_select_prefill": (_I, [_P, _P, _L, _I, _I, _I, _I, _I, _c_i32p, _I, _P, _P, _P, _SZ, _P]),
     "rtp_workspace_size_select_decode": (_SZ, [_I, _I, _I, _I]),
-    "rtp_select_decode": (_I, [_P, _P, _I, _I, _I, _I, _I, _c_i32p, _I, _P, _P, _SZ, _P]),
+    "rtp_select_decode": (_I, [_P, _P, _L, _I, _I, _I, _I, _I, _c_i32p, _I, _P, _P, _SZ, _P]),
+    "rtp_index_quantize": (_I, [_P, _L, _I, _I, _I, _I, _P, _P, _P]),
+    "rtp_select_decode_q8": (_I, [_P, _P, _P, _P, _L, _I, _I, _I, _I, _I, _c_i32p, _I, _P, _P, _SZ, _P]),
     "rtp_workspace_size_sparse_attn_prefill": (_SZ, [_I, _I, _I, _I]),
     "rtp_sparse_attn_prefill": (_I, [_P, Strides, _P, Strides, _P, Strides, _P, Strides, _I, _I, _I,
                                      _I, _c_i32p, _I, _P, _P, _I, _I, _I, _F, _P, _SZ, _P]),
+    "rtp_workspace_size_triangle_prefill": (_SZ, []),
+    "rtp_triangle_prefill": (_I, [_P, Strides, _P, Strides, _P, Strides, _P, Strides, _I, _I, _I, _I, _c_i32p, _I,
+                                  _I, _I, _I, _F, _P, _SZ, _P]),
     "rtp_workspace_size_sparse_attn_decode": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "rtp_sparse_attn_decode": (_I, [_P, _P, Strides, _P, Strides, _P, _I, _I, _I, _I, _c_i32p, _I,
                                     _P, _I, _I, _I, _F, _P, _SZ, _P]),
@@ -57,7 +64,8 @@ _SIGNATURES = {
     "rtp_decode_attn_hybrid": (_I, [_P, _P, Strides, _P, Strides, _P, _I, _I, _I, _I, _c_i32p, _I, _P, _I,
                                     _I, _I, _c_i32p, _I, _I, _F, _P, _SZ, _P]),
     "rtp_workspace_size_decode_step": (_SZ, [_I, _I, _I, _I, _I, _I]),
-    "rtp_decode_step": (_I, [_P, _P, _P, _P, Strides, _P, Strides, _P, _I, _I, _I, _I, _c_i32p, _I, _I, _I, _I,
+    "rtp_decode_step": (_I, [_P, _P, _P, _L, _P, _P, _P, Strides, _P, Strides, _P, _I, _I, _I, _I, _c_i32p, _I, _I,
+                             _I, _I,
                              _c_i32p, _I, _I, _F, _P, _P, _SZ, _P]),
     "rtp_workspace_size_swa": (_SZ, [_I, _I, _I, _I, _I]),
     "rtp_swa": (_I, [_P, Strides, _P, Strides, _P, Strides, _P, Strides, _I, _I, _I, _I, _I, _I,
@@ -116,9 +124,12 @@ def _wsptr(buf):
 
 
 def workspace_status(ws: torch.Tensor, stream=None) -> int:
-    """Synchronises the stream and returns the status word a prefill attention
-    call left in ``ws`` (0 = RTP_OK, 4 = RTP_ERR_TIMEOUT)."""
-    return lib().rtp_workspace_status(ws.data_ptr(), _stream(stream))
+    """Synchronises the stream and returns the status word the last call that
+    used ``ws`` left there (0 = RTP_OK, 4 = RTP_ERR_TIMEOUT)."""
+    out = ctypes.c_int(0)
+    _check(lib().rtp_get_device_status(ws.data_ptr(), _stream(stream), ctypes.byref(out)),
+           "rtp_get_device_status")
+    return out.value
 
 
 def kv_of(h: int, Hq: int, Hkv: int) -> int:
@@ -142,12 +153,24 @@ def index_project(x: torch.Tensor, P: torch.Tensor, heads: Sequence[int], proj_o
     return out
 
 
+def index_append(k: torch.Tensor, P: torch.Tensor, kindex: torch.Tensor, pos: int, stream=None):
+    """Projects the keys k [B, n_new, Hkv, D] (every KV head, P [Hkv, D, r])
+    into rows pos .. pos + n_new - 1 of the key index kindex [B, Hkv, cap, r]."""
+    B, n_new, Hkv, _ = k.shape
+    assert kindex.is_contiguous() and kindex.shape[:2] == (B, Hkv)
+    _check(lib().rtp_index_append(k.data_ptr(), _strides4(k), B, n_new, Hkv, P.data_ptr(), P.shape[2],
+                                  kindex.data_ptr(), kindex.shape[2], pos, _stream(stream)), "rtp_index_append")
+    return kindex
+
+
 def select_prefill(qt: torch.Tensor, kt: torch.Tensor, kv_of_ret: Sequence[int], topk: int,
                    blocks: Optional[torch.Tensor] = None, counts: Optional[torch.Tensor] = None,
                    ws: Optional[torch.Tensor] = None, stream=None):
-    """qt [B,Hr,N,r], kt [B,Hkv,N,r] bf16 -> (blocks [B,Hr,N/64,k], counts [B,Hr,N/64])."""
+    """qt [B,Hr,N,r], kt [B,Hkv,cap,r] bf16 (rows 0..N-1 used, cap >= N)
+    -> (blocks [B,Hr,N/64,k], counts [B,Hr,N/64])."""
     B, Hr, N, r = qt.shape
     Hkv = kt.shape[1]
+    assert kt.is_contiguous()
     nb = N // BLOCK
     if blocks is None:
         blocks = torch.empty(B, Hr, nb, topk, dtype=torch.int32, device=qt.device)
@@ -155,24 +178,62 @@ def select_prefill(qt: torch.Tensor, kt: torch.Tensor, kv_of_ret: Sequence[int],
         counts = torch.empty(B, Hr, nb, dtype=torch.int32, device=qt.device)
     need = lib().rtp_workspace_size_select_prefill(B, N, Hr, topk)
     buf, nbytes = _ws(need, qt.device, ws)
-    _check(lib().rtp_select_prefill(qt.data_ptr(), kt.data_ptr(), B, N, Hr, Hkv, r, _i32(kv_of_ret),
+    _check(lib().rtp_select_prefill(qt.data_ptr(), kt.data_ptr(), kt.shape[2], B, N, Hr, Hkv, r, _i32(kv_of_ret),
                                     topk, blocks.data_ptr(), counts.data_ptr(), _wsptr(buf), nbytes,
                                     _stream(stream)), "rtp_select_prefill")
     return blocks, counts
 
 
 def select_decode(qt: torch.Tensor, kindex: torch.Tensor, kv_of_ret: Sequence[int], topk: int,
-                  idx: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
-    """qt [B,Hr,r] fp32, kindex [B,Hkv,L,r] bf16 -> idx [B,Hr,k] int32 ascending."""
+                  idx: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None,
+                  L: Optional[int] = None):
+    """qt [B,Hr,r] fp32, kindex [B,Hkv,cap,r] bf16 (rows 0..L-1 used; L
+    defaults to cap) -> idx [B,Hr,k] int32 ascending."""
     B, Hr, r = qt.shape
-    Hkv, L = kindex.shape[1], kindex.shape[2]
+    Hkv = kindex.shape[1]
+    L = kindex.shape[2] if L is None else L
+    assert kindex.is_contiguous()
     if idx is None:
         idx = torch.empty(B, Hr, topk, dtype=torch.int32, device=qt.device)
     need = lib().rtp_workspace_size_select_decode(B, L, Hr, topk)
     buf, nbytes = _ws(need, qt.device, ws)
-    _check(lib().rtp_select_decode(qt.data_ptr(), kindex.data_ptr(), B, L, Hr, Hkv, r,
+    _check(lib().rtp_select_decode(qt.data_ptr(), kindex.data_ptr(), kindex.shape[2], B, L, Hr, Hkv, r,
                                    _i32(kv_of_ret), topk, idx.data_ptr(), _wsptr(buf), nbytes,
                                    _stream(stream)), "rtp_select_decode")
+    return idx
+
+
+def index_quantize(kindex: torch.Tensor, g0: int, g1: int, kindex8: Optional[torch.Tensor] = None,
+                   kscale: Optional[torch.Tensor] = None, stream=None):
+    """8-bit codes and per-64-token scales of groups g0..g1-1 of the bf16 key
+    index kindex [B,Hkv,cap,r] -> (kindex8 int8 [B,Hkv,cap,r], kscale fp32
+    [B,Hkv,ceil(cap/64)])."""
+    B, Hkv, cap, r = kindex.shape
+    assert kindex.is_contiguous()
+    if kindex8 is None:
+        kindex8 = torch.zeros(B, Hkv, cap, r, dtype=torch.int8, device=kindex.device)
+    if kscale is None:
+        kscale = torch.zeros(B, Hkv, (cap + 63) // 64, dtype=torch.float32, device=kindex.device)
+    _check(lib().rtp_index_quantize(kindex.data_ptr(), cap, B, Hkv, g0, g1, kindex8.data_ptr(), kscale.data_ptr(),
+                                    _stream(stream)), "rtp_index_quantize")
+    return kindex8, kscale
+
+
+def select_decode_q8(qt: torch.Tensor, kindex8: torch.Tensor, kscale: torch.Tensor, kindex: torch.Tensor,
+                     kv_of_ret: Sequence[int], topk: int, idx: Optional[torch.Tensor] = None,
+                     ws: Optional[torch.Tensor] = None, stream=None, L: Optional[int] = None):
+    """Token top-k over the 8-bit key index (full 64-token groups) and the bf16
+    rows of the partial last group -> idx [B,Hr,k] int32 ascending."""
+    B, Hr, r = qt.shape
+    Hkv = kindex.shape[1]
+    L = kindex.shape[2] if L is None else L
+    if idx is None:
+        idx = torch.empty(B, Hr, topk, dtype=torch.int32, device=qt.device)
+    need = lib().rtp_workspace_size_select_decode(B, L, Hr, topk)
+    buf, nbytes = _ws(need, qt.device, ws)
+    _check(lib().rtp_select_decode_q8(qt.data_ptr(), kindex8.data_ptr(), kscale.data_ptr(), kindex.data_ptr(),
+                                      kindex.shape[2], B, L, Hr, Hkv, r, _i32(kv_of_ret), topk, idx.data_ptr(),
+                                      _wsptr(buf), nbytes, _stream(stream)), "rtp_select_decode_q8")
     return idx
 
 
@@ -192,6 +253,22 @@ def sparse_attn_prefill(q, k, v, o, heads: Sequence[int], blocks, counts, window
                                          counts.data_ptr(), topk, window_blocks, sink_blocks, scale,
                                          _wsptr(buf), nbytes, _stream(stream)),
            "rtp_sparse_attn_prefill")
+    return o
+
+
+def triangle_prefill(q, k, v, o, heads: Sequence[int], sink_blocks: int, window_blocks: int, last_tokens: int,
+                     scale: Optional[float] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """Triangle-shaped-mask prefill attention (streaming region: sink and band
+    blocks; last Q-K region: the last ``last_tokens`` rows see every key);
+    writes o[:, :, heads, :]. q/o [B,N,Hq,D], k/v [B,N,Hkv,D]."""
+    B, N, Hq, D = q.shape
+    Hkv = k.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    buf, nbytes = _ws(lib().rtp_workspace_size_triangle_prefill(), q.device, ws)
+    _check(lib().rtp_triangle_prefill(q.data_ptr(), _strides4(q), k.data_ptr(), _strides4(k), v.data_ptr(),
+                                      _strides4(v), o.data_ptr(), _strides4(o), B, N, Hq, Hkv, _i32(heads),
+                                      len(heads), sink_blocks, window_blocks, last_tokens, scale, _wsptr(buf),
+                                      nbytes, _stream(stream)), "rtp_triangle_prefill")
     return o
 
 
@@ -234,18 +311,27 @@ def decode_attn_hybrid(q, kc, vc, o, ret_heads: Sequence[int], idx, ret_window: 
 
 def decode_step(q, P, kindex, kc, vc, o, ret_heads: Sequence[int], idx, ret_window: int,
                 swa_heads: Sequence[int], swa_window: int, topk: int, sink: int = 1,
-                scale: Optional[float] = None, ws: Optional[torch.Tensor] = None, stream=None):
+                scale: Optional[float] = None, ws: Optional[torch.Tensor] = None, stream=None,
+                L: Optional[int] = None, kindex8: Optional[torch.Tensor] = None,
+                kscale: Optional[torch.Tensor] = None):
     """One decode step in one call: q~ projection, top-k selection into idx and
     the attention of retrieval and streaming heads. q/o [B,Hq,D], P [Hkv,D,r],
-    kindex [B,Hkv,L,r], kc/vc [B,L,Hkv,D], idx [B,Hr,topk] int32 (written)."""
+    kindex [B,Hkv,cap,r], kc/vc [B,cap,Hkv,D] (rows 0..L-1 are the cache; L
+    defaults to kc's length), idx [B,Hr,topk] int32 (written)."""
     B, Hq, D = q.shape
-    L, Hkv = kc.shape[1], kc.shape[2]
+    Hkv = kc.shape[2]
+    L = kc.shape[1] if L is None else L
+    if ret_heads:
+        assert kindex.is_contiguous() and kindex.shape[2] >= L
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     wmax = max(ret_window if ret_heads else 0, swa_window if swa_heads else 0)
     need = lib().rtp_workspace_size_decode_step(B, L, Hq, len(ret_heads), topk, wmax)
     buf, nbytes = _ws(need, q.device, ws)
     _check(lib().rtp_decode_step(q.data_ptr(), P.data_ptr() if ret_heads else None,
-                                 kindex.data_ptr() if ret_heads else None, kc.data_ptr(), _strides4(kc),
+                                 kindex.data_ptr() if ret_heads else None, kindex.shape[2] if ret_heads else 0,
+                                 kindex8.data_ptr() if kindex8 is not None else None,
+                                 kscale.data_ptr() if kscale is not None else None,
+                                 kc.data_ptr(), _strides4(kc),
                                  vc.data_ptr(), _strides4(vc), o.data_ptr(), B, L, Hq, Hkv, _i32(ret_heads),
                                  len(ret_heads), topk, ret_window, sink, _i32(swa_heads), len(swa_heads),
                                  swa_window, scale, idx.data_ptr() if ret_heads else None, _wsptr(buf), nbytes,
@@ -299,11 +385,25 @@ class PrefillLayer:
             self.blocks = torch.empty(B, len(self.ret), nb, topk, dtype=torch.int32, device=device)
             self.counts = torch.empty(B, len(self.ret), nb, dtype=torch.int32, device=device)
 
-    def __call__(self, q, k, v, P, o, stream=None):
+    def __call__(self, q, k, v, P, o, stream=None, index_out: Optional[torch.Tensor] = None):
+        """q/o [B,N,Hq,D], k/v [B,N,Hkv,D], P [Hkv,D,r].
+
+        ``index_out`` (optional, bf16 [B, Hkv, cap, r] with cap >= N) is the
+        decode key index of the cache this prefill fills: the layer then
+        projects the keys of every KV head into its rows 0..N-1
+        (``index_append``) and the block selection reads them from there, so
+        decode steps continue on the same index (appending one row per new
+        token) without a second projection."""
+        if index_out is not None:
+            index_append(k, P, index_out, 0, stream=stream)
         if self.ret:
-            index_project(k, P, self.kv_used, self.kv_used, out=self.kt, stream=stream)
+            if index_out is None:
+                index_project(k, P, self.kv_used, self.kv_used, out=self.kt, stream=stream)
+                kt, kv = self.kt, self.kv_slot
+            else:
+                kt, kv = index_out, self.kv_ret
             index_project(q, P, self.ret, self.kv_ret, out=self.qt, stream=stream)
-            select_prefill(self.qt, self.kt, self.kv_slot, self.topk, self.blocks, self.counts,
+            select_prefill(self.qt, kt, kv, self.topk, self.blocks, self.counts,
                            ws=self.ws_sel, stream=stream)
             sparse_attn_prefill(q, k, v, o, self.ret, self.blocks, self.counts, self.window_blocks,
                                 self.sink_blocks, self.scale, ws=self.ws_sparse, stream=stream)
@@ -317,6 +417,45 @@ class PrefillLayer:
                    workspace_status(self.ws_sel, stream))
 
 
+class OrthrosStep:
+    """The two working modes of one Orthros attention on the existing calls
+    (Orthros article, section on one attention with two working modes): every
+    token runs sliding-window attention, and only the position that predicts
+    the next token also runs a full cross-attention over the whole cache.
+
+    ``prefill(q, k, v, o, o_ca)``: SWA over every prompt row (all heads, one
+    rtp_swa call) and the full cross-attention of the last prompt row
+    (``o_ca`` [B, Hq, D]: the decode form of rtp_swa at position N-1 with a
+    window as long as the prompt). ``decode(q, kc, vc, o, o_ca, L)``: for the
+    new token at position L-1, its SWA row into ``o`` [B, Hq, D] and its full
+    cross-attention over the L cached tokens into ``o_ca``. The trained
+    Scale-Offset that tells the two queries apart is out of scope: both use
+    the same query."""
+
+    def __init__(self, B, L, Hq, Hkv, window, device, scale=None):
+        self.B, self.L, self.Hq, self.Hkv, self.window = B, L, Hq, Hkv, window
+        self.heads = list(range(Hq))
+        self.scale = 1.0 / math.sqrt(D_HEAD) if scale is None else scale
+        self.ws_swa = torch.zeros(lib().rtp_workspace_size_swa(B, 1, L, Hq, window), dtype=torch.uint8, device=device)
+        self.ws_ca = torch.zeros(lib().rtp_workspace_size_swa(B, 1, L, Hq, L), dtype=torch.uint8, device=device)
+        self.ws_pre = torch.zeros(256, dtype=torch.uint8, device=device)
+
+    def prefill(self, q, k, v, o, o_ca, stream=None):
+        N = q.shape[1]
+        swa(q, k, v, o, self.heads, self.window, 0, self.scale, ws=self.ws_pre, stream=stream)
+        swa(q[:, N - 1:N], k, v, o_ca.unsqueeze(1), self.heads, N, N - 1, self.scale, ws=self.ws_ca, stream=stream)
+        return o, o_ca
+
+    def decode(self, q, kc, vc, o, o_ca, L: Optional[int] = None, stream=None):
+        L = kc.shape[1] if L is None else L
+        assert L <= self.L
+        kv, vv = kc[:, :L], vc[:, :L]
+        swa(q.unsqueeze(1), kv, vv, o.unsqueeze(1), self.heads, self.window, L - 1, self.scale, ws=self.ws_swa,
+            stream=stream)
+        swa(q.unsqueeze(1), kv, vv, o_ca.unsqueeze(1), self.heads, L, L - 1, self.scale, ws=self.ws_ca, stream=stream)
+        return o, o_ca
+
+
 class DecodeStep:
     """One decode step over a cache with a precomputed key index: query
     projection, token selection, sparse attention on retrieval heads and SWA
@@ -324,6 +463,8 @@ class DecodeStep:
 
     def __init__(self, B, L, Hq, Hkv, ret_heads, window, ret_window, topk, device, sink=1,
                  scale=None):
+        """``L`` is the longest cache the step will see (its workspace is sized
+        for it); each call may pass a shorter current length."""
         self.B, self.L, self.Hq, self.Hkv = B, L, Hq, Hkv
         self.ret = list(ret_heads)
         self.swa_heads = [h for h in range(Hq) if h not in set(self.ret)]
@@ -335,13 +476,18 @@ class DecodeStep:
         self.ws = torch.empty(lib().rtp_workspace_size_decode_step(B, L, Hq, len(self.ret), topk, wmax),
                               dtype=torch.uint8, device=device)
 
-    def __call__(self, q, kc, vc, kindex, P, o, stream=None):
-        """q/o [B,Hq,D]; kc/vc [B,L,Hkv,D]; kindex [B,Hkv,L,r]; one rtp_decode_step call."""
+    def __call__(self, q, kc, vc, kindex, P, o, stream=None, L: Optional[int] = None, kindex8=None, kscale=None):
+        """q/o [B,Hq,D]; kc/vc [B,cap,Hkv,D]; kindex [B,Hkv,cap,r]; the cache
+        holds L <= self.L tokens (default: kc's length). With ``kindex8`` /
+        ``kscale`` (``index_quantize``) the selection scans the 8-bit index.
+        One rtp_decode_step call."""
+        L = kc.shape[1] if L is None else L
+        assert L <= self.L, "the workspace is sized for at most L tokens"
         decode_step(q, P, kindex, kc, vc, o, self.ret, self.idx, self.ret_window, self.swa_heads, self.window,
-                    self.topk, self.sink, self.scale, self.ws, stream=stream)
+                    self.topk, self.sink, self.scale, self.ws, stream=stream, L=L, kindex8=kindex8, kscale=kscale)
         return o
 
-    def graph(self, q, kc, vc, kindex, P, o) -> "torch.cuda.CUDAGraph":
+    def graph(self, q, kc, vc, kindex, P, o, kindex8=None, kscale=None) -> "torch.cuda.CUDAGraph":
         """Captures one step on these buffers into a CUDA graph.
 
         ``graph.replay()`` then runs the whole step (projection, selection,
@@ -351,10 +497,12 @@ class DecodeStep:
         eagerly before capturing, so that every kernel attribute is set."""
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            self(q, kc, vc, kindex, P, o)
+            self(q, kc, vc, kindex, P, o, kindex8=kindex8, kscale=kscale)
         return g
 
 
-__all__ = ["lib", "RtpError", "index_project", "select_prefill", "select_decode",
-           "sparse_attn_prefill", "sparse_attn_decode", "swa", "decode_attn_hybrid", "PrefillLayer", "DecodeStep",
+__all__ = ["lib", "RtpError", "index_project", "index_append", "index_quantize", "select_prefill", "select_decode",
+           "select_decode_q8",
+           "sparse_attn_prefill", "triangle_prefill", "sparse_attn_decode", "swa", "decode_attn_hybrid",
+           "PrefillLayer", "DecodeStep", "OrthrosStep",
            "kv_of", "LIB_PATH"]

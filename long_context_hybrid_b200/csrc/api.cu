@@ -4,6 +4,7 @@
 #include <stdint.h>
 
 #include "../../include/rtp.h"
+#include "../../include/rtp_testing.h"
 #include "attn_prefill_common.cuh"
 #include "rtp_common.cuh"
 #include "rtp_internal.h"
@@ -40,7 +41,7 @@ rtp_status check_heads(const int32_t* heads, int n, int H) {
 
 // Tensor maps for q/k/v and the tcgen05 launch; the status word (first 4 bytes
 // of ws) is cleared on the stream first and set by a CTA whose wait ran out.
-rtp_status launch_tc(PrefillAttnParams& p, int B, void* ws, cudaStream_t stream) {
+rtp_status launch_tc(PrefillAttnParams& p, int B, void* ws, cudaStream_t stream, bool clear_status = true) {
   CUtensorMap tq, tk, tv;
   if (!make_tmap_bnhd(&tq, p.q.p, B, p.Nq, p.Hq, p.q.sb, p.q.sn, p.q.sh, 128) ||
       !make_tmap_bnhd(&tk, p.k.p, B, p.Nk, p.Hkv, p.k.sb, p.k.sn, p.k.sh, 64) ||
@@ -48,7 +49,7 @@ rtp_status launch_tc(PrefillAttnParams& p, int B, void* ws, cudaStream_t stream)
     return RTP_ERR_CUDA;
   if (prefill_attn_tc_smem_bytes(p) > 227 * 1024) return RTP_ERR_UNSUPPORTED;
   int* status = static_cast<int*>(ws);
-  if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return RTP_ERR_CUDA;
+  if (clear_status && cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return RTP_ERR_CUDA;
   const int n_tiles = (p.Nq + 127) / 128;
   return from_cuda(launch_prefill_attn_tc(p, tq, tk, tv, n_tiles, B, status, stream));
 }
@@ -57,12 +58,13 @@ rtp_status launch_tc(PrefillAttnParams& p, int B, void* ws, cudaStream_t stream)
 
 extern "C" {
 
-rtp_status rtp_workspace_status(const void* ws, rtp_stream_t stream) {
-  if (!ws) return RTP_ERR_INVALID_ARG;
+rtp_status rtp_get_device_status(const void* ws, rtp_stream_t stream, rtp_status* out) {
+  if (!ws || !out) return RTP_ERR_INVALID_ARG;
   int v = 0;
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RTP_ERR_CUDA;
   if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return RTP_ERR_CUDA;
-  return v == 0 ? RTP_OK : (rtp_status)v;
+  *out = v == 0 ? RTP_OK : (rtp_status)v;
+  return RTP_OK;
 }
 
 const char* rtp_status_string(rtp_status s) {
@@ -97,16 +99,29 @@ rtp_status rtp_index_project(const void* x, rtp_strides xs, int B, int N, int Hx
                                   out_dtype == RTP_F32, (cudaStream_t)stream));
 }
 
+rtp_status rtp_index_append(const void* k, rtp_strides ks, int B, int n_new, int Hkv, const void* P, int r,
+                            void* kindex, int64_t cap, int pos, rtp_stream_t stream) {
+  if (!k || !P || !kindex) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || n_new < 1 || Hkv < 1 || Hkv > kMaxHeads || pos < 0 || cap < 1) return RTP_ERR_INVALID_ARG;
+  if ((int64_t)pos + n_new > cap) return RTP_ERR_INVALID_ARG;
+  if (r != RTP_R) return RTP_ERR_UNSUPPORTED;
+  if (!aligned16(k) || !aligned16(P) || !aligned16(kindex) || !stride_ok(ks)) return RTP_ERR_INVALID_ARG;
+  rtp_status st = check_device();
+  if (st != RTP_OK) return st;
+  return from_cuda(launch_index_append(k, ks.b, ks.n, ks.h, B, n_new, Hkv, P, kindex, cap, pos, (cudaStream_t)stream));
+}
+
 size_t rtp_workspace_size_select_prefill(int B, int N, int Hr, int topk) {
   return select_prefill_ws_bytes(B, N, Hr, topk);
 }
 
-rtp_status rtp_select_prefill(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
+rtp_status rtp_select_prefill(const void* qt, const void* kt, int64_t kt_cap, int B, int N, int Hr, int Hkv,
                               int r, const int32_t* kv_of, int topk,
                               int32_t* blocks, int32_t* counts,
                               void* ws, size_t ws_bytes, rtp_stream_t stream) {
   if (!qt || !kt || !blocks || !counts || !kv_of) return RTP_ERR_INVALID_ARG;
   if (B < 1 || N < RTP_BLOCK || Hr < 1 || Hr > kMaxHeads || Hkv < 1 || topk < 1) return RTP_ERR_INVALID_ARG;
+  if (kt_cap < N) return RTP_ERR_INVALID_ARG;
   if (N % RTP_BLOCK != 0 || r != RTP_R) return RTP_ERR_UNSUPPORTED;
   if (select_prefill_tc_smem(N / RTP_BLOCK) > 227 * 1024) return RTP_ERR_UNSUPPORTED;
   if (!aligned16(qt) || !aligned16(kt) || !aligned16(blocks) || !aligned16(counts)) return RTP_ERR_INVALID_ARG;
@@ -116,7 +131,7 @@ rtp_status rtp_select_prefill(const void* qt, const void* kt, int B, int N, int 
   if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
   rtp_status st = check_device();
   if (st != RTP_OK) return st;
-  return from_cuda(launch_select_prefill(qt, kt, B, N, Hr, Hkv, kv_of, topk, blocks, counts, ws,
+  return from_cuda(launch_select_prefill(qt, kt, kt_cap, B, N, Hr, Hkv, kv_of, topk, blocks, counts, ws,
                                          (cudaStream_t)stream));
 }
 
@@ -124,12 +139,13 @@ size_t rtp_workspace_size_select_decode(int B, int L, int Hr, int topk) {
   return select_decode_ws_bytes(B, L, Hr, topk);
 }
 
-rtp_status rtp_select_decode(const float* qt, const void* kindex, int B, int L, int Hr, int Hkv,
+rtp_status rtp_select_decode(const float* qt, const void* kindex, int64_t kindex_cap, int B, int L, int Hr, int Hkv,
                              int r, const int32_t* kv_of, int topk, int32_t* idx,
                              void* ws, size_t ws_bytes, rtp_stream_t stream) {
   if (!qt || !kindex || !idx || !kv_of) return RTP_ERR_INVALID_ARG;
   if (B < 1 || L < 1 || Hr < 1 || Hr > kMaxHeads || Hkv < 1 || topk < 1) return RTP_ERR_INVALID_ARG;
-  if (r != RTP_R || topk > 4096) return RTP_ERR_UNSUPPORTED;
+  if (kindex_cap < L) return RTP_ERR_INVALID_ARG;
+  if (r != RTP_R || topk > kMaxDecodeTopk) return RTP_ERR_UNSUPPORTED;
   if (!aligned16(qt) || !aligned16(kindex) || !aligned16(idx)) return RTP_ERR_INVALID_ARG;
   for (int j = 0; j < Hr; ++j)
     if (kv_of[j] < 0 || kv_of[j] >= Hkv) return RTP_ERR_INVALID_ARG;
@@ -143,8 +159,44 @@ rtp_status rtp_select_decode(const float* qt, const void* kindex, int B, int L, 
   if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
   rtp_status st = check_device();
   if (st != RTP_OK) return st;
-  return from_cuda(launch_select_decode(qt, kindex, B, L, Hr, Hkv, kv_of, topk, idx, ws,
-                                        (cudaStream_t)stream));
+  return from_cuda(launch_select_decode(qt, IndexRef{kindex, nullptr, nullptr, kindex_cap}, B, L, Hr, Hkv, kv_of,
+                                        topk, idx, ws, (cudaStream_t)stream));
+}
+
+rtp_status rtp_index_quantize(const void* kindex, int64_t cap, int B, int Hkv, int g0, int g1, void* kindex8,
+                              float* kscale, rtp_stream_t stream) {
+  if (!kindex || !kindex8 || !kscale) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || Hkv < 1 || cap < 1 || g0 < 0 || g1 < g0 || (int64_t)g1 * QGROUP_TOKENS > cap) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(kindex) || !aligned16(kindex8) || (reinterpret_cast<uintptr_t>(kscale) & 3u)) return RTP_ERR_INVALID_ARG;
+  rtp_status st = check_device();
+  if (st != RTP_OK) return st;
+  return from_cuda(launch_index_quantize(kindex, cap, B, Hkv, g0, g1, kindex8, kscale, (cudaStream_t)stream));
+}
+
+rtp_status rtp_select_decode_q8(const float* qt, const void* kindex8, const float* kscale, const void* kindex,
+                                int64_t kindex_cap, int B, int L, int Hr, int Hkv, int r, const int32_t* kv_of,
+                                int topk, int32_t* idx, void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  if (!kindex8 || !kscale) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(kindex8) || (reinterpret_cast<uintptr_t>(kscale) & 3u)) return RTP_ERR_INVALID_ARG;
+  if (!qt || !kindex || !idx || !kv_of) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || Hr < 1 || Hr > kMaxHeads || Hkv < 1 || topk < 1) return RTP_ERR_INVALID_ARG;
+  if (kindex_cap < L) return RTP_ERR_INVALID_ARG;
+  if (r != RTP_R || topk > kMaxDecodeTopk) return RTP_ERR_UNSUPPORTED;
+  if (!aligned16(qt) || !aligned16(kindex) || !aligned16(idx)) return RTP_ERR_INVALID_ARG;
+  for (int j = 0; j < Hr; ++j)
+    if (kv_of[j] < 0 || kv_of[j] >= Hkv) return RTP_ERR_INVALID_ARG;
+  if (Hkv > 16) return RTP_ERR_UNSUPPORTED;
+  for (int g = 0; g < Hkv; ++g) {
+    int c = 0;
+    for (int j = 0; j < Hr; ++j) c += kv_of[j] == g;
+    if (c > 16) return RTP_ERR_UNSUPPORTED;
+  }
+  const size_t need = select_decode_ws_bytes(B, L, Hr, topk);
+  if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
+  rtp_status st = check_device();
+  if (st != RTP_OK) return st;
+  return from_cuda(launch_select_decode(qt, IndexRef{kindex, kindex8, kscale, kindex_cap}, B, L, Hr, Hkv, kv_of,
+                                        topk, idx, ws, (cudaStream_t)stream));
 }
 
 size_t rtp_workspace_size_sparse_attn_prefill(int B, int N, int Hr, int topk) {
@@ -185,6 +237,66 @@ rtp_status rtp_sparse_attn_prefill(const void* q, rtp_strides qs, const void* k,
   for (int j = 0; j < Hr; ++j) p.head[j] = heads[j];
   if (nb > 32 * 4096) return RTP_ERR_UNSUPPORTED;
   return launch_tc(p, B, ws, (cudaStream_t)stream);
+}
+
+size_t rtp_workspace_size_triangle_prefill(void) { return kStatusBytes; }
+
+rtp_status rtp_triangle_prefill(const void* q, rtp_strides qs, const void* k, rtp_strides ks,
+                                const void* v, rtp_strides vs, void* o, rtp_strides os,
+                                int B, int N, int Hq, int Hkv, const int32_t* heads, int n_heads,
+                                int sink_blocks, int window_blocks, int last_tokens, float scale,
+                                void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  if (!q || !k || !v || !o) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || N < RTP_BLOCK || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return RTP_ERR_INVALID_ARG;
+  if (window_blocks < 1 || sink_blocks < 0 || last_tokens < 0 || last_tokens > N || !(scale > 0.f))
+    return RTP_ERR_INVALID_ARG;
+  if (N % RTP_BLOCK != 0 || last_tokens % RTP_BLOCK != 0) return RTP_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
+  if (!stride_ok(qs) || !stride_ok(ks) || !stride_ok(vs) || !stride_ok(os)) return RTP_ERR_INVALID_ARG;
+  rtp_status st = check_heads(heads, n_heads, Hq);
+  if (st != RTP_OK) return st;
+  if (!ws || ws_bytes < kStatusBytes || !aligned256(ws)) return RTP_ERR_WORKSPACE;
+  if ((st = check_device()) != RTP_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess) return RTP_ERR_CUDA;
+  const int n_stream = N - last_tokens;     // query rows of the streaming region
+  const float sl2 = scale * 1.4426950408889634f;
+  if (n_stream > 0) {
+    // Streaming region: rows 0 .. n_stream-1 attend the sink and window blocks
+    // (no selected blocks). Causal, so only the first n_stream keys are read.
+    PrefillAttnParams p{};
+    p.q = {q, qs.b, qs.n, qs.h}; p.k = {k, ks.b, ks.n, ks.h}; p.v = {v, vs.b, vs.n, vs.h};
+    p.o = o; p.o_sb = os.b; p.o_sn = os.n; p.o_sh = os.h;
+    p.Nq = n_stream; p.Nk = n_stream; p.q_pos0 = 0; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv;
+    p.sparse = 1; p.blocks = nullptr; p.counts = nullptr; p.topk = 1;
+    p.window_tokens = window_blocks * RTP_BLOCK; p.window_blocks = window_blocks; p.sink_blocks = sink_blocks;
+    p.scale_log2 = sl2;
+    p.n_heads = n_heads;
+    const int nb = n_stream / RTP_BLOCK;
+    if (nb > 32 * 4096) return RTP_ERR_UNSUPPORTED;
+    p.bitmap_words = (nb + 31) / 32;
+    const long cap = 2L * ((long)sink_blocks + window_blocks);
+    p.list_cap = (int)(cap < nb ? cap : nb);
+    for (int j = 0; j < n_heads; ++j) p.head[j] = heads[j];
+    if ((st = launch_tc(p, B, ws, s, false)) != RTP_OK) return st;
+  }
+  if (last_tokens > 0) {
+    // Last Q-K region: rows n_stream .. N-1 attend every earlier key (a
+    // window as long as the sequence), by the banded kernel on those rows.
+    PrefillAttnParams p{};
+    const char* qb = static_cast<const char*>(q) + (int64_t)n_stream * qs.n * 2;
+    char* ob = static_cast<char*>(o) + (int64_t)n_stream * os.n * 2;
+    p.q = {qb, qs.b, qs.n, qs.h}; p.k = {k, ks.b, ks.n, ks.h}; p.v = {v, vs.b, vs.n, vs.h};
+    p.o = ob; p.o_sb = os.b; p.o_sn = os.n; p.o_sh = os.h;
+    p.Nq = last_tokens; p.Nk = N; p.q_pos0 = n_stream; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv;
+    p.sparse = 0; p.window_tokens = N;
+    p.scale_log2 = sl2;
+    p.n_heads = n_heads;
+    p.list_cap = 0;
+    for (int j = 0; j < n_heads; ++j) p.head[j] = heads[j];
+    if ((st = launch_tc(p, B, ws, s, false)) != RTP_OK) return st;
+  }
+  return RTP_OK;
 }
 
 size_t rtp_workspace_size_sparse_attn_decode(int B, int L, int Hq, int Hr, int topk, int window) {
@@ -254,7 +366,8 @@ size_t rtp_workspace_size_decode_step(int B, int L, int Hq, int Hr, int topk, in
   return n;
 }
 
-rtp_status rtp_decode_step(const void* q, const void* P, const void* kindex, const void* kc, rtp_strides ks,
+rtp_status rtp_decode_step(const void* q, const void* P, const void* kindex, int64_t kindex_cap,
+                           const void* kindex8, const float* kscale, const void* kc, rtp_strides ks,
                            const void* vc, rtp_strides vs, void* o, int B, int L, int Hq, int Hkv,
                            const int32_t* ret_heads, int Hr, int topk, int ret_window, int sink,
                            const int32_t* swa_heads, int n_swa, int swa_window, float scale, int32_t* idx,
@@ -265,7 +378,10 @@ rtp_status rtp_decode_step(const void* q, const void* P, const void* kindex, con
   if (Hq / Hkv > 16 || Hkv > 16) return RTP_ERR_UNSUPPORTED;
   if (Hr > 0) {
     if (!P || !kindex || !idx || !ret_heads || topk < 1 || ret_window < 1) return RTP_ERR_INVALID_ARG;
-    if (topk > 4096) return RTP_ERR_UNSUPPORTED;
+    if (kindex_cap < L) return RTP_ERR_INVALID_ARG;
+    if (!kindex8 != !kscale) return RTP_ERR_INVALID_ARG;
+    if (kindex8 && (!aligned16(kindex8) || (reinterpret_cast<uintptr_t>(kscale) & 3u))) return RTP_ERR_INVALID_ARG;
+    if (topk > kMaxDecodeTopk) return RTP_ERR_UNSUPPORTED;
     if (!aligned16(P) || !aligned16(kindex) || !aligned16(idx)) return RTP_ERR_INVALID_ARG;
   }
   if (n_swa > 0 && swa_window < 1) return RTP_ERR_INVALID_ARG;
@@ -299,7 +415,8 @@ rtp_status rtp_decode_step(const void* q, const void* P, const void* kindex, con
     cudaError_t e = launch_project(q, (int64_t)Hq * RTP_D, (int64_t)Hq * RTP_D, RTP_D, B, 1, P, ret_heads, kv_of, Hr,
                                    qt, 1, s);
     if (e != cudaSuccess) return from_cuda(e);
-    e = launch_select_decode(qt, kindex, B, L, Hr, Hkv, kv_of, topk, idx, ws_sel, s);
+    e = launch_select_decode(qt, IndexRef{kindex, kindex8, kscale, kindex_cap}, B, L, Hr, Hkv, kv_of, topk, idx,
+                             ws_sel, s);
     if (e != cudaSuccess) return from_cuda(e);
   }
   // The kernel before the attention is the selection's filter (or nothing of

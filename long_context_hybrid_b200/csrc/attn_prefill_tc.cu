@@ -95,7 +95,7 @@ template <int NT>
 __device__ void mark_blocks(const PrefillAttnParams& p, int b, int jh, int q, unsigned* bits) {
   const int nb = p.Nq / RTP_BLOCK;
   const size_t row = ((size_t)b * p.n_heads + jh) * nb + q;
-  const int cnt = min(p.counts[row], p.topk);
+  const int cnt = p.counts ? min(p.counts[row], p.topk) : 0;
   const int32_t* sel = p.blocks + row * p.topk;
   for (int e = threadIdx.x; e < cnt; e += NT) {
     const int x = sel[e];

@@ -27,6 +27,7 @@
 //     of the segment (running max in the log2 domain, sum, o[128]); a second
 //     kernel, one CTA per head, merges each head's partials and writes its
 //     output.
+#include <cuda.h>
 #include <mutex>
 
 #include "rtp_common.cuh"
@@ -55,7 +56,8 @@ struct DecodeParams {
   const __nv_bfloat16* v; int64_t v_sb, v_sn, v_sh;
   __nv_bfloat16* o; int64_t o_sb, o_sh;
   int B, G;
-  const int32_t* idx; int topk;
+  const int32_t* idx; int topk;     // idx rows hold topk entries
+  int n_sel;                         // entries read per row: min(topk, L) (valid entries come first)
   int sink;
   float scale_log2;
   int n_heads, n_ret;                // call heads: retrieval heads first (0..n_ret-1)
@@ -180,7 +182,7 @@ __device__ __forceinline__ int slot_fetch(const DecodeParams& p, const Cursor& c
   const int j = c.a;                          // retrieval heads are call heads 0..n_ret-1
   const int n_sink = min(p.sink, p.wlo[j]);
   const int e = c.local * kChunk + s;         // virtual list: sink tokens, then the selected entries
-  if (e < n_sink || e - n_sink >= p.topk) return -1;
+  if (e < n_sink || e - n_sink >= p.n_sel) return -1;
   return __ldg(p.idx + ((size_t)c.b * p.n_ret + j) * p.topk + (e - n_sink));
 }
 __device__ __forceinline__ int slot_pos(const DecodeParams& p, const Cursor& c, int s, int fetched) {
@@ -192,7 +194,7 @@ __device__ __forceinline__ int slot_pos(const DecodeParams& p, const Cursor& c, 
   const int n_sink = min(p.sink, wlo);
   const int e = c.local * kChunk + s;
   if (e < n_sink) return e;
-  if (e - n_sink >= p.topk) return -1;
+  if (e - n_sink >= p.n_sel) return -1;
   return (fetched >= p.sink && fetched < wlo) ? fetched : -1;
 }
 }  // namespace
@@ -508,6 +510,7 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
   p.B = B; p.G = Hq / Hkv;
   if (p.G > kMaxGroup || Hkv > kMaxGroup) return cudaErrorInvalidValue;
   p.idx = idx; p.topk = n_ret > 0 ? topk : 0; p.sink = sink;
+  p.n_sel = p.topk < L ? p.topk : L;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.whi = q_pos + 1 < L ? q_pos + 1 : L;
   p.n_heads = n_ret + n_swa;
@@ -543,7 +546,7 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
   }
   p.wlo_union = wlo_union;
   p.n_wc = (p.whi - wlo_union + kChunk - 1) / kChunk;
-  p.n_gc = n_ret > 0 ? n_gathered_chunks(p.topk, sink) : 0;
+  p.n_gc = n_ret > 0 ? n_gathered_chunks(p.n_sel, sink) : 0;
   p.max_slots = kWarps * (p.n_wc + p.n_gc);
   p.n_win_chunks = B * p.n_ag * p.n_wc;
   p.n_gat_chunks = B * n_ret * p.n_gc;
@@ -598,25 +601,54 @@ static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchBytes / s
 
 namespace {
 constexpr int kMaxDevices = 64;
+struct ScratchSlot {
+  void* ctx;     // the context the address belongs to
+  void* ptr;     // device address of g_decode_scratch in that context
+};
 std::mutex g_scratch_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
+ScratchSlot g_scratch[kMaxDevices] = {};
+
+// The current context, through the runtime's driver entry-point query (the
+// library has no link-time dependency on libcuda). NULL if unavailable.
+void* current_context() {
+  using Fn = CUresult (*)(CUcontext*);
+  static Fn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<Fn>(ptr);
+  });
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
 }  // namespace
 
-// Device address of g_decode_scratch on the current device, looked up once
-// per device (with that device current) and cached.
+// Device address of g_decode_scratch on the current device, looked up with
+// that device current the first time a call runs on it, and again whenever the
+// device's context has changed since (after a cudaDeviceReset the primary
+// context, and the array's address with it, is new).
 static cudaError_t decode_scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  // No context may be current yet on the first call: the lookup creates the
+  // device's primary context, and the slot records the context it found.
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
+  ScratchSlot& slot = g_scratch[dev];
+  if (!slot.ptr || !ctx || slot.ctx != ctx) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = ptr;
+    slot.ptr = ptr;
+    slot.ctx = current_context();
   }
-  *out = g_scratch_ptr[dev];
+  *out = slot.ptr;
   return cudaSuccess;
 }
 

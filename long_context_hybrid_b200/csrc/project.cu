@@ -41,11 +41,15 @@ struct ProjectParams {
   int64_t sb, sn, sh;
   int B, N;
   const __nv_bfloat16* P;   // [Hp, 128, 16]
-  void* out;                // [B, n_heads, N, 16]
+  void* out;                // [B, out_nh, out_cap, 16]: row r of listed head j -> [b, out_slot[j], out_pos0 + r]
   int out_f32;
   int n_heads;
+  int out_nh;               // heads of the output tensor
+  int64_t out_cap;          // rows per (sequence, head) of the output tensor
+  int out_pos0;             // first output row
   int head[kMaxHeads];
   int proj[kMaxHeads];
+  int out_slot[kMaxHeads];
 };
 
 constexpr int kProjWarps = 4;
@@ -97,7 +101,7 @@ project_kernel(const ProjectParams p) {
       mma_bf16_16816(acc[1], a, bfrag[kk][1]);
     }
     // D fragment: (row g, cols 2t, 2t+1) and (row g+8, same cols) per n-tile.
-    const size_t obase = ((size_t)b * p.n_heads + j) * (size_t)p.N;
+    const size_t obase = ((size_t)b * p.out_nh + p.out_slot[j]) * (size_t)p.out_cap + p.out_pos0;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       const int col = nt * 8 + 2 * t;
@@ -130,7 +134,7 @@ project_small_kernel(const ProjectParams p) {
   for (int e = threadIdx.x; e < p.N * RTP_D; e += blockDim.x)
     xs[e / RTP_D][e % RTP_D] = __bfloat162float(xb[(size_t)(e / RTP_D) * p.sn + e % RTP_D]);
   __syncthreads();
-  const size_t obase = ((size_t)b * p.n_heads + j) * (size_t)p.N;
+  const size_t obase = ((size_t)b * p.out_nh + p.out_slot[j]) * (size_t)p.out_cap + p.out_pos0;
   for (int e = threadIdx.x; e < p.N * RTP_R; e += blockDim.x) {
     const int row = e / RTP_R, c = e % RTP_R;
     float acc = 0.f;
@@ -141,15 +145,8 @@ project_small_kernel(const ProjectParams p) {
   }
 }
 
-cudaError_t launch_project(const void* x, int64_t sb, int64_t sn, int64_t sh, int B, int N,
-                           const void* P, const int32_t* heads, const int32_t* proj, int n_heads,
-                           void* out, int out_f32, cudaStream_t stream) {
-  ProjectParams p;
-  p.x = static_cast<const __nv_bfloat16*>(x);
-  p.sb = sb; p.sn = sn; p.sh = sh; p.B = B; p.N = N;
-  p.P = static_cast<const __nv_bfloat16*>(P);
-  p.out = out; p.out_f32 = out_f32; p.n_heads = n_heads;
-  for (int i = 0; i < n_heads; ++i) { p.head[i] = heads[i]; p.proj[i] = proj[i]; }
+static cudaError_t launch_project_params(ProjectParams& p, cudaStream_t stream) {
+  const int N = p.N, B = p.B, n_heads = p.n_heads;
   if (N <= kSmallRows) {
     dim3 grid(n_heads, B);
     project_small_kernel<<<grid, 256, 0, stream>>>(p);
@@ -163,6 +160,31 @@ cudaError_t launch_project(const void* x, int64_t sb, int64_t sn, int64_t sh, in
   dim3 grid(gx, B, n_heads);
   project_kernel<<<grid, kProjWarps * 32, 0, stream>>>(p);
   return cudaGetLastError();
+}
+
+cudaError_t launch_project(const void* x, int64_t sb, int64_t sn, int64_t sh, int B, int N,
+                           const void* P, const int32_t* heads, const int32_t* proj, int n_heads,
+                           void* out, int out_f32, cudaStream_t stream) {
+  ProjectParams p;
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.sb = sb; p.sn = sn; p.sh = sh; p.B = B; p.N = N;
+  p.P = static_cast<const __nv_bfloat16*>(P);
+  p.out = out; p.out_f32 = out_f32; p.n_heads = n_heads;
+  p.out_nh = n_heads; p.out_cap = N; p.out_pos0 = 0;
+  for (int i = 0; i < n_heads; ++i) { p.head[i] = heads[i]; p.proj[i] = proj[i]; p.out_slot[i] = i; }
+  return launch_project_params(p, stream);
+}
+
+cudaError_t launch_index_append(const void* k, int64_t sb, int64_t sn, int64_t sh, int B, int n_new, int Hkv,
+                                const void* P, void* kindex, int64_t cap, int pos, cudaStream_t stream) {
+  ProjectParams p;
+  p.x = static_cast<const __nv_bfloat16*>(k);
+  p.sb = sb; p.sn = sn; p.sh = sh; p.B = B; p.N = n_new;
+  p.P = static_cast<const __nv_bfloat16*>(P);
+  p.out = kindex; p.out_f32 = 0; p.n_heads = Hkv;
+  p.out_nh = Hkv; p.out_cap = cap; p.out_pos0 = pos;
+  for (int g = 0; g < Hkv; ++g) { p.head[g] = g; p.proj[g] = g; p.out_slot[g] = g; }
+  return launch_project_params(p, stream);
 }
 
 }  // namespace rtp

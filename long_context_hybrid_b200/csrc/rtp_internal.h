@@ -32,13 +32,36 @@ cudaError_t launch_project(const void* x, int64_t sb, int64_t sn, int64_t sh, in
                            const void* P, const int32_t* heads, const int32_t* proj, int n_heads,
                            void* out, int out_f32, cudaStream_t stream);
 
+// Projects keys k[b, t, g, :] (t < n_new, every g < Hkv, with P[g]) into
+// rows pos .. pos + n_new - 1 of the key index [B, Hkv, cap, 16] (bf16).
+cudaError_t launch_index_append(const void* k, int64_t sb, int64_t sn, int64_t sh, int B, int n_new, int Hkv,
+                                const void* P, void* kindex, int64_t cap, int pos, cudaStream_t stream);
+
+// The 8-bit key index: int8 codes [B, Hkv, cap, 16] and one fp32 scale per
+// group of QGROUP_TOKENS tokens, [B, Hkv, ceil(cap / QGROUP_TOKENS)].
+#define QGROUP_TOKENS 64
+cudaError_t launch_index_quantize(const void* kindex, int64_t cap, int B, int Hkv, int g0, int g1, void* kindex8,
+                                  float* kscale, cudaStream_t stream);
+
+// Where the decode scan reads the key index: bf16 rows [B, Hkv, cap, 16] and,
+// when k8 is set, int8 codes for the tokens of the full groups (the first
+// QGROUP_TOKENS * floor(L / QGROUP_TOKENS) of each row) with their scales.
+struct IndexRef {
+  const void* bf16;
+  const void* k8;
+  const float* scale;
+  int64_t cap;
+};
+
+// Largest token top-k of a decode selection (any k >= L selects every token).
+constexpr int kMaxDecodeTopk = 1 << 22;
 size_t select_decode_ws_bytes(int B, int L, int Hr, int topk);
-cudaError_t launch_select_decode(const float* qt, const void* kindex, int B, int L, int Hr,
+cudaError_t launch_select_decode(const float* qt, IndexRef index, int B, int L, int Hr,
                                  int Hkv, const int32_t* kv_of, int topk, int32_t* idx,
                                  void* ws, cudaStream_t stream);
 
 size_t select_prefill_ws_bytes(int B, int N, int Hr, int topk);
-cudaError_t launch_select_prefill(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
+cudaError_t launch_select_prefill(const void* qt, const void* kt, int64_t kt_cap, int B, int N, int Hr, int Hkv,
                                   const int32_t* kv_of, int topk, int32_t* blocks,
                                   int32_t* counts, void* ws, cudaStream_t stream);
 
@@ -79,25 +102,18 @@ cudaError_t launch_decode_attn_noalloc(const void* q, int64_t q_sb, int64_t q_sh
                                        const int32_t* heads, int n_heads, const int32_t* idx, int topk,
                                        int window, int sink, float scale, cudaStream_t stream);
 
-// Prefill attention over per-query-block key-block lists (SWA band or
-// selected/sink/window union).
+// A [B, N, H, D] tensor: base pointer and element strides (D contiguous).
 struct Tensor4 {
   const void* p;
   int64_t sb, sn, sh;
 };
-cudaError_t launch_prefill_attn(Tensor4 q, Tensor4 k, Tensor4 v, void* o, int64_t o_sb,
-                                int64_t o_sn, int64_t o_sh, int B, int Nq, int Nk, int q_pos0,
-                                int Hq, int Hkv, const int32_t* heads, int n_heads,
-                                int sparse, const int32_t* blocks, const int32_t* counts, int topk,
-                                int window_tokens, int window_blocks, int sink_blocks, float scale,
-                                cudaStream_t stream);
 
 bool make_tmap_bnhd(CUtensorMap* map, const void* ptr, int B, int N, int H, int64_t sb, int64_t sn,
                     int64_t sh, int box_rows);
 
-bool make_tmap_index(CUtensorMap* map, const void* ptr, int B, int H, int N, int box_rows);
+bool make_tmap_index(CUtensorMap* map, const void* ptr, int B, int H, int N, int64_t cap, int box_rows);
 size_t select_prefill_tc_smem(int nb);
-cudaError_t launch_select_prefill_tc(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
+cudaError_t launch_select_prefill_tc(const void* qt, const void* kt, int64_t kt_cap, int B, int N, int Hr, int Hkv,
                                      const int32_t* kv_of, int topk, int32_t* blocks, int32_t* counts,
                                      int* status, cudaStream_t stream);
 

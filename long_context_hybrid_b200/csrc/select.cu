@@ -39,7 +39,6 @@ constexpr int kMaxHeadsPerGroup = 16;                               // retrieval
 constexpr int kBins = 2048;                                        // top 11 bits
 constexpr int kFiltThreads = 512;
 constexpr int kFiltStep = kFiltThreads * 16;                       // scores per CTA step
-constexpr int kMaxTopk = 4096;
 constexpr int kLocCap = 4096;                                      // shared slots for a CTA's candidates
 constexpr int kSmemCand = 4096;                                    // shared slots for a row's candidates
 constexpr int kSmemWords = 4096;                                   // shared bitmap words (rows up to 128K)
@@ -139,10 +138,17 @@ struct GroupHeads {
 // the row's. MAXJ > 0: the group's q~ rows sit in
 // registers (at most MAXJ heads per group); MAXJ == 0: any number, read from
 // shared memory. Each thread keeps the loads of BATCH tokens in flight.
-template <int MAXJ, int BATCH>
+// Q8: tokens of full 64-token groups are scored from the 8-bit index (one
+// 16-byte row of codes per token, score = scale * sum q_c code_c), the rest
+// (the partial last group) from the bf16 rows.
+template <int MAXJ, int BATCH, bool Q8>
 __global__ void __launch_bounds__(kScanThreads)
-decode_scan_kernel(const float* __restrict__ qt, const uint4* __restrict__ kindex, int B, int L, int Hr, int Hkv,
-                   const GroupHeads gh, const DecodeWs w) {
+decode_scan_kernel(const float* __restrict__ qt, const IndexRef index, int B, int L,
+                   int Hr, int Hkv, const GroupHeads gh, const DecodeWs w) {
+  const uint4* __restrict__ kindex = static_cast<const uint4*>(index.bf16);
+  const int64_t kcap = index.cap;
+  const int ufull = Q8 ? (L / QGROUP_TOKENS) * QGROUP_TOKENS : 0;   // tokens read from the codes
+  const int64_t ngroups = (kcap + QGROUP_TOKENS - 1) / QGROUP_TOKENS;
   pdl_trigger();                                       // the filter may launch and wait for this grid
   extern __shared__ uint32_t shist[];                  // [heads of the group][kBins]
   __shared__ float qs[MAXJ > 0 ? 1 : kMaxHeadsPerGroup][RTP_R];
@@ -172,7 +178,9 @@ decode_scan_kernel(const float* __restrict__ qt, const uint4* __restrict__ kinde
     }
     for (int e = threadIdx.x; e < n * kBins; e += kScanThreads) shist[e] = 0u;
     __syncthreads();
-    const uint4* krow = kindex + ((size_t)b * Hkv + g) * (size_t)L * 2;
+    const uint4* krow = kindex + ((size_t)b * Hkv + g) * (size_t)kcap * 2;
+    const uint4* k8row = Q8 ? static_cast<const uint4*>(index.k8) + ((size_t)b * Hkv + g) * (size_t)kcap : nullptr;
+    const float* srow_scale = Q8 ? index.scale + ((size_t)b * Hkv + g) * (size_t)ngroups : nullptr;
 #pragma unroll 1
     for (int base = u0; base < u1; base += kScanThreads * BATCH) {
       uint4 lo[BATCH], hi[BATCH];
@@ -181,18 +189,38 @@ decode_scan_kernel(const float* __restrict__ qt, const uint4* __restrict__ kinde
         const int u = base + t * kScanThreads + threadIdx.x;
         if (u < u1) {
           // read once: evict-first, so that the scores stay in L2 for the filter
-          lo[t] = __ldcs(krow + (size_t)u * 2);
-          hi[t] = __ldcs(krow + (size_t)u * 2 + 1);
+          if (Q8 && u < ufull) {
+            lo[t] = __ldcs(k8row + u);
+          } else {
+            lo[t] = __ldcs(krow + (size_t)u * 2);
+            hi[t] = __ldcs(krow + (size_t)u * 2 + 1);
+          }
         }
       }
 #pragma unroll
       for (int t = 0; t < BATCH; ++t) {
         const int u = base + t * kScanThreads + threadIdx.x;
         if (u >= u1) break;
-        const float k[16] = {bf16_lo(lo[t].x), bf16_hi(lo[t].x), bf16_lo(lo[t].y), bf16_hi(lo[t].y),
-                             bf16_lo(lo[t].z), bf16_hi(lo[t].z), bf16_lo(lo[t].w), bf16_hi(lo[t].w),
-                             bf16_lo(hi[t].x), bf16_hi(hi[t].x), bf16_lo(hi[t].y), bf16_hi(hi[t].y),
-                             bf16_lo(hi[t].z), bf16_hi(hi[t].z), bf16_lo(hi[t].w), bf16_hi(hi[t].w)};
+        float k[16];
+        float ks = 1.f;
+        if (Q8 && u < ufull) {
+          const uint32_t v4[4] = {lo[t].x, lo[t].y, lo[t].z, lo[t].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            k[4 * i + 0] = (float)((int32_t)(v4[i] << 24) >> 24);
+            k[4 * i + 1] = (float)((int32_t)(v4[i] << 16) >> 24);
+            k[4 * i + 2] = (float)((int32_t)(v4[i] << 8) >> 24);
+            k[4 * i + 3] = (float)((int32_t)v4[i] >> 24);
+          }
+          ks = __ldg(srow_scale + (u / QGROUP_TOKENS));
+        } else {
+          const uint32_t v8[8] = {lo[t].x, lo[t].y, lo[t].z, lo[t].w, hi[t].x, hi[t].y, hi[t].z, hi[t].w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            k[2 * i] = bf16_lo(v8[i]);
+            k[2 * i + 1] = bf16_hi(v8[i]);
+          }
+        }
         if constexpr (MAXJ > 0) {
 #pragma unroll
           for (int jj = 0; jj < MAXJ; ++jj) {
@@ -200,6 +228,7 @@ decode_scan_kernel(const float* __restrict__ qt, const uint4* __restrict__ kinde
             float acc = 0.f;
 #pragma unroll
             for (int c = 0; c < RTP_R; ++c) acc = fmaf(q[jj][c], k[c], acc);
+            if (Q8) acc *= ks;
             srow[jj][u] = acc;
             atomicAdd(&shist[jj * kBins + (f2key(acc) >> 21)], 1u);
           }
@@ -208,6 +237,7 @@ decode_scan_kernel(const float* __restrict__ qt, const uint4* __restrict__ kinde
             float acc = 0.f;
 #pragma unroll
             for (int c = 0; c < RTP_R; ++c) acc = fmaf(qs[jj][c], k[c], acc);
+            if (Q8) acc *= ks;
             w.scores[((size_t)b * Hr + gh.j[g][jj]) * L + u] = acc;
             atomicAdd(&shist[jj * kBins + (f2key(acc) >> 21)], 1u);
           }
@@ -531,9 +561,9 @@ size_t select_decode_ws_bytes(int B, int L, int Hr, int topk) {
   return decode_ws_layout(nullptr, B, L, Hr).total;
 }
 
-cudaError_t launch_select_decode(const float* qt, const void* kindex, int B, int L, int Hr, int Hkv,
+cudaError_t launch_select_decode(const float* qt, IndexRef index, int B, int L, int Hr, int Hkv,
                                  const int32_t* kv_of, int topk, int32_t* idx, void* ws, cudaStream_t stream) {
-  if (topk > kMaxTopk) return cudaErrorInvalidValue;
+  if (topk > kMaxDecodeTopk) return cudaErrorInvalidValue;
   if (Hkv > kMaxGroups) return cudaErrorInvalidValue;
   GroupHeads gh;
   int max_nj = 0;
@@ -569,14 +599,20 @@ cudaError_t launch_select_decode(const float* qt, const void* kindex, int B, int
     int64_t grid = (int64_t)(per_sm > 0 ? per_sm : 1) * sms;
     const int64_t min_tokens = kScanThreads * kScanBatch;   // at least one batch of tokens per CTA
     if (grid * min_tokens > total) grid = (total + min_tokens - 1) / min_tokens;
-    kernel<<<(int)grid, kScanThreads, scan_smem, stream>>>(qt, static_cast<const uint4*>(kindex), B, L, Hr, Hkv, gh,
-                                                           w);
+    kernel<<<(int)grid, kScanThreads, scan_smem, stream>>>(qt, index, B, L, Hr, Hkv, gh, w);
     return cudaGetLastError();
   };
-  if (max_nj <= 1) e = scan(decode_scan_kernel<1, kScanBatch>);
-  else if (max_nj <= 2) e = scan(decode_scan_kernel<2, kScanBatch>);
-  else if (max_nj <= 4) e = scan(decode_scan_kernel<4, kScanBatch>);
-  else e = scan(decode_scan_kernel<0, kScanBatch>);
+  if (index.k8) {
+    if (max_nj <= 1) e = scan(decode_scan_kernel<1, kScanBatch, true>);
+    else if (max_nj <= 2) e = scan(decode_scan_kernel<2, kScanBatch, true>);
+    else if (max_nj <= 4) e = scan(decode_scan_kernel<4, kScanBatch, true>);
+    else e = scan(decode_scan_kernel<0, kScanBatch, true>);
+  } else {
+    if (max_nj <= 1) e = scan(decode_scan_kernel<1, kScanBatch, false>);
+    else if (max_nj <= 2) e = scan(decode_scan_kernel<2, kScanBatch, false>);
+    else if (max_nj <= 4) e = scan(decode_scan_kernel<4, kScanBatch, false>);
+    else e = scan(decode_scan_kernel<0, kScanBatch, false>);
+  }
   if (e != cudaSuccess) return e;
   // filter: one wave of CTAs over all rows; slices are whole CTA steps
   e = cudaFuncSetAttribute(decode_filter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(FiltSmem));

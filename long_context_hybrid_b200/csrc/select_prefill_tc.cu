@@ -355,7 +355,7 @@ size_t select_prefill_tc_smem(int nb) {
   return 1024 + kScoreOff + (size_t)nb * 8 + sizeof(SelBars);
 }
 
-cudaError_t launch_select_prefill_tc(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
+cudaError_t launch_select_prefill_tc(const void* qt, const void* kt, int64_t kt_cap, int B, int N, int Hr, int Hkv,
                                      const int32_t* kv_of, int topk, int32_t* blocks, int32_t* counts,
                                      int* status, cudaStream_t stream) {
   SelectTcParams p;
@@ -363,7 +363,7 @@ cudaError_t launch_select_prefill_tc(const void* qt, const void* kt, int B, int 
   p.blocks = blocks; p.counts = counts;
   for (int j = 0; j < Hr; ++j) p.kv[j] = kv_of[j];
   CUtensorMap tq, tk;
-  if (!make_tmap_index(&tq, qt, B, Hr, N, 128) || !make_tmap_index(&tk, kt, B, Hkv, N, kChunkKeys))
+  if (!make_tmap_index(&tq, qt, B, Hr, N, N, 128) || !make_tmap_index(&tk, kt, B, Hkv, N, kt_cap, kChunkKeys))
     return cudaErrorInvalidValue;
   const size_t smem = select_prefill_tc_smem(p.nb);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
@@ -378,9 +378,10 @@ cudaError_t launch_select_prefill_tc(const void* qt, const void* kt, int B, int 
 }
 
 size_t select_prefill_ws_bytes(int B, int N, int Hr, int topk) { (void)B; (void)N; (void)Hr; (void)topk; return kStatusBytes; }
-cudaError_t launch_select_prefill(const void* qt, const void* kt, int B, int N, int Hr, int Hkv,
+cudaError_t launch_select_prefill(const void* qt, const void* kt, int64_t kt_cap, int B, int N, int Hr, int Hkv,
                                   const int32_t* kv_of, int topk, int32_t* blocks, int32_t* counts, void* ws,
                                   cudaStream_t stream) {
-  return launch_select_prefill_tc(qt, kt, B, N, Hr, Hkv, kv_of, topk, blocks, counts, static_cast<int*>(ws), stream);
+  return launch_select_prefill_tc(qt, kt, kt_cap, B, N, Hr, Hkv, kv_of, topk, blocks, counts, static_cast<int*>(ws),
+                                  stream);
 }
 }  // namespace rtp

@@ -43,13 +43,14 @@ bool make_tmap_bnhd(CUtensorMap* map, const void* ptr, int B, int N, int H, int6
   return r == CUDA_SUCCESS;
 }
 
-// Tensor map over an index x~[b, h, n, 0..16) (bf16, contiguous): box of one
-// 32-byte row x `box_rows` rows, 32-byte swizzle.
-bool make_tmap_index(CUtensorMap* map, const void* ptr, int B, int H, int N, int box_rows) {
+// Tensor map over rows 0 .. N-1 of an index x~[b, h, n, 0..16) (bf16; `cap`
+// rows per (b, h), contiguous): box of one 32-byte row x `box_rows` rows,
+// 32-byte swizzle.
+bool make_tmap_index(CUtensorMap* map, const void* ptr, int B, int H, int N, int64_t cap, int box_rows) {
   auto fn = encoder();
   if (!fn) return false;
   cuuint64_t dims[4] = {16, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
-  cuuint64_t strides[3] = {32, (cuuint64_t)N * 32, (cuuint64_t)H * N * 32};
+  cuuint64_t strides[3] = {32, (cuuint64_t)cap * 32, (cuuint64_t)H * cap * 32};
   cuuint32_t box[4] = {16, (cuuint32_t)box_rows, 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,

@@ -8,6 +8,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "rtp.h")
+TEST_HEADER = os.path.join(ROOT, "include", "rtp_testing.h")
 
 
 @pytest.fixture(scope="module")
@@ -18,8 +19,8 @@ def L():
     return rtp.lib()
 
 
-def declared_symbols():
-    text = open(HEADER).read()
+def declared_symbols(header=HEADER):
+    text = open(header).read()
     return sorted(set(re.findall(r"RTP_API\s+[\w\s\*]+?\b(rtp_\w+)\s*\(", text)))
 
 
@@ -31,8 +32,13 @@ def test_header_declares_the_six_calls():
 
 
 def test_every_declared_symbol_is_exported(L):
-    for name in declared_symbols():
+    for name in declared_symbols() + declared_symbols(TEST_HEADER):
         assert hasattr(L, name), name
+
+
+def test_test_hooks_stay_out_of_the_public_header():
+    assert not any("debug" in n for n in declared_symbols())
+    assert declared_symbols(TEST_HEADER) == ["rtp_debug_prefill_timeout_probe"]
 
 
 def test_version_and_status_strings(L):
@@ -72,16 +78,36 @@ def test_rejects_bad_arguments_without_launching(L):
     assert L.rtp_index_project(fake + 2, st, 1, 64, 4, fake, 1, 16, _heads([0]), _heads([0]), 1, fake, 0, None) == INVALID
     assert L.rtp_index_project(fake, S(8192, 516, 128), 1, 64, 4, fake, 1, 16, _heads([0]), _heads([0]), 1, fake, 0, None) == INVALID
     # N not a multiple of 64 for prefill selection
-    assert L.rtp_select_prefill(fake, fake, 1, 100, 1, 1, 16, _heads([0]), 4, fake, fake, None, 0, None) == UNSUP
+    assert L.rtp_select_prefill(fake, fake, 100, 1, 100, 1, 1, 16, _heads([0]), 4, fake, fake, None, 0, None) == UNSUP
     # kv head out of range
-    assert L.rtp_select_prefill(fake, fake, 1, 128, 1, 1, 16, _heads([1]), 4, fake, fake, None, 0, None) == INVALID
+    assert L.rtp_select_prefill(fake, fake, 128, 1, 128, 1, 1, 16, _heads([1]), 4, fake, fake, None, 0, None) == INVALID
+    # index capacity below the rows used
+    assert L.rtp_select_prefill(fake, fake, 64, 1, 128, 1, 1, 16, _heads([0]), 4, fake, fake, fake, 256, None) == INVALID
+    assert L.rtp_select_decode(fake, fake, 999, 1, 1000, 1, 1, 16, _heads([0]), 8, fake, fake, 1 << 30, None) == INVALID
+    assert L.rtp_decode_step(fake, fake, fake, 639, None, None, fake, S(640 * 256, 256, 128), fake, S(640 * 256, 256, 128), fake,
+                             1, 640, 8, 2, _heads([0]), 1, 16, 64, 1, _heads([1]), 1, 64, ctypes.c_float(0.1),
+                             fake, fake, 1 << 24, None) == INVALID
+    # 8-bit index: groups past the capacity, reversed range, one of codes/scales missing
+    assert L.rtp_index_quantize(fake, 128, 1, 2, 0, 3, fake, fake, None) == INVALID
+    assert L.rtp_index_quantize(fake, 128, 1, 2, 2, 1, fake, fake, None) == INVALID
+    assert L.rtp_select_decode_q8(fake, None, fake, fake, 1000, 1, 1000, 1, 1, 16, _heads([0]), 8, fake, fake,
+                                  1 << 30, None) == INVALID
+    assert L.rtp_decode_step(fake, fake, fake, 640, fake, None, fake, S(640 * 256, 256, 128), fake,
+                             S(640 * 256, 256, 128), fake, 1, 640, 8, 2, _heads([0]), 1, 16, 64, 1, _heads([1]), 1,
+                             64, ctypes.c_float(0.1), fake, fake, 1 << 24, None) == INVALID
+    # index append: rows past the capacity, r != 16, negative position
+    ka = S(4 * 2 * 128, 2 * 128, 128)
+    assert L.rtp_index_append(fake, ka, 1, 4, 2, fake, 16, fake, 100, 97, None) == INVALID
+    assert L.rtp_index_append(fake, ka, 1, 4, 2, fake, 8, fake, 100, 0, None) == UNSUP
+    assert L.rtp_index_append(fake, ka, 1, 4, 2, fake, 16, fake, 100, -1, None) == INVALID
+    assert L.rtp_index_append(None, ka, 1, 4, 2, fake, 16, fake, 100, 0, None) == INVALID
     # decode selection without a workspace
-    assert L.rtp_select_decode(fake, fake, 1, 1000, 1, 1, 16, _heads([0]), 8, fake, None, 0, None) == WS
-    assert L.rtp_select_decode(fake, fake, 1, 1000, 1, 1, 16, _heads([0]), 8, fake, fake, 10, None) == WS
-    assert L.rtp_select_decode(fake, fake, 1, 1000, 1, 1, 16, _heads([0]), 5000, fake, fake, 1 << 30, None) == UNSUP
+    assert L.rtp_select_decode(fake, fake, 1000, 1, 1000, 1, 1, 16, _heads([0]), 8, fake, None, 0, None) == WS
+    assert L.rtp_select_decode(fake, fake, 1000, 1, 1000, 1, 1, 16, _heads([0]), 8, fake, fake, 10, None) == WS
+    assert L.rtp_select_decode(fake, fake, 1000, 1, 1000, 1, 1, 16, _heads([0]), (1 << 22) + 1, fake, fake, 1 << 30, None) == UNSUP
     # more than 16 KV groups, or more than 16 retrieval heads on one group
-    assert L.rtp_select_decode(fake, fake, 1, 1000, 1, 17, 16, _heads([0]), 8, fake, fake, 1 << 30, None) == UNSUP
-    assert L.rtp_select_decode(fake, fake, 1, 1000, 17, 2, 16, _heads([0] * 17), 8, fake, fake, 1 << 30,
+    assert L.rtp_select_decode(fake, fake, 1000, 1, 1000, 1, 17, 16, _heads([0]), 8, fake, fake, 1 << 30, None) == UNSUP
+    assert L.rtp_select_decode(fake, fake, 1000, 1, 1000, 17, 2, 16, _heads([0] * 17), 8, fake, fake, 1 << 30,
                                None) == UNSUP
     # sparse prefill: bad window / scale / GQA ratio
     qs = S(64 * 8 * 128, 8 * 128, 128)
@@ -105,13 +131,13 @@ def test_rejects_bad_arguments_without_launching(L):
                                     16, 64, 1, ctypes.c_float(0.1), fake, 1 << 20, None) == INVALID
     # fused decode step: retrieval heads need P, the index and idx; workspace checked; sink bound
     f = ctypes.c_float(0.1)
-    assert L.rtp_decode_step(fake, None, fake, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, 16, 64, 1,
+    assert L.rtp_decode_step(fake, None, fake, 640, None, None, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, 16, 64, 1,
                              _heads([1]), 1, 64, f, fake, fake, 1 << 24, None) == INVALID
-    assert L.rtp_decode_step(fake, fake, fake, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, 16, 64, 1,
+    assert L.rtp_decode_step(fake, fake, fake, 640, None, None, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, 16, 64, 1,
                              _heads([1]), 1, 64, f, fake, None, 0, None) == WS
-    assert L.rtp_decode_step(fake, fake, fake, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, 16, 64, 65,
+    assert L.rtp_decode_step(fake, fake, fake, 640, None, None, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, 16, 64, 65,
                              _heads([1]), 1, 64, f, fake, fake, 1 << 24, None) == INVALID
-    assert L.rtp_decode_step(fake, fake, fake, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, 5000, 64, 1,
+    assert L.rtp_decode_step(fake, fake, fake, 640, None, None, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, (1 << 22) + 1, 64, 1,
                              _heads([1]), 1, 64, f, fake, fake, 1 << 30, None) == UNSUP
     # its workspace holds the three calls' workspaces
     B, Lc, Hq, Hr, k, w = 4, 20000, 32, 5, 2048, 4096

@@ -71,8 +71,12 @@ def run_prefill_fullsize(cfg, n_random=3):
             ok, amb, msg = band_check(got, res["sel"][(h, i)], res["scores"][(h, i)], cfg.topk)
             assert ok, f"{cfg.name} selection h{h} i{i}: {msg}"
             if not np.array_equal(np.sort(got), res["sel"][(h, i)]):
+                # tolerated near-tie: the oracle recomputes the row over the GPU's set
                 n_tol += 1
-                continue
+                g = h // G
+                att = O.attended_blocks(got, i, cfg.ret_window // 64, cfg.sink_blocks)
+                ref = O.sparse_attn_prefill_block(qc[:, h, :], kc[:, g, :], vc[:, g, :], i, att,
+                                                  1 / math.sqrt(128))
         outs.append(_f64(o[0, i * 64:(i + 1) * 64, h].cpu()))
         refs.append(ref)
     assert n_tol <= max(2, len(res["out"]) // 20)
@@ -103,8 +107,11 @@ def run_decode_fullsize(cfg, seqs):
                 ok, amb, msg = band_check(idx[b, j], res["sel"][h], res["scores"][h], cfg.topk)
                 assert ok, f"{cfg.name} b{b} h{h}: {msg}"
                 if not np.array_equal(np.sort(idx[b, j]), res["sel"][h]):
+                    # tolerated near-tie: the oracle's attention over the GPU's set
                     n_tol += 1
-                    continue
+                    g = h // (cfg.Hq // cfg.Hkv)
+                    att = O.decode_attended(idx[b, j][idx[b, j] >= 0], L, cfg.ret_window, cfg.sink)
+                    ref = O.attend_decode(q[b, h].cpu(), kcb[:, g], vcb[:, g], att, 1 / math.sqrt(128))
             outs.append(_f64(o[b, h].cpu()))
             refs.append(ref)
     return assert_attn_close(np.stack(outs), np.stack(refs), cfg.name)

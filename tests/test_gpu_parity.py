@@ -14,7 +14,7 @@ import torch
 
 import oracle as O
 import synth
-from helpers import assert_attn_close, assert_index_close, band_check
+from helpers import assert_attn_close, assert_f32_index_close, assert_index_close, band_check
 
 pytestmark = pytest.mark.gpu
 
@@ -67,9 +67,7 @@ def test_index_project_bf16_and_f32(N):
     for j, (h, p) in enumerate(zip(heads, proj)):
         for b in range(2):
             assert_index_close(_f64(out[b, j]), x[b, :, h], P[p])
-            exact = O.project(x[b, :, h], P[p], round_to_bf16=False)
-            bound = np.abs(_f64(x[b, :, h])) @ np.abs(_f64(P[p])) * 128 * 2.0 ** -24 + 1e-30
-            assert np.all(np.abs(_f64(out32[b, j]) - exact) <= bound)
+            assert_f32_index_close(_f64(out32[b, j]), x[b, :, h], P[p])
 
 
 def test_index_project_strided_input():
@@ -320,8 +318,13 @@ def _prefill_e2e(cfg, data, qblocks, heads=None, check_kt=True):
                                       cfg.topk)
             assert ok, f"selection h{h} i{i}: {msg}"
             if not np.array_equal(np.sort(blocks[0, j, i, :n]), res["sel"][(h, i)]):
+                # a tolerated near-tie changed the set: the oracle recomputes the
+                # row's attention over the GPU's set
                 n_amb_rows += 1
-                continue   # a tolerated near-tie changed the set: outputs differ legitimately
+                g = O.kv_of(h, cfg.Hq, cfg.Hkv)
+                att = O.attended_blocks(blocks[0, j, i, :n], i, cfg.ret_window // 64, cfg.sink_blocks)
+                ref = O.sparse_attn_prefill_block(qc[:, h, :], kc[:, g, :], vc[:, g, :], i, att,
+                                                  1 / math.sqrt(128))
         outs.append(_f64(o[0, i * 64:(i + 1) * 64, h].cpu()))
         refs.append(ref)
     worst = assert_attn_close(np.stack(outs), np.stack(refs), cfg.name)
@@ -359,10 +362,17 @@ def test_e2e_decode_reduced():
                 j = cfg.ret_heads.index(h)
                 ok, amb, msg = band_check(idx[b, j], res["sel"][h], res["scores"][h], cfg.topk)
                 assert ok, f"b{b} h{h}: {msg}"
+                ref = res["out"][h]
                 if not np.array_equal(np.sort(idx[b, j]), res["sel"][h]):
-                    continue
+                    # tolerated near-tie: the oracle's attention over the GPU's set
+                    g = O.kv_of(h, cfg.Hq, cfg.Hkv)
+                    att = O.decode_attended(idx[b, j][idx[b, j] >= 0], L, cfg.ret_window, cfg.sink)
+                    ref = O.attend_decode(q[b, h].cpu(), kc[b, :, g].cpu(), vc[b, :, g].cpu(), att,
+                                          1 / math.sqrt(128))
+            else:
+                ref = res["out"][h]
             outs.append(_f64(o[b, h].cpu()))
-            refs.append(res["out"][h])
+            refs.append(ref)
     assert_attn_close(np.stack(outs), np.stack(refs), "decode")
     # the same step captured as a CUDA graph and replayed with a new query
     o_eager = o.clone()

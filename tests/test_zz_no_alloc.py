@@ -6,7 +6,8 @@ decode loop that cannot afford cudaMalloc/cudaFree per step): its split-K
 partials live in a fixed array inside the library. This test calls it through
 the C ABI twice in a row and checks each result against the workspace-taking
 rtp_sparse_attn_decode on the same inputs, within the attention tolerance the
-other parity tests use. It lives in its own file, collected last.
+other parity tests use, and one sequence of each call against the fp64
+oracle. It lives in its own file, collected last.
 """
 import ctypes
 import math
@@ -15,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from helpers import assert_attn_close
 
 pytestmark = pytest.mark.gpu
@@ -68,6 +70,13 @@ def test_noalloc_matches_workspace_entry_point(rtp):
             assert_attn_close(out[:, h].float().cpu().numpy(), ref[:, h].float().cpu().numpy(),
                               f"call {call} head {h}")
         assert torch.all(out[:, [h for h in range(Hq) if h not in heads]] == 0)
+        b = call                                    # one sequence per call against the oracle
+        for j, h in enumerate(heads):
+            g = h // (Hq // Hkv)
+            sel = idx[b, j].cpu().numpy()
+            att = O.decode_attended(sel[sel >= 0], L, window, sink)
+            ref = O.attend_decode(q[b, h].cpu(), kc[b, :, g].cpu(), vc[b, :, g].cpu(), att, scale)
+            assert_attn_close(out[b, h].float().cpu().numpy(), ref, f"call {call} oracle head {h}")
 
 
 def test_noalloc_rejects_partials_beyond_its_array(rtp):

@@ -83,22 +83,23 @@ def run_prefill_fullsize(cfg, n_random=3):
     return assert_attn_close(np.stack(outs), np.stack(refs), cfg.name)
 
 
-def run_decode_fullsize(cfg, seqs):
+def run_decode_fullsize(cfg, seqs, index_bits=16):
     d = synth.make_decode(cfg, device=DEV)
     q, kc, vc, P = d["q"], d["kc"], d["vc"], d["P"]
     B, L = cfg.B, cfg.L
     kindex = rtp.index_project(kc, P, list(range(cfg.Hkv)), list(range(cfg.Hkv)))
+    k8, ks = rtp.index_quantize(kindex, 0, L // 64) if index_bits == 8 else (None, None)
     step = rtp.DecodeStep(B, L, cfg.Hq, cfg.Hkv, cfg.ret_heads, cfg.window, cfg.ret_window, cfg.topk, DEV,
                           sink=cfg.sink)
     o = torch.zeros(B, cfg.Hq, 128, dtype=torch.bfloat16, device=DEV)
-    step(q, kc, vc, kindex, P, o)
+    step(q, kc, vc, kindex, P, o, kindex8=k8, kscale=ks)
     torch.cuda.synchronize()
     idx = step.idx.cpu().numpy()
     outs, refs, n_tol = [], [], 0
     for b in seqs:
         kcb, vcb = kc[b].cpu(), vc[b].cpu()
         res = O.decode_layer(q[b].cpu(), kcb, vcb, P.cpu(), cfg.ret_heads, cfg.window, cfg.ret_window,
-                             cfg.topk, 1 / math.sqrt(128), sink=cfg.sink)
+                             cfg.topk, 1 / math.sqrt(128), sink=cfg.sink, index_bits=index_bits)
         for g in res["kt"]:
             assert_index_close(_f64(kindex[b, g]), kcb[:, g, :], P[g].cpu())
         for h, ref in res["out"].items():
@@ -123,6 +124,10 @@ def test_prefill_32k_fullsize():
 
 def test_decode_128k_b8_fullsize():
     run_decode_fullsize(synth.DECODE_128K, seqs=range(synth.DECODE_128K.B))
+
+
+def test_decode_128k_b8_8bit_index_fullsize():
+    run_decode_fullsize(synth.DECODE_128K, seqs=[0, 3, 7], index_bits=8)
 
 
 def test_prefill_1m_fullsize():

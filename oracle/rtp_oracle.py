@@ -290,6 +290,80 @@ def decode_scores_q8(qt, codes, scales, kt_tail, group: int = QGROUP) -> np.ndar
 
 
 # ---------------------------------------------------------------------------
+# K-cache clustering: two-level decode selection
+# ---------------------------------------------------------------------------
+FIX_SCALE = 2.0 ** 20          # fixed-point step of the centroid sums
+
+
+def kmeans_assign(x32, mu32) -> np.ndarray:
+    """Nearest centroid of every row: argmin_i sum_c (x_c - mu_ic)^2, the sum
+    taken over c = 0, 1, ... with every subtraction, square and addition
+    rounded to fp32 (no fused multiply-add), ties to the smaller index.
+    ``x32`` [L, r] and ``mu32`` [C, r] are float32."""
+    L, r = x32.shape
+    out = np.empty(L, np.int64)
+    for u0 in range(0, L, 4096):                              # bounded temporaries
+        xs = x32[u0:u0 + 4096]
+        d = np.zeros((xs.shape[0], mu32.shape[0]), np.float32)
+        for c in range(r):
+            diff = xs[:, c:c + 1] - mu32[None, :, c]          # float32, one rounding
+            d = d + diff * diff                               # float32 product, then float32 sum
+        out[u0:u0 + 4096] = np.argmin(d, axis=1)              # first minimum: smaller index
+    return out
+
+
+def kmeans_update(x32, assign, mu32) -> np.ndarray:
+    """New centroids: the mean of each cluster's rows. The sums are exact
+    integer sums of trunc(x * 2^20) (so that their value does not depend on
+    the order of the additions), then mean = fp32(double(sum) / double(count)
+    * 2^-20); a cluster with no rows keeps its centroid."""
+    C, r = mu32.shape
+    fixed = np.trunc(x32.astype(np.float64) * FIX_SCALE).astype(np.int64)
+    sums = np.zeros((C, r), np.int64)
+    np.add.at(sums, assign, fixed)
+    cnt = np.bincount(assign, minlength=C).astype(np.int64)
+    new = mu32.copy()
+    nz = cnt > 0
+    new[nz] = ((sums[nz].astype(np.float64) / cnt[nz, None].astype(np.float64)) / FIX_SCALE).astype(np.float32)
+    return new
+
+
+def kmeans_index(kt, cluster_size: int = 64, iters: int = 2):
+    """K-means over one KV head's key index (RTPurboV2 article: the keys of the
+    retrieval heads are clustered in the low-rank space, so that decode can
+    skip whole groups of semantically unrelated tokens; the pages give no
+    algorithm, so this is plain Lloyd k-means). C = ceil(L / cluster_size)
+    centroids start at the rows 0, cluster_size, 2 cluster_size, ...; each of
+    ``iters`` iterations assigns every row to its nearest centroid and moves
+    the centroids to their clusters' means; a final assignment pairs every
+    row with its nearest final centroid. Returns (centroids [C, r] float32,
+    assignment [L] int64)."""
+    x = to_f64(kt).astype(np.float32)
+    L = x.shape[0]
+    C = (L + cluster_size - 1) // cluster_size
+    mu = x[np.arange(C) * cluster_size].copy()
+    for _ in range(iters):
+        mu = kmeans_update(x, kmeans_assign(x, mu), mu)
+    return mu, kmeans_assign(x, mu)
+
+
+def select_decode_clustered(qt, kt, centroids, assign, n_probe: int, topk: int):
+    """Two-level token selection: the n_probe clusters whose centroids score
+    highest against q~ (ties to the smaller cluster), then the top-k tokens by
+    q~ . k~ among those clusters' members (ties to the smaller token; all of
+    them when fewer). Returns a dict with the ascending selection ``sel`` and
+    the intermediate ``cluster_scores``, ``clusters`` (chosen, ascending),
+    ``cand`` (ascending candidate tokens) and ``cand_scores``."""
+    qt = to_f64(qt)
+    cs = to_f64(centroids) @ qt
+    chosen = topk_desc(cs, n_probe)
+    cand = np.flatnonzero(np.isin(np.asarray(assign), chosen))
+    sc = to_f64(kt)[cand] @ qt
+    sel = cand[topk_desc(sc, topk)]
+    return dict(sel=np.sort(sel), cluster_scores=cs, clusters=chosen, cand=cand, cand_scores=sc)
+
+
+# ---------------------------------------------------------------------------
 # Static patterns on the same attention (presets)
 # ---------------------------------------------------------------------------
 def triangle_keys(t: int, N: int, sink_blocks: int, window_blocks: int, last_tokens: int,
@@ -425,5 +499,6 @@ __all__ = [
     "attended_blocks", "attend", "sparse_attn_prefill_block", "swa_rows", "decode_scores",
     "select_decode", "decode_attended", "attend_decode", "kv_of", "prefill_layer",
     "decode_layer", "triangle_keys", "triangle_rows", "dense_decode", "QGROUP", "quantize_index",
-    "decode_scores_q8",
+    "decode_scores_q8", "FIX_SCALE", "kmeans_assign", "kmeans_update", "kmeans_index",
+    "select_decode_clustered",
 ]

@@ -605,3 +605,95 @@ def test_planted_q8_mistakes_are_caught():
 
     assert not _golden_q8_ok(truncating)
     assert not _golden_q8_ok(scale_by_128)
+
+
+# ---------------------------------------------------------------------------
+# K-cache clustering (two-level decode selection)
+# ---------------------------------------------------------------------------
+def _golden_kcluster_ok(kmeans, select):
+    g = json.load(open(os.path.join(GOLDEN, "kcluster_hand.json")))
+    kt = np.array(g["kt"], np.float64)
+    mu, a = kmeans(kt, g["cluster_size"], g["iters"])
+    if not (np.array_equal(mu, np.array(g["centroids"], np.float32)) and list(a) == g["assign"]):
+        return False
+    for c in g["selections"]:
+        r = select(np.array(g["q"], np.float64), kt, mu, a, c["n_probe"], c["topk"])
+        if list(r["clusters"]) != c["clusters"] or list(r["sel"]) != c["sel"]:
+            return False
+    return True
+
+
+def test_golden_kcluster():
+    assert _golden_kcluster_ok(O.kmeans_index, O.select_decode_clustered)
+
+
+def test_kcluster_reduces_to_flat_topk():
+    """Every token its own cluster, or every cluster probed: the two-level
+    selection is the flat top-k over the whole cache."""
+    rs = np.random.default_rng(50)
+    L = 700
+    kt = O.bf16_round(rs.standard_normal((L, 16)) * 2)
+    q = rs.standard_normal(16)
+    flat = O.select_decode(q, kt, 64)
+    mu, a = O.kmeans_index(kt, 1, 1)
+    assert list(a) == list(range(L))                          # distinct rows: each its own centroid
+    assert list(O.select_decode_clustered(q, kt, mu, a, 64, 64)["sel"]) == list(flat)
+    mu, a = O.kmeans_index(kt, 64, 2)
+    assert list(O.select_decode_clustered(q, kt, mu, a, len(mu), 64)["sel"]) == list(flat)
+
+
+def test_kmeans_objective_does_not_increase():
+    """Lloyd's iterations never raise the within-cluster sum of squares, and
+    every row ends at its nearest final centroid."""
+    rs = np.random.default_rng(51)
+    c = rs.standard_normal((12, 16)) * 4
+    kt = O.bf16_round(c[rs.integers(0, 12, 3000)] + rs.standard_normal((3000, 16)) * 0.5)
+    x = kt.astype(np.float32)
+    prev = None
+    for it in range(4):
+        mu, a = O.kmeans_index(kt, 256, it)
+        obj = float(((x.astype(np.float64) - mu[a].astype(np.float64)) ** 2).sum())
+        d = ((x[:, None, :].astype(np.float64) - mu[None].astype(np.float64)) ** 2).sum(-1)
+        assert np.all(d[np.arange(len(a)), a] <= d.min(1) * (1 + 1e-6) + 1e-9)
+        if prev is not None:
+            assert obj <= prev * (1 + 1e-6)
+        prev = obj
+
+
+def test_planted_kcluster_mistakes_are_caught():
+    def far_assign(x32, mu32):                       # argmax instead of argmin
+        d = ((x32[:, None, :] - mu32[None]) ** 2).sum(-1)
+        return np.argmax(d, axis=1)
+
+    def kmeans_far(kt, cs, iters):
+        x = O.to_f64(kt).astype(np.float32)
+        C = (len(x) + cs - 1) // cs
+        mu = x[np.arange(C) * cs].copy()
+        for _ in range(iters):
+            mu = O.kmeans_update(x, far_assign(x, mu), mu)
+        return mu, far_assign(x, mu)
+
+    def kmeans_ties_high(kt, cs, iters):             # ties to the larger centroid index
+        x = O.to_f64(kt).astype(np.float32)
+        C = (len(x) + cs - 1) // cs
+        mu = x[np.arange(C) * cs].copy()
+
+        def asg(mu_):
+            d = np.zeros((len(x), len(mu_)), np.float32)
+            for c in range(x.shape[1]):
+                diff = x[:, c:c + 1] - mu_[None, :, c]
+                d = d + diff * diff
+            return len(mu_) - 1 - np.argmin(d[:, ::-1], axis=1)
+        for _ in range(iters):
+            mu = O.kmeans_update(x, asg(mu), mu)
+        return mu, asg(mu)
+
+    def select_lowest_clusters(q, kt, mu, a, n_probe, topk):   # probes the lowest-scoring clusters
+        r = O.select_decode_clustered(-np.asarray(q), kt, mu, a, n_probe, topk)
+        cand = r["cand"]
+        sc = O.to_f64(kt)[cand] @ np.asarray(q, np.float64)
+        return dict(r, sel=np.sort(cand[O.topk_desc(sc, topk)]))
+
+    assert not _golden_kcluster_ok(kmeans_far, O.select_decode_clustered)
+    assert not _golden_kcluster_ok(kmeans_ties_high, O.select_decode_clustered)
+    assert not _golden_kcluster_ok(O.kmeans_index, select_lowest_clusters)

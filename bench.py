@@ -206,18 +206,36 @@ def decode_bytes(cfg, idx: torch.Tensor, L: int, B: int) -> dict:
 NOMINAL_BF16_TFLOPS = 2250.0
 NOMINAL_HBM_GBS = 7700.0
 
-# DRAM bytes per launch (read + write) from one-pass ncu counters of the
-# current kernels at full size (profiles/traffic_prefill_1m.md and
-# profiles/decode_128k_b8.md); None where no capture of the current kernel
-# exists. Reset an entry whenever its kernel changes.
-MEASURED_TRAFFIC = {
-    ("prefill_1m", "select_prefill"): 316478208 + 73203200,
-    ("prefill_1m", "sparse_attn_prefill"): 112003927552 + 1351792128,
-    ("prefill_1m", "swa_prefill"): 21796575744 + 7232377088,
-    # decode step: scan + filter + attention + merge (cold cache, as the bench
-    # flushes L2 before each step)
-    ("decode_128k_b8", "step"): 134311936 + 6669824 + 21367296 + 173760768 + 3689216 + 6118912,
-}
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per unit of
+# work, from one ncu capture of each kernel on a small case of the same
+# kernel (profiles/ names the command), scaled here by the units one launch of
+# the benchmark processes. Each entry records a digest of the sources the
+# kernel is built from: when they have changed since the capture, the entry
+# is stale and the line reports null.
+NCU_TRAFFIC = {}
+
+
+def _sources_digest(files):
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "long_context_hybrid_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(name, units):
+    """DRAM bytes of one launch of kernel ``name`` processing ``units`` units
+    of work, or None when no capture of the current sources exists."""
+    e = NCU_TRAFFIC.get(name)
+    if e is None:
+        return None
+    try:
+        if _sources_digest(e["sources"]) != e["digest"]:
+            return None
+    except OSError:
+        return None
+    return int(e["bytes_per_unit"] * units)
 
 
 def run_ours(args, rank, world):
@@ -384,12 +402,15 @@ def run_ours(args, rank, world):
     sw_pairs = n_swa * pcfg.B * swa_pairs(N, pcfg.window)
     sp_pairs = sparse_pairs(layer.blocks, layer.counts, layer.window_blocks, layer.sink_blocks)
     sel_pairs = len(layer.ret) * pcfg.B * causal_pairs(N)
+    # units: what the traffic of a launch scales with (attended pairs; rows)
     work = {
-        "swa_prefill": {"flops": 4 * D * sw_pairs, "bound": "tensor"},
-        "sparse_attn_prefill": {"flops": 4 * D * sp_pairs, "bound": "tensor"},
-        "select_prefill": {"flops": 2 * R * sel_pairs, "bound": "tensor"},
-        "project_k": {"bytes": pcfg.B * N * len(layer.kv_used) * (D + R) * 2, "bound": "hbm"},
-        "project_q": {"bytes": pcfg.B * N * len(layer.ret) * (D + R) * 2, "bound": "hbm"},
+        "swa_prefill": {"flops": 4 * D * sw_pairs, "bound": "tensor", "units": sw_pairs},
+        "sparse_attn_prefill": {"flops": 4 * D * sp_pairs, "bound": "tensor", "units": sp_pairs},
+        "select_prefill": {"flops": 2 * R * sel_pairs, "bound": "tensor", "units": sel_pairs},
+        "project_k": {"bytes": pcfg.B * N * len(layer.kv_used) * (D + R) * 2, "bound": "hbm",
+                      "units": pcfg.B * N * len(layer.kv_used)},
+        "project_q": {"bytes": pcfg.B * N * len(layer.ret) * (D + R) * 2, "bound": "hbm",
+                      "units": pcfg.B * N * len(layer.ret)},
     }
     tflops_peak = peaks["bf16_tflops_sustained"]
     kernels = {}
@@ -409,13 +430,13 @@ def run_ours(args, rank, world):
     if "flops" in dw:
         roofline = {"bound": "tensor", "kernel": dom, "achieved": kernels[dom]["achieved"],
                     "peak": tflops_peak, "unit": "TFLOP/s", "frac": kernels[dom]["frac"],
-                    "traffic": MEASURED_TRAFFIC.get((pcfg.name, dom)),
+                    "traffic": traffic_for(dom, dw["units"]),
                     "peak_source": f"{peaks['source']} bf16 sustained",
                     "work_per_launch": dw["flops"]}
     else:
         roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["achieved"],
                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kernels[dom]["frac"],
-                    "traffic": MEASURED_TRAFFIC.get((pcfg.name, dom)), "peak_source": f"{peaks['source']} copy",
+                    "traffic": traffic_for(dom, dw["units"]), "peak_source": f"{peaks['source']} copy",
                     "work_per_launch": dw["bytes"]}
     selected_flops = sum(work[n]["flops"] for n in ("swa_prefill", "sparse_attn_prefill", "select_prefill"))
     layer_frac = selected_flops / (p_step_ms / 1e3) / 1e12 / tflops_peak
@@ -445,6 +466,9 @@ def run_ours(args, rank, world):
     if args.e2e:
         e2e = run_e2e(args, pcfg, layer, q, k, v, P, o, qd, od, g_step, world, stream)
 
+    # ---- the other workloads (one GPU only: they are reported, not scaled)
+    others = run_other_configs(args, dev, peaks, stream) if (args.configs and world == 1) else None
+
     line = {
         "metric": "hybrid-attn prefill tok/s @1M & decode tok/s @128K per layer; % of roofline",
         "value": round(value, 1), "unit": "tok/s", "n_gpus": world, "steps": args.steps,
@@ -468,13 +492,98 @@ def run_ours(args, rank, world):
                    "roofline": {"bound": "hbm", "achieved": round(d_ach, 1), "peak": peaks["hbm_gbs"],
                                 "unit": "GB/s", "frac": round(d_ach / peaks["hbm_gbs"], 4),
                                 "frac_nominal": round(d_ach / NOMINAL_HBM_GBS, 4),
-                                "traffic": MEASURED_TRAFFIC.get((dcfg.name, "step")), "bytes_per_step": db},
+                                "traffic": traffic_for("decode_step", Bd * L), "bytes_per_step": db},
                    "kernels": d_kern},
+        "other_configs": others,
         "gpu_launches": launches * args.steps,
         "clocks": clk,
         "e2e": e2e,
     }
     return line
+
+
+def run_other_configs(args, dev, peaks, stream):
+    """The other seeded workloads, each timed on its own (device-resident
+    inputs, CUDA events on the launching stream, median of the timed steps),
+    with the roofline fraction of its own algorithmic work: prefill layers
+    against the sustained bf16 peak (selected work: attended pairs x 4 D plus
+    the indexer's 2 r per causal pair), decode steps against the HBM peak
+    (bytes: key index scan, window K/V once per KV group, gathered rows once
+    per KV group, q and o). The 128K decode also runs over the 8-bit key index
+    (16 bytes per token in the scan instead of 32)."""
+    import long_context_hybrid_b200 as rtp
+    out = {}
+    tflops = peaks["bf16_tflops_sustained"]
+    for name in ("prefill_2k_tiny", "prefill_32k", "prefill_128k_all_sparse"):
+        cfg = synth.ALL_CONFIGS[name]
+        d = synth.make_prefill(cfg, device=dev)
+        q, k, v, P = d["q"], d["k"], d["v"], d["P"]
+        layer = rtp.PrefillLayer(cfg.B, cfg.N, cfg.Hq, cfg.Hkv, cfg.ret_heads, cfg.window, cfg.ret_window,
+                                 cfg.topk, dev)
+        o = torch.empty(cfg.B, cfg.N, cfg.Hq, D, dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            layer(q, k, v, P, o)
+        times = []
+        for _ in range(5):
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            layer(q, k, v, P, o)
+            s1.record(stream)
+            torch.cuda.synchronize()
+            times.append(s0.elapsed_time(s1))
+        if layer.device_status() != 0:
+            raise RuntimeError(f"{name}: a prefill kernel reported a timed-out wait")
+        ms = statistics.median(times)
+        flops = 4 * D * len(layer.swa_heads) * cfg.B * swa_pairs(cfg.N, cfg.window)
+        if layer.ret:
+            flops += 4 * D * sparse_pairs(layer.blocks, layer.counts, layer.window_blocks, layer.sink_blocks)
+            flops += 2 * R * len(layer.ret) * cfg.B * causal_pairs(cfg.N)
+        ach = flops / (ms / 1e3) / 1e12
+        out[name] = {"value": round(cfg.B * cfg.N / (ms / 1e3), 1), "unit": "tok/s", "ms_per_step": round(ms, 4),
+                     "roofline": {"bound": "tensor", "achieved": round(ach, 2), "peak": tflops, "unit": "TFLOP/s",
+                                  "frac": round(ach / tflops, 4), "work": "selected work of the layer"}}
+        del d, q, k, v, P, layer, o
+    flush = synth.flush_buffer(dev)
+    for name, bits in (("decode_64k_b32_all_sparse", 16), ("decode_128k_b8", 8)):
+        cfg = synth.ALL_CONFIGS[name]
+        d = synth.make_decode(cfg, device=dev)
+        qd, kc, vc, P = d["q"], d["kc"], d["vc"], d["P"]
+        kindex = rtp.index_project(kc, P, list(range(cfg.Hkv)), list(range(cfg.Hkv)))
+        k8, ks = rtp.index_quantize(kindex, 0, cfg.L // 64) if bits == 8 else (None, None)
+        step = rtp.DecodeStep(cfg.B, cfg.L, cfg.Hq, cfg.Hkv, cfg.ret_heads, cfg.window, cfg.ret_window, cfg.topk,
+                              dev, sink=cfg.sink)
+        od = torch.empty(cfg.B, cfg.Hq, D, dtype=torch.bfloat16, device=dev)
+        step(qd, kc, vc, kindex, P, od, kindex8=k8, kscale=ks)
+        torch.cuda.synchronize()
+        g = step.graph(qd, kc, vc, kindex, P, od, kindex8=k8, kscale=ks)
+        for _ in range(3):
+            flush.zero_()
+            g.replay()
+        times = []
+        for _ in range(10):
+            flush.zero_()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            g.replay()
+            s1.record(stream)
+            torch.cuda.synchronize()
+            times.append(s0.elapsed_time(s1))
+        ms = statistics.median(times)
+        db = decode_bytes(cfg, step.idx, cfg.L, cfg.B)
+        if bits == 8:       # codes of the full groups + their scales + the bf16 rows of a partial group
+            n_full = cfg.L // 64 * 64
+            n_kv = db["scan"] // (cfg.B * cfg.L * R * 2)
+            scan8 = cfg.B * n_kv * (n_full * R + (n_full // 64) * 4 + (cfg.L - n_full) * R * 2)
+            db["total"] += scan8 - db["scan"]
+            db["scan"] = scan8
+        ach = db["total"] / (ms / 1e3) / 1e9
+        key = name if bits == 16 else name + "_8bit_index"
+        out[key] = {"value": round(cfg.B / (ms / 1e3), 1), "unit": "tok/s", "ms_per_step": round(ms, 4),
+                    "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                 "frac": round(ach / peaks["hbm_gbs"], 4), "bytes_per_step": db}}
+        del g, d, qd, kc, vc, P, kindex, k8, ks, step, od
+    torch.cuda.synchronize()
+    return out
 
 
 def run_e2e(args, pcfg, layer, q, k, v, P, o, qd, od, g_step, world, stream):
@@ -577,13 +686,17 @@ def run_e2e(args, pcfg, layer, q, k, v, P, o, qd, od, g_step, world, stream):
 # ---------------------------------------------------------------------------
 # CPU oracle (baseline and reference arm)
 # ---------------------------------------------------------------------------
-def oracle_prefill_rate(pcfg, q, k, v, P, n_blocks: int, seed: int = 0):
+def oracle_prefill_rate(pcfg, q, k, v, P, budget_s: float = 20.0, seed: int = 0):
     """Oracle prefill throughput, extrapolated from a bounded sample.
 
     Times the index projection of the whole sequence (the keys of every KV
     head serving a retrieval head, the queries of every retrieval head) once,
-    then a full layer (all heads) on ``n_blocks`` sampled query blocks, and
-    returns tokens / (t_projection + (N/64) * t_per_block)."""
+    then a full layer (all heads) on the first, last and window-boundary query
+    blocks and on seeded uniformly drawn blocks until ``budget_s`` seconds of
+    block work have run (at least four drawn blocks). The rate is
+    tokens / (t_projection + (N/64) * mean time of a drawn block): the drawn
+    blocks are a uniform sample of the per-block cost, which grows with the
+    block's position; the fixed blocks are reported beside it."""
     import numpy as np
     import oracle as O
     N = q.shape[0]
@@ -593,16 +706,30 @@ def oracle_prefill_rate(pcfg, q, k, v, P, n_blocks: int, seed: int = 0):
     kt = {g: O.project(k[:, g, :], P[g]) for g in sorted(set(h // G for h in pcfg.ret_heads))}
     qt = {h: O.project(q[:, h, :], P[h // G]) for h in pcfg.ret_heads}
     t_proj = time.perf_counter() - t0
+    index = {"kt": kt, "qt": qt}
+
+    def block_time(i):
+        t = time.perf_counter()
+        O.prefill_layer(q, k, v, P, pcfg.ret_heads, pcfg.window, pcfg.ret_window, pcfg.topk,
+                        1 / math.sqrt(D), qblocks=[i], index=index)
+        return time.perf_counter() - t
+
+    wb = pcfg.ret_window // BLOCK
+    fixed = sorted({0, min(nb - 1, wb - 1), min(nb - 1, wb), nb - 1})
+    fixed_t = {i: round(block_time(i), 3) for i in fixed}
     rs = np.random.default_rng(seed)
-    blocks = sorted(set([nb - 1] + rs.choice(nb, n_blocks - 1, replace=False).tolist()))[:n_blocks]
-    t0 = time.perf_counter()
-    O.prefill_layer(q, k, v, P, pcfg.ret_heads, pcfg.window, pcfg.ret_window, pcfg.topk,
-                    1 / math.sqrt(D), qblocks=blocks, index={"kt": kt, "qt": qt})
-    t_blocks = time.perf_counter() - t0
-    per_block = t_blocks / len(blocks)
+    drawn, spent = [], 0.0
+    while len(drawn) < 4 or spent < budget_s:
+        i = int(rs.integers(0, nb))
+        dt = block_time(i)
+        drawn.append((i, round(dt, 3)))
+        spent += dt
+        if len(drawn) >= 64:
+            break
+    per_block = sum(t for _, t in drawn) / len(drawn)
     rate = N / (t_proj + nb * per_block)
     return rate, {"t_projection_s": round(t_proj, 3), "t_per_block_s": round(per_block, 3),
-                  "blocks": blocks}
+                  "drawn_blocks": drawn, "fixed_blocks": fixed_t}
 
 
 def cpu_cores():
@@ -620,14 +747,15 @@ def host_copies(pcfg, dev_tensors):
     return q[0].cpu(), k[0].cpu(), v[0].cpu(), P.cpu()
 
 
-def run_cpu_baseline(pcfg, q, k, v, P, n_blocks):
+def run_cpu_baseline(pcfg, q, k, v, P, budget_s):
     qc, kc_, vc_, Pc = host_copies(pcfg, (q, k, v, P))
     t0 = time.perf_counter()
-    rate, info = oracle_prefill_rate(pcfg, qc, kc_, vc_, Pc, n_blocks)
+    rate, info = oracle_prefill_rate(pcfg, qc, kc_, vc_, Pc, budget_s)
     wall = time.perf_counter() - t0
     return {"value": round(rate, 2), "unit": "tok/s", "cores": cpu_cores(), "kind": "oracle",
-            "sample": (f"{pcfg.name}: index projection of the whole sequence + all {pcfg.Hq} heads on "
-                       f"{len(info['blocks'])} sampled query blocks of 64, extrapolated to N={pcfg.N}"),
+            "sample": (f"{pcfg.name}: index projection of the whole sequence, then all {pcfg.Hq} heads on "
+                       f"{len(info['drawn_blocks'])} uniformly drawn query blocks of 64 (plus the first, last and "
+                       f"window-boundary blocks, reported apart), extrapolated to N={pcfg.N}"),
             "wall_s": round(wall, 1), "detail": info}
 
 
@@ -686,7 +814,10 @@ def main():
     ap.add_argument("--decode", default="decode_128k_b8")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
-    ap.add_argument("--cpu-blocks", type=int, default=4)
+    ap.add_argument("--no-configs", dest="configs", action="store_false",
+                    help="skip the other workloads' timings")
+    ap.add_argument("--cpu-budget", type=float, default=20.0,
+                    help="seconds of oracle block work in the CPU baseline sample")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local = dist_setup(args.gpus)
@@ -698,7 +829,7 @@ def main():
             pcfg = synth.ALL_CONFIGS[args.prefill]
             pd = synth.make_prefill(pcfg, device=torch.device("cuda", 0))
             line["cpu_baseline"] = run_cpu_baseline(pcfg, pd["q"], pd["k"], pd["v"], pd["P"],
-                                                    args.cpu_blocks)
+                                                    args.cpu_budget)
         elif line is not None:
             line["cpu_baseline"] = None
     if rank == 0 and line is not None:

@@ -73,3 +73,15 @@ def test_max_over_ranks_gloo_world2():
         p.join(120)
         assert p.exitcode == 0
     assert out[0] == 15.0 and out[1] == 15.0
+
+
+def test_traffic_is_reported_only_for_the_captured_sources(monkeypatch):
+    files = ["select.cu", "rtp_common.cuh"]
+    digest = bench._sources_digest(files)
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", {
+        "k_current": {"bytes_per_unit": 2.5, "sources": files, "digest": digest},
+        "k_stale": {"bytes_per_unit": 2.5, "sources": files, "digest": "0" * 16},
+    })
+    assert bench.traffic_for("k_current", 1000) == 2500
+    assert bench.traffic_for("k_stale", 1000) is None
+    assert bench.traffic_for("k_missing", 1000) is None

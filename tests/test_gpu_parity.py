@@ -83,7 +83,10 @@ def test_index_project_strided_input():
 # ---------------------------------------------------------------------------
 # Decode selection
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("L,topk", [(5003, 64), (40, 64), (1, 1), (2048, 2048), (70000, 2048)])
+# 24577: one token past a 24576-token slice; 196608 and 200003: rows longer
+# than the largest bench workload
+@pytest.mark.parametrize("L,topk", [(5003, 64), (40, 64), (1, 1), (2048, 2048), (70000, 2048), (24577, 100),
+                                    (196608, 2048), (200003, 2048)])
 def test_select_decode_matches_oracle(L, topk):
     B, Hkv, kv = 2, 2, [0, 0, 1]
     kindex = _clustered_bf16((B, Hkv, L, 16), 10 + L)
@@ -106,10 +109,11 @@ def test_select_decode_matches_oracle(L, topk):
             assert ok, f"b{b} j{j}: {msg}"
 
 
-@pytest.mark.parametrize("L", [1500, 3000, 6000])
+@pytest.mark.parametrize("L", [1500, 3000, 6000, 60000, 250000])
 def test_select_decode_ties_pick_lowest_index(L):
     """All keys equal: the lowest k indices must be chosen (the tied bin fits
-    in shared memory at L = 1500; it does not at 3000 and 6000)."""
+    in shared memory at L = 1500; it does not at 3000 and beyond, and at
+    60000 and 250000 it spans several filter blocks)."""
     topk = 100
     kindex = torch.ones(1, 1, L, 16, dtype=torch.bfloat16)
     qt = torch.ones(1, 1, 16)

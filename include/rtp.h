@@ -237,6 +237,65 @@ RTP_API rtp_status rtp_select_decode_q8(const float* qt, const void* kindex8, co
                                         rtp_stream_t stream);
 
 /*
+ * rtp_kcluster_build - clusters the key index of every (sequence, KV head)
+ * for the two-level decode selection.
+ *   Source: RTPurboV2 article (th-motor.com), the sequence-dimension
+ *   compression paragraph (clustering lets decode skip most semantically
+ *   unrelated tokens; the low-rank key vectors make the cluster centres
+ *   accurate) and the Qwen3-Coder-30B-A3B recipe (the retrieval heads' K
+ *   cache is clustered). The pages give no algorithm; this is Lloyd k-means.
+ *   Over rows 0 .. L-1 of each (sequence, KV head): C = ceil(L / cluster_size)
+ *   centroids start at rows 0, cluster_size, 2 cluster_size, ...; each of
+ *   `iters` rounds assigns every row to its nearest centroid (squared
+ *   Euclidean distance summed over c = 0..15 with every subtraction, square
+ *   and addition rounded to fp32, no fused multiply-add; ties to the smaller
+ *   centroid) and moves every centroid to its cluster's mean (exact int64
+ *   sums of trunc(x * 2^20), mean = fp32(double(sum) / double(count) *
+ *   2^-20); an empty cluster keeps its centroid); a last assignment pairs
+ *   every row with its nearest final centroid.
+ *
+ *   kindex     bf16 [B, Hkv, cap, 16] device (rtp_index_append); cap >= L.
+ *   centroids  fp32 [B, Hkv, C, 16] device out.
+ *   assign     int32 [B, Hkv, L] device out: each row's cluster.
+ *   offsets    int32 [B, Hkv, C + 1] device out, members int32 [B, Hkv, L]
+ *              device out: cluster i's rows are members[offsets[i] ..
+ *              offsets[i+1]) (in no particular order).
+ *   ws         rtp_workspace_size_kcluster_build(B, Hkv, L, cluster_size) bytes.
+ *   cluster_size >= 1, 0 <= iters <= 64, B * Hkv <= 65535.
+ */
+RTP_API size_t rtp_workspace_size_kcluster_build(int B, int Hkv, int L, int cluster_size);
+RTP_API rtp_status rtp_kcluster_build(const void* kindex, int64_t cap, int B, int Hkv, int L, int cluster_size,
+                                      int iters, float* centroids, int32_t* assign, int32_t* offsets,
+                                      int32_t* members, void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * rtp_select_decode_clustered - the two-level token selection over a
+ * clustered key index.
+ *   Source: as rtp_kcluster_build; the 128K decode workload statement for the
+ *   token-level top-k, the sink and the window it is unioned with (by the
+ *   attention calls, as for rtp_select_decode).
+ *   Per (sequence b, retrieval head j): the n_probe clusters of KV head
+ *   kv_of[j] whose centroids score highest against q~ (fp32 dot products;
+ *   ties to the smaller cluster), then the top-k tokens by q~ . k~ among
+ *   those clusters' members and every token appended after the build
+ *   (positions L0 .. L-1), ties to the smaller token; all candidates when
+ *   there are fewer than k.
+ *
+ *   qt         fp32 [B, Hr, 16] device; kindex bf16 [B, Hkv, kindex_cap, 16].
+ *   centroids, offsets, members  from rtp_kcluster_build over L0 rows (C
+ *              clusters).
+ *   idx        int32 [B, Hr, topk] device out: ascending tokens, -1 padded.
+ *   ws         rtp_workspace_size_select_decode_clustered(B, Hr, C, n_probe, L).
+ *   1 <= L0 <= L <= 262144 (RTP_ERR_UNSUPPORTED beyond), n_probe >= 1.
+ */
+RTP_API size_t rtp_workspace_size_select_decode_clustered(int B, int Hr, int C, int n_probe, int L);
+RTP_API rtp_status rtp_select_decode_clustered(const float* qt, const void* kindex, int64_t kindex_cap,
+                                               const float* centroids, const int32_t* offsets,
+                                               const int32_t* members, int B, int L0, int L, int Hr, int Hkv,
+                                               int C, const int32_t* kv_of, int n_probe, int topk, int32_t* idx,
+                                               void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
  * rtp_sparse_attn_prefill - exact attention of retrieval heads over their
  * selected key blocks, the sink blocks and the local window blocks.
  *   Source: RTPurbo digest (honest attention at full dimension over the

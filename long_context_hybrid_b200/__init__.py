@@ -50,6 +50,11 @@ _SIGNATURES = {
     "rtp_workspace_size_select_decode": (_SZ, [_I, _I, _I, _I]),
     "rtp_select_decode": (_I, [_P, _P, _L, _I, _I, _I, _I, _I, _c_i32p, _I, _P, _P, _SZ, _P]),
     "rtp_index_quantize": (_I, [_P, _L, _I, _I, _I, _I, _P, _P, _P]),
+    "rtp_workspace_size_kcluster_build": (_SZ, [_I, _I, _I, _I]),
+    "rtp_kcluster_build": (_I, [_P, _L, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
+    "rtp_workspace_size_select_decode_clustered": (_SZ, [_I, _I, _I, _I, _I]),
+    "rtp_select_decode_clustered": (_I, [_P, _P, _L, _P, _P, _P, _I, _I, _I, _I, _I, _I, _c_i32p, _I, _I, _P, _P, _SZ,
+                                         _P]),
     "rtp_select_decode_q8": (_I, [_P, _P, _P, _P, _L, _I, _I, _I, _I, _I, _c_i32p, _I, _P, _P, _SZ, _P]),
     "rtp_workspace_size_sparse_attn_prefill": (_SZ, [_I, _I, _I, _I]),
     "rtp_sparse_attn_prefill": (_I, [_P, Strides, _P, Strides, _P, Strides, _P, Strides, _I, _I, _I,
@@ -234,6 +239,60 @@ def select_decode_q8(qt: torch.Tensor, kindex8: torch.Tensor, kscale: torch.Tens
     _check(lib().rtp_select_decode_q8(qt.data_ptr(), kindex8.data_ptr(), kscale.data_ptr(), kindex.data_ptr(),
                                       kindex.shape[2], B, L, Hr, Hkv, r, _i32(kv_of_ret), topk, idx.data_ptr(),
                                       _wsptr(buf), nbytes, _stream(stream)), "rtp_select_decode_q8")
+    return idx
+
+
+class KeyClusters:
+    """The clustered key index of a cache (rtp_kcluster_build): centroids
+    [B,Hkv,C,r] fp32, assign [B,Hkv,L0], and the members of every cluster as
+    offsets [B,Hkv,C+1] / members [B,Hkv,L0] (int32), over the first L0 rows."""
+
+    def __init__(self, centroids, assign, offsets, members, L0):
+        self.centroids, self.assign, self.offsets, self.members, self.L0 = centroids, assign, offsets, members, L0
+
+    @property
+    def C(self):
+        return self.centroids.shape[2]
+
+
+def kcluster_build(kindex: torch.Tensor, L: int, cluster_size: int = 64, iters: int = 2, ws=None,
+                   stream=None) -> KeyClusters:
+    """Lloyd k-means over rows 0..L-1 of every (sequence, KV head) of the key
+    index kindex [B,Hkv,cap,r]."""
+    B, Hkv, cap, r = kindex.shape
+    assert kindex.is_contiguous()
+    C = (L + cluster_size - 1) // cluster_size
+    dev = kindex.device
+    cen = torch.empty(B, Hkv, C, r, dtype=torch.float32, device=dev)
+    asg = torch.empty(B, Hkv, L, dtype=torch.int32, device=dev)
+    off = torch.empty(B, Hkv, C + 1, dtype=torch.int32, device=dev)
+    mem = torch.empty(B, Hkv, L, dtype=torch.int32, device=dev)
+    need = lib().rtp_workspace_size_kcluster_build(B, Hkv, L, cluster_size)
+    buf, nbytes = _ws(need, dev, ws)
+    _check(lib().rtp_kcluster_build(kindex.data_ptr(), cap, B, Hkv, L, cluster_size, iters, cen.data_ptr(),
+                                    asg.data_ptr(), off.data_ptr(), mem.data_ptr(), _wsptr(buf), nbytes,
+                                    _stream(stream)), "rtp_kcluster_build")
+    return KeyClusters(cen, asg, off, mem, L)
+
+
+def select_decode_clustered(qt: torch.Tensor, kindex: torch.Tensor, clusters: KeyClusters,
+                            kv_of_ret: Sequence[int], n_probe: int, topk: int, L: Optional[int] = None,
+                            idx: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """Two-level token top-k: the n_probe best clusters by centroid score, then
+    the top-k tokens among their members and the rows appended after the
+    build (clusters.L0 .. L-1) -> idx [B,Hr,topk] int32 ascending."""
+    B, Hr, r = qt.shape
+    Hkv, cap = kindex.shape[1], kindex.shape[2]
+    L = cap if L is None else L
+    if idx is None:
+        idx = torch.empty(B, Hr, topk, dtype=torch.int32, device=qt.device)
+    need = lib().rtp_workspace_size_select_decode_clustered(B, Hr, clusters.C, n_probe, L)
+    buf, nbytes = _ws(need, qt.device, ws)
+    _check(lib().rtp_select_decode_clustered(qt.data_ptr(), kindex.data_ptr(), cap, clusters.centroids.data_ptr(),
+                                             clusters.offsets.data_ptr(), clusters.members.data_ptr(), B,
+                                             clusters.L0, L, Hr, Hkv, clusters.C, _i32(kv_of_ret), n_probe, topk,
+                                             idx.data_ptr(), _wsptr(buf), nbytes, _stream(stream)),
+           "rtp_select_decode_clustered")
     return idx
 
 
@@ -502,7 +561,7 @@ class DecodeStep:
 
 
 __all__ = ["lib", "RtpError", "index_project", "index_append", "index_quantize", "select_prefill", "select_decode",
-           "select_decode_q8",
+           "select_decode_q8", "KeyClusters", "kcluster_build", "select_decode_clustered",
            "sparse_attn_prefill", "triangle_prefill", "sparse_attn_decode", "swa", "decode_attn_hybrid",
            "PrefillLayer", "DecodeStep", "OrthrosStep",
            "kv_of", "LIB_PATH"]

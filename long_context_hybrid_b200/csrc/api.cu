@@ -199,6 +199,52 @@ rtp_status rtp_select_decode_q8(const float* qt, const void* kindex8, const floa
                                         topk, idx, ws, (cudaStream_t)stream));
 }
 
+size_t rtp_workspace_size_kcluster_build(int B, int Hkv, int L, int cluster_size) {
+  if (B < 1 || Hkv < 1 || L < 1 || cluster_size < 1) return 0;
+  return kcluster_build_ws_bytes(B, Hkv, L, cluster_size);
+}
+
+rtp_status rtp_kcluster_build(const void* kindex, int64_t cap, int B, int Hkv, int L, int cluster_size, int iters,
+                              float* centroids, int32_t* assign, int32_t* offsets, int32_t* members, void* ws,
+                              size_t ws_bytes, rtp_stream_t stream) {
+  if (!kindex || !centroids || !assign || !offsets || !members) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || Hkv < 1 || L < 1 || cap < L || cluster_size < 1 || iters < 0 || iters > 64) return RTP_ERR_INVALID_ARG;
+  if ((int64_t)B * Hkv > 65535) return RTP_ERR_UNSUPPORTED;
+  if (!aligned16(kindex) || (reinterpret_cast<uintptr_t>(centroids) & 3u) || (reinterpret_cast<uintptr_t>(assign) & 3u) ||
+      (reinterpret_cast<uintptr_t>(offsets) & 3u) || (reinterpret_cast<uintptr_t>(members) & 3u))
+    return RTP_ERR_INVALID_ARG;
+  const size_t need = kcluster_build_ws_bytes(B, Hkv, L, cluster_size);
+  if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
+  rtp_status st = check_device();
+  if (st != RTP_OK) return st;
+  return from_cuda(launch_kcluster_build(kindex, cap, B, Hkv, L, cluster_size, iters, centroids, assign, offsets,
+                                         members, ws, (cudaStream_t)stream));
+}
+
+size_t rtp_workspace_size_select_decode_clustered(int B, int Hr, int C, int n_probe, int L) {
+  if (B < 1 || Hr < 1 || C < 1 || n_probe < 1 || L < 1) return 0;
+  return kcluster_select_ws_bytes(B, Hr, C, n_probe, L);
+}
+
+rtp_status rtp_select_decode_clustered(const float* qt, const void* kindex, int64_t kindex_cap, const float* centroids,
+                                       const int32_t* offsets, const int32_t* members, int B, int L0, int L, int Hr,
+                                       int Hkv, int C, const int32_t* kv_of, int n_probe, int topk, int32_t* idx,
+                                       void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  if (!qt || !kindex || !centroids || !offsets || !members || !kv_of || !idx) return RTP_ERR_INVALID_ARG;
+  if (B < 1 || Hr < 1 || Hr > kMaxHeads || Hkv < 1 || C < 1 || n_probe < 1 || topk < 1) return RTP_ERR_INVALID_ARG;
+  if (L0 < 1 || L < L0 || kindex_cap < L) return RTP_ERR_INVALID_ARG;
+  if (L > kClusterSelectMaxTokens || topk > kMaxDecodeTopk) return RTP_ERR_UNSUPPORTED;
+  if (!aligned16(qt) || !aligned16(kindex) || (reinterpret_cast<uintptr_t>(idx) & 3u)) return RTP_ERR_INVALID_ARG;
+  for (int j = 0; j < Hr; ++j)
+    if (kv_of[j] < 0 || kv_of[j] >= Hkv) return RTP_ERR_INVALID_ARG;
+  const size_t need = kcluster_select_ws_bytes(B, Hr, C, n_probe, L);
+  if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
+  rtp_status st = check_device();
+  if (st != RTP_OK) return st;
+  return from_cuda(launch_kcluster_select(qt, kindex, kindex_cap, centroids, offsets, members, B, L0, L, Hr, Hkv, C,
+                                          kv_of, n_probe, topk, idx, ws, (cudaStream_t)stream));
+}
+
 size_t rtp_workspace_size_sparse_attn_prefill(int B, int N, int Hr, int topk) {
   (void)B; (void)N; (void)Hr; (void)topk;
   return kStatusBytes;

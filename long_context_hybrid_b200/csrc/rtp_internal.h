@@ -53,6 +53,18 @@ struct IndexRef {
   int64_t cap;
 };
 
+// K-cache clustering: k-means over a key index and the two-level selection.
+size_t kcluster_build_ws_bytes(int B, int Hkv, int L, int S);
+cudaError_t launch_kcluster_build(const void* kindex, int64_t cap, int B, int Hkv, int L, int S, int iters,
+                                  float* mu, int32_t* assign, int32_t* offsets, int32_t* members, void* ws,
+                                  cudaStream_t stream);
+size_t kcluster_select_ws_bytes(int B, int Hr, int C, int n_probe, int L);
+cudaError_t launch_kcluster_select(const float* qt, const void* kindex, int64_t cap, const float* mu,
+                                   const int32_t* offsets, const int32_t* members, int B, int L0, int L, int Hr,
+                                   int Hkv, int C, const int32_t* kv_of, int n_probe, int topk, int32_t* idx,
+                                   void* ws, cudaStream_t stream);
+constexpr int kClusterSelectMaxTokens = 262144;
+
 // Largest token top-k of a decode selection (any k >= L selects every token).
 constexpr int kMaxDecodeTopk = 1 << 22;
 size_t select_decode_ws_bytes(int B, int L, int Hr, int topk);

@@ -12,11 +12,13 @@
 //     a row only sees its own block's set, with the causal mask.
 //
 // Warp roles (64 + 128 * NQ threads):
-//   warp 0   TMA producer: the Q tiles once, then K and V of two list blocks
-//            (128 keys) per step into a 2-stage ring (128-byte swizzle);
+//   warp 0   TMA producer: the Q tiles once (NQ = 2), then K and V of two
+//            list blocks (128 keys) per step into an ST-stage ring (128-byte
+//            swizzle);
 //   warp 1   TMEM owner and single-thread MMA issuer:
-//            S_t = Q_t K^T (M=128, N=128, K=128, both operands in shared
-//            memory) and O_t += P_t V (P read from TMEM, V read MN-major);
+//            S_t = Q_t K^T (M=128, N=128, K=128; NQ = 2: Q from shared memory,
+//            NQ = 1: Q from TMEM) and O_t += P_t V (P read from TMEM, V read
+//            MN-major);
 //   softmax  warps 2.. : one warpgroup of 4 warps per query tile; warp w reads
 //            TMEM lanes 32 (w % 4) .. +31, so thread r owns row r (TMEM lane r):
 //            it reads S, masks, keeps an online softmax in the log2 domain
@@ -27,7 +29,13 @@
 //            in TMEM, where the next MMA reads it; each 64-key half is handled
 //            on its own so that a thread holds 64 scores at a time.
 // With NQ = 2 the MMA order QK0 QK1 | PV0 QK0' PV1 QK1' | ... keeps the tensor
-// core busy on one tile while the other tile's softmax runs.
+// core busy on one tile while the other tile's softmax runs, and each K/V
+// stage feeds both tiles. With NQ = 1 a stage feeds one tile, so the ring is
+// three stages deep: the retrieval heads' query tile lives in TMEM (the
+// softmax threads store their own rows there), which frees the shared memory
+// for the third stage, and the copies of tile j + 2 start one tile earlier
+// than with two stages (their key blocks lie anywhere in the sequence, most
+// of them in DRAM).
 // Every wait is bounded; a wait that runs out marks the CTA aborted, all roles
 // drain, TMEM is freed and RTP_ERR_TIMEOUT is written to `status`.
 #include "attn_prefill_common.cuh"
@@ -40,25 +48,27 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kStages = 2;
+constexpr int kMaxStages = 3;
 constexpr uint32_t kQTileBytes = 32768;                       // [D half][128 rows][128 B]
 constexpr uint32_t kStageBytes = 65536;                       // K 32 KB + V 32 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr int kStatusTimeout = 4;
 
-template <int NQ>
+template <int NQ, int ST>
 struct Layout {
   static constexpr int kThreads = 64 + 128 * NQ;
-  static constexpr uint32_t kQOff = 0;
-  static constexpr uint32_t kKVOff = NQ * kQTileBytes;
-  static constexpr uint32_t kListOff = kKVOff + kStages * kStageBytes;
+  static constexpr uint32_t kQOff = 0;                                   // NQ = 2 only
+  static constexpr uint32_t kKVOff = NQ == 2 ? NQ * kQTileBytes : 0;
+  static constexpr uint32_t kListOff = kKVOff + ST * kStageBytes;
   // TMEM columns: NQ = 2 -> tile t: S at 256 t, O at 256 t + 128.
-  //               NQ = 1 -> S buffers at 0 and 128, O at 256.
+  //               NQ = 1 -> S buffers at 0 and 128, O at 256, Q at 384
+  //               (64 columns of bf16 pairs).
+  static constexpr uint32_t kQTmem = 384;
 };
 
 struct Bars {
   uint64_t q_full;
-  uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+  uint64_t k_full[kMaxStages], v_full[kMaxStages], kv_empty[kMaxStages];
   uint64_t s_full[2], p_full[2], pv_done;
   uint64_t fin;
   uint32_t tmem_base;
@@ -166,6 +176,15 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint3
                 kk > 0 ? 1u : 0u);
   }
 }
+// Issue S = Q K^T with Q read from TMEM (128 lanes x 64 columns of bf16 pairs).
+__device__ __forceinline__ void issue_qk_tq(uint32_t d_tmem, uint32_t q_tmem, uint32_t k_smem) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+    mma_bf16_ts(d_tmem, q_tmem + kk * 8u, desc_sw128(k_smem + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+  }
+}
 // Issue O (+)= P V for one Q tile (P in TMEM: 8 K-steps of 16 keys = 8 columns each).
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
@@ -177,12 +196,13 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
 
 }  // namespace
 
-template <int NQ>
+template <int NQ, int ST>
 __global__ void __launch_bounds__(64 + 128 * NQ, 1)
 prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        int* status) {
-  using Lay = Layout<NQ>;
+  static_assert(ST >= 2 && ST <= kMaxStages, "ring depth");
+  using Lay = Layout<NQ, ST>;
   constexpr int NT = Lay::kThreads;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -216,8 +236,8 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
     if (tid == 0) bars.kb_lo = lo;
   }
   if (tid == 0) {
-    mbar_init(smem_u32(&bars.q_full), 1);
-    for (int s = 0; s < kStages; ++s) {
+    mbar_init(smem_u32(&bars.q_full), NQ == 1 ? 128 : 1);    // NQ = 1: the softmax threads' Q rows
+    for (int s = 0; s < ST; ++s) {
       mbar_init(smem_u32(&bars.k_full[s]), 1);
       mbar_init(smem_u32(&bars.v_full[s]), 1);
       mbar_init(smem_u32(&bars.kv_empty[s]), 1);
@@ -249,7 +269,7 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
       tma_prefetch(&tmK);
       tma_prefetch(&tmV);
       const uint32_t qbar = smem_u32(&bars.q_full);
-      if (!p.withhold_q) {
+      if (NQ == 2 && !p.withhold_q) {
         mbar_arrive_expect_tx(qbar, kQTileBytes * NQ);
 #pragma unroll
         for (int t = 0; t < NQ; ++t) {
@@ -259,8 +279,8 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
       }
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
-        const int s = j & 1;
-        if (j >= kStages && !mbar_wait(smem_u32(&bars.kv_empty[s]), ((j - kStages) >> 1) & 1, abort_flag)) break;
+        const int s = j % ST;
+        if (j >= ST && !mbar_wait(smem_u32(&bars.kv_empty[s]), (j / ST - 1) & 1, abort_flag)) break;
         int kb0, kb1;
         if (NQ == 1 && p.sparse) {
           kb0 = list[2 * j].x;
@@ -294,10 +314,10 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
         }
       }
       if (*abort_flag) {
-        if (!p.withhold_q) wait_short(qbar, 0);
-        for (int j = max(0, issued - kStages); j < issued; ++j) {
-          wait_short(smem_u32(&bars.k_full[j & 1]), (j >> 1) & 1);
-          wait_short(smem_u32(&bars.v_full[j & 1]), (j >> 1) & 1);
+        if (NQ == 2 && !p.withhold_q) wait_short(qbar, 0);
+        for (int j = max(0, issued - ST); j < issued; ++j) {
+          wait_short(smem_u32(&bars.k_full[j % ST]), (j / ST) & 1);
+          wait_short(smem_u32(&bars.v_full[j % ST]), (j / ST) & 1);
         }
       }
     }
@@ -342,21 +362,22 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
           }
         }
       } else {
-        // QK(0) | QK(j+1) PV(j) | ... with S double-buffered
+        // QK(0) | QK(j+1) PV(j) | ... with S double-buffered, Q from TMEM,
+        // K/V tile j in ring stage j % ST
         for (int j = 0; ok && j <= n_tiles; ++j) {
           if (j < n_tiles) {
-            const int s = j & 1;
-            if (!mbar_wait(smem_u32(&bars.k_full[s]), (j >> 1) & 1, abort_flag)) { ok = false; break; }
+            const int s = j % ST, sb2 = j & 1;
+            if (!mbar_wait(smem_u32(&bars.k_full[s]), (j / ST) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            issue_qk(tmem + s * 128u, q_s, sb + Lay::kKVOff + s * kStageBytes);
-            mma_commit(smem_u32(&bars.s_full[s]));
+            issue_qk_tq(tmem + sb2 * 128u, tmem + Lay::kQTmem, sb + Lay::kKVOff + s * kStageBytes);
+            mma_commit(smem_u32(&bars.s_full[sb2]));
           }
           if (j >= 1) {
-            const int jp = j - 1, s = jp & 1;
-            if (!mbar_wait(smem_u32(&bars.p_full[s]), (jp >> 1) & 1, abort_flag)) { ok = false; break; }
-            if (!mbar_wait(smem_u32(&bars.v_full[s]), (jp >> 1) & 1, abort_flag)) { ok = false; break; }
+            const int jp = j - 1, s = jp % ST, sb2 = jp & 1;
+            if (!mbar_wait(smem_u32(&bars.p_full[sb2]), (jp >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(smem_u32(&bars.v_full[s]), (jp / ST) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            issue_pv(tmem + 256, tmem + s * 128u, sb + Lay::kKVOff + s * kStageBytes + 32768u, jp > 0);
+            issue_pv(tmem + 256, tmem + sb2 * 128u, sb + Lay::kKVOff + s * kStageBytes + 32768u, jp > 0);
             mma_commit(smem_u32(&bars.pv_done));
             mma_commit(smem_u32(&bars.kv_empty[s]));
           }
@@ -378,6 +399,26 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
     const uint32_t o_col = NQ == 2 ? (uint32_t)(t * 256 + 128) : 256u;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
+    if (NQ == 1) {
+      // this thread's query row into TMEM lane r, columns kQTmem .. +63 (bf16
+      // pairs, in memory order); rows past the sequence are zero
+      const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q.p) + (int64_t)b * p.q.sb +
+                                  (int64_t)row * p.q.sn + (int64_t)h * p.q.sh;
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        uint32_t qv[32];
+#pragma unroll
+        for (int v4 = 0; v4 < 8; ++v4) {
+          const uint4 x = row < p.Nq ? __ldg(reinterpret_cast<const uint4*>(qrow + c2 * 64) + v4)
+                                     : make_uint4(0u, 0u, 0u, 0u);
+          qv[4 * v4] = x.x; qv[4 * v4 + 1] = x.y; qv[4 * v4 + 2] = x.z; qv[4 * v4 + 3] = x.w;
+        }
+        tmem_st32(tmem + lane_off + Lay::kQTmem + c2 * 32u, qv);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars.q_full));
+    }
     for (int j = 0; j < n_tiles; ++j) {
       const int sbuf = NQ == 2 ? t : (j & 1);
       const uint32_t s_col = NQ == 2 ? (uint32_t)(t * 256) : (uint32_t)(sbuf * 128);
@@ -536,9 +577,18 @@ prefill_attn_tc_kernel(const PrefillAttnParams p, const __grid_constant__ CUtens
   if (tid == 0 && bars.abort) atomicExch(status, kStatusTimeout);
 }
 
-size_t prefill_attn_tc_smem_bytes(const PrefillAttnParams& p) {
-  const uint32_t list_off = p.sparse ? Layout<1>::kListOff : Layout<2>::kListOff;
+namespace {
+size_t smem_bytes(uint32_t list_off, const PrefillAttnParams& p) {
   return 1024 + list_off + (size_t)p.list_cap * sizeof(int2) + sizeof(Bars);
+}
+}  // namespace
+
+// Retrieval heads take the three-stage ring when their block list leaves room
+// for it, else two stages.
+size_t prefill_attn_tc_smem_bytes(const PrefillAttnParams& p) {
+  if (!p.sparse) return smem_bytes(Layout<2, 2>::kListOff, p);
+  const size_t s3 = smem_bytes(Layout<1, 3>::kListOff, p);
+  return s3 <= 227 * 1024 ? s3 : smem_bytes(Layout<1, 2>::kListOff, p);
 }
 
 cudaError_t launch_prefill_attn_tc(const PrefillAttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
@@ -546,17 +596,18 @@ cudaError_t launch_prefill_attn_tc(const PrefillAttnParams& p, const CUtensorMap
   const size_t smem = prefill_attn_tc_smem_bytes(p);
   (void)n_tiles;
   if (p.sparse) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_attn_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    const bool three = smem == smem_bytes(Layout<1, 3>::kListOff, p);
+    auto kernel = three ? prefill_attn_tc_kernel<1, 3> : prefill_attn_tc_kernel<1, 2>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((p.Nq + 127) / 128, p.n_heads, B);
-    prefill_attn_tc_kernel<1><<<grid, Layout<1>::kThreads, smem, stream>>>(p, tmQ, tmK, tmV, status);
+    kernel<<<grid, Layout<1, 3>::kThreads, smem, stream>>>(p, tmQ, tmK, tmV, status);
   } else {
-    cudaError_t e = cudaFuncSetAttribute(prefill_attn_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(prefill_attn_tc_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((p.Nq + 255) / 256, p.n_heads, B);
-    prefill_attn_tc_kernel<2><<<grid, Layout<2>::kThreads, smem, stream>>>(p, tmQ, tmK, tmV, status);
+    prefill_attn_tc_kernel<2, 2><<<grid, Layout<2, 2>::kThreads, smem, stream>>>(p, tmQ, tmK, tmV, status);
   }
   return cudaGetLastError();
 }

@@ -173,6 +173,18 @@ def causal_pairs(N: int) -> int:
     return BLOCK * BLOCK * nb * (nb - 1) // 2 + BLOCK * (BLOCK + 1) // 2 * nb
 
 
+def triangle_pairs(N: int, sink_blocks: int, window_blocks: int, last: int) -> int:
+    """Attended causal pairs of one head under the triangle-shaped mask:
+    streaming-region query block i attends its band blocks (min(i+1, wb)) and
+    the sink blocks outside the band, the diagonal block holding 64*65/2
+    causal pairs; a row t of the last region attends every key u <= t."""
+    n_stream = N - last
+    nb = n_stream // BLOCK
+    blocks = sum(min(i + 1, window_blocks) + max(0, min(sink_blocks, i + 1 - window_blocks)) for i in range(nb))
+    pairs = (blocks - nb) * BLOCK * BLOCK + nb * BLOCK * (BLOCK + 1) // 2
+    return pairs + sum(n_stream + t + 1 for t in range(last))
+
+
 def decode_bytes(cfg, idx: torch.Tensor, L: int, B: int) -> dict:
     """HBM bytes a decode step must move: the key index of every KV head that
     serves a retrieval head (32 B/token), the window K/V of every KV group once
@@ -589,7 +601,124 @@ def run_other_configs(args, dev, peaks, stream):
                     "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                  "frac": round(ach / peaks["hbm_gbs"], 4), "bytes_per_step": db}}
         del g, d, qd, kc, vc, P, kindex, k8, ks, step, od
+    out.update(run_preset_configs(dev, peaks, stream, flush))
     torch.cuda.synchronize()
+    return out
+
+
+def _time_graph(fn, stream, flush, reps=10):
+    """Median CUDA-event time (ms) of ``fn`` captured as one graph, L2 flushed
+    before every replay."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    for _ in range(3):
+        flush.zero_()
+        g.replay()
+    times = []
+    for _ in range(reps):
+        flush.zero_()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        g.replay()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        times.append(s0.elapsed_time(s1))
+    del g
+    return statistics.median(times)
+
+
+def run_preset_configs(dev, peaks, stream, flush):
+    """The rows beyond the hot path, each on the workload shape it belongs to:
+    the 128K decode over a clustered key index (two-level selection, then the
+    attention), Orthros' decode (SWA plus a full cross-attention over the
+    128K cache, every head), and the triangle-mask prefill on the 128K
+    all-sparse shape (sink block, 2048-token band, last 2048 queries dense)."""
+    import long_context_hybrid_b200 as rtp
+    out = {}
+    hbm = peaks["hbm_gbs"]
+    tflops = peaks["bf16_tflops_sustained"]
+    cfg = synth.DECODE_128K
+    d = synth.make_decode(cfg, device=dev)
+    qd, kc, vc, P = d["q"], d["kc"], d["vc"], d["P"]
+    B, L, Hq, Hkv = cfg.B, cfg.L, cfg.Hq, cfg.Hkv
+    kindex = rtp.index_project(kc, P, list(range(Hkv)), list(range(Hkv)))
+    ret = list(cfg.ret_heads)
+    kv_ret = [rtp.kv_of(h, Hq, Hkv) for h in ret]
+    swa_heads = [h for h in range(Hq) if h not in ret]
+    # clustered selection: clusters of 64 tokens, 64 probed per head
+    cl = rtp.kcluster_build(kindex, L, 64, 2)
+    n_probe = 64
+    qt = torch.empty(B, len(ret), R, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, len(ret), cfg.topk, dtype=torch.int32, device=dev)
+    od = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+    ws_sel = torch.empty(rtp.lib().rtp_workspace_size_select_decode_clustered(B, len(ret), cl.C, n_probe, L),
+                         dtype=torch.uint8, device=dev)
+    ws_att = torch.empty(rtp.lib().rtp_workspace_size_decode_attn_hybrid(B, L, Hq, cfg.topk, cfg.window),
+                         dtype=torch.uint8, device=dev)
+
+    def clustered_step():
+        rtp.index_project(qd.unsqueeze(1), P, ret, kv_ret, out=qt.view(B, len(ret), 1, R))
+        rtp.select_decode_clustered(qt, kindex, cl, kv_ret, n_probe, cfg.topk, idx=idx, ws=ws_sel)
+        rtp.decode_attn_hybrid(qd, kc, vc, od, ret, idx, cfg.ret_window, swa_heads, cfg.window, cfg.sink, None,
+                               ws_att)
+    ms = _time_graph(clustered_step, stream, flush)
+    counts = torch.diff(cl.offsets.long(), dim=-1)                         # [B, Hkv, C]
+    probed = 0
+    for j, g in enumerate(kv_ret):
+        top = torch.topk((cl.centroids[:, g] @ qt[:, j].unsqueeze(-1)).squeeze(-1), n_probe, dim=1).indices
+        probed += int(torch.gather(counts[:, g], 1, top).sum())
+    db = decode_bytes(cfg, idx, L, B)
+    sel_bytes = B * len(kv_ret) * cl.C * R * 4 + probed * R * 2       # centroids + the probed rows of the index
+    total = db["total"] - db["scan"] + sel_bytes
+    ach = total / (ms / 1e3) / 1e9
+    out["decode_128k_b8_clustered"] = {
+        "value": round(B / (ms / 1e3), 1), "unit": "tok/s", "ms_per_step": round(ms, 4),
+        "n_probe": n_probe, "cluster_size": 64,
+        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
+                     "bytes_per_step": total}}
+    # Orthros decode: SWA (window 8192) and a full cross-attention, every head
+    orth = rtp.OrthrosStep(B, L, Hq, Hkv, cfg.window, dev)
+    o_ca = torch.empty_like(od)
+    ms = _time_graph(lambda: orth.decode(qd, kc, vc, od, o_ca, L=L), stream, flush)
+    total = B * Hkv * (min(cfg.window, L) + L) * D * 2 * 2 + 3 * B * Hq * D * 2
+    ach = total / (ms / 1e3) / 1e9
+    out["decode_128k_b8_orthros"] = {
+        "value": round(B / (ms / 1e3), 1), "unit": "tok/s", "ms_per_step": round(ms, 4),
+        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
+                     "bytes_per_step": total}}
+    del d, qd, kc, vc, P, kindex, cl, qt, idx, od, ws_sel, ws_att, orth, o_ca
+    # triangle mask on the 128K all-sparse shape
+    pc = synth.PREFILL_128K_ALL
+    dp = synth.make_prefill(pc, device=dev)
+    q, k, v = dp["q"], dp["k"], dp["v"]
+    o = torch.empty(pc.B, pc.N, pc.Hq, D, dtype=torch.bfloat16, device=dev)
+    heads = list(range(pc.Hq))
+    sink, wb, last = 1, pc.ret_window // BLOCK, 2048
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    rtp.triangle_prefill(q, k, v, o, heads, sink, wb, last, ws=ws)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(5):
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        rtp.triangle_prefill(q, k, v, o, heads, sink, wb, last, ws=ws)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        times.append(s0.elapsed_time(s1))
+    if rtp.workspace_status(ws) != 0:
+        raise RuntimeError("triangle prefill reported a timed-out wait")
+    ms = statistics.median(times)
+    flops = 4 * D * triangle_pairs(pc.N, sink, wb, last) * len(heads) * pc.B
+    ach = flops / (ms / 1e3) / 1e12
+    out["prefill_128k_triangle"] = {
+        "value": round(pc.B * pc.N / (ms / 1e3), 1), "unit": "tok/s", "ms_per_step": round(ms, 4),
+        "sink_blocks": sink, "window_blocks": wb, "last_tokens": last,
+        "roofline": {"bound": "tensor", "achieved": round(ach, 2), "peak": tflops, "unit": "TFLOP/s",
+                     "frac": round(ach / tflops, 4), "work": "attended causal pairs x 4 D"}}
+    del dp, q, k, v, o
     return out
 
 

@@ -85,3 +85,9 @@ def test_traffic_is_reported_only_for_the_captured_sources(monkeypatch):
     assert bench.traffic_for("k_current", 1000) == 2500
     assert bench.traffic_for("k_stale", 1000) is None
     assert bench.traffic_for("k_missing", 1000) is None
+
+
+def test_triangle_pairs_match_oracle_key_sets():
+    for N, sink, wb, last in [(1024, 1, 2, 256), (640, 0, 3, 0), (512, 2, 1, 512), (1536, 1, 4, 320), (960, 3, 2, 64)]:
+        want = sum(len(O.triangle_keys(t, N, sink, wb, last)) for t in range(N))
+        assert bench.triangle_pairs(N, sink, wb, last) == want, (N, sink, wb, last)

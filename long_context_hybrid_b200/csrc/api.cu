@@ -159,8 +159,8 @@ rtp_status rtp_select_decode(const float* qt, const void* kindex, int64_t kindex
   if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
   rtp_status st = check_device();
   if (st != RTP_OK) return st;
-  return from_cuda(launch_select_decode(qt, IndexRef{kindex, nullptr, nullptr, kindex_cap}, B, L, Hr, Hkv, kv_of,
-                                        topk, idx, ws, (cudaStream_t)stream));
+  return from_cuda(launch_select_decode(qt, nullptr, nullptr, IndexRef{kindex, nullptr, nullptr, kindex_cap}, B, L,
+                                        Hr, Hkv, kv_of, topk, idx, ws, (cudaStream_t)stream));
 }
 
 rtp_status rtp_index_quantize(const void* kindex, int64_t cap, int B, int Hkv, int g0, int g1, void* kindex8,
@@ -195,8 +195,8 @@ rtp_status rtp_select_decode_q8(const float* qt, const void* kindex8, const floa
   if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
   rtp_status st = check_device();
   if (st != RTP_OK) return st;
-  return from_cuda(launch_select_decode(qt, IndexRef{kindex, kindex8, kscale, kindex_cap}, B, L, Hr, Hkv, kv_of,
-                                        topk, idx, ws, (cudaStream_t)stream));
+  return from_cuda(launch_select_decode(qt, nullptr, nullptr, IndexRef{kindex, kindex8, kscale, kindex_cap}, B, L,
+                                        Hr, Hkv, kv_of, topk, idx, ws, (cudaStream_t)stream));
 }
 
 size_t rtp_workspace_size_kcluster_build(int B, int Hkv, int L, int cluster_size) {
@@ -457,12 +457,16 @@ rtp_status rtp_decode_step(const void* q, const void* P, const void* kindex, int
   if (Hr > 0) {
     float* qt = reinterpret_cast<float*>(base + align256(decode_attn_ws_bytes(B, L, Hq, topk, wmax)));
     void* ws_sel = reinterpret_cast<char*>(qt) + step_qt_bytes(B, Hr);
-    // q~ = q . P for the retrieval heads (fp32, unrounded), then the top-k
-    cudaError_t e = launch_project(q, (int64_t)Hq * RTP_D, (int64_t)Hq * RTP_D, RTP_D, B, 1, P, ret_heads, kv_of, Hr,
-                                   qt, 1, s);
-    if (e != cudaSuccess) return from_cuda(e);
-    e = launch_select_decode(qt, IndexRef{kindex, kindex8, kscale, kindex_cap}, B, L, Hr, Hkv, kv_of, topk, idx,
-                             ws_sel, s);
+    // q~ = q . P for the retrieval heads (fp32, unrounded, formed by the
+    // selection's first kernel), then the top-k
+    DecodeQuery dq;
+    dq.q = q;
+    dq.q_sb = (int64_t)Hq * RTP_D;
+    dq.q_sh = RTP_D;
+    dq.P = P;
+    for (int i = 0; i < Hr; ++i) dq.qhead[i] = ret_heads[i];
+    cudaError_t e = launch_select_decode(nullptr, &dq, qt, IndexRef{kindex, kindex8, kscale, kindex_cap}, B, L, Hr,
+                                         Hkv, kv_of, topk, idx, ws_sel, s);
     if (e != cudaSuccess) return from_cuda(e);
   }
   // The kernel before the attention is the selection's filter (or nothing of

@@ -68,9 +68,20 @@ constexpr int kClusterSelectMaxTokens = 262144;
 // Largest token top-k of a decode selection (any k >= L selects every token).
 constexpr int kMaxDecodeTopk = 1 << 22;
 size_t select_decode_ws_bytes(int B, int L, int Hr, int topk);
-cudaError_t launch_select_decode(const float* qt, IndexRef index, int B, int L, int Hr,
-                                 int Hkv, const int32_t* kv_of, int topk, int32_t* idx,
-                                 void* ws, cudaStream_t stream);
+// The step's queries, projected by the selection's first kernel (q~ = q . P
+// of the head's KV group, fp32 in the order of the standalone projection).
+constexpr int kDecodeQueryHeads = 128;
+struct DecodeQuery {
+  const void* q;              // bf16 [B, Hq, D] (row strides q_sb, q_sh, elements)
+  int64_t q_sb, q_sh;
+  const void* P;              // bf16 [Hkv, D, R]
+  int qhead[kDecodeQueryHeads];   // query head of each retrieval head
+};
+// Decode selection: q~ from `qt` ([B, Hr, R] fp32) or, when `dq` is given,
+// formed into `qt_out` by the first kernel.
+cudaError_t launch_select_decode(const float* qt, const DecodeQuery* dq, float* qt_out, IndexRef index, int B,
+                                 int L, int Hr, int Hkv, const int32_t* kv_of, int topk, int32_t* idx, void* ws,
+                                 cudaStream_t stream);
 
 size_t select_prefill_ws_bytes(int B, int N, int Hr, int topk);
 cudaError_t launch_select_prefill(const void* qt, const void* kt, int64_t kt_cap, int B, int N, int Hr, int Hkv,

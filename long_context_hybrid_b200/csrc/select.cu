@@ -3,7 +3,11 @@
 // statement: token-level top-2048 over the whole cache; RTPurbo digest: the
 // 16-d indexer is the scout). Exact ties rank the smaller token first.
 //
-// Two kernels:
+// Three kernels:
+//   zero    clears the histograms and the per-row state; inside a decode step
+//           it also forms q~ = q . P. The scan launches behind it at once
+//           (programmatic dependent launch) and waits for it before its
+//           first read.
 //   scan    one pass over the key index by as many CTAs as fit on the GPU, each
 //           a contiguous run of the (sequence, KV group) token ranges laid end
 //           to end; a group's index is read once for all its retrieval heads
@@ -150,6 +154,7 @@ decode_scan_kernel(const float* __restrict__ qt, const IndexRef index, int B, in
   const int ufull = Q8 ? (L / QGROUP_TOKENS) * QGROUP_TOKENS : 0;   // tokens read from the codes
   const int64_t ngroups = (kcap + QGROUP_TOKENS - 1) / QGROUP_TOKENS;
   pdl_trigger();                                       // the filter may launch and wait for this grid
+  pdl_wait();                                          // q~ and the cleared histograms (previous kernel)
   extern __shared__ uint32_t shist[];                  // [heads of the group][kBins]
   __shared__ float qs[MAXJ > 0 ? 1 : kMaxHeadsPerGroup][RTP_R];
   const int64_t total = (int64_t)B * gh.n_ag * L;
@@ -561,8 +566,48 @@ size_t select_decode_ws_bytes(int B, int L, int Hr, int topk) {
   return decode_ws_layout(nullptr, B, L, Hr).total;
 }
 
-cudaError_t launch_select_decode(const float* qt, IndexRef index, int B, int L, int Hr, int Hkv,
-                                 const int32_t* kv_of, int topk, int32_t* idx, void* ws, cudaStream_t stream) {
+// Clears the selection's histograms and row state and, inside a decode step,
+// forms q~ = q . P for the retrieval heads (CTA i < B*Hr forms row i: fp32
+// FMAs over d = 0 .. D-1 in order, as the standalone projection does). The
+// scan launches behind it at once and waits for it before its first read.
+struct ZeroParams {
+  uint4* p;
+  size_t n16;
+  float* qt;                  // [B, Hr, R] out (when q is given)
+  int B, Hr;
+  DecodeQuery dq;
+  int kv[kDecodeQueryHeads];  // KV group of each retrieval head
+};
+
+__global__ void __launch_bounds__(256) decode_zero_kernel(const ZeroParams zp) {
+  __shared__ __align__(16) __nv_bfloat16 sP[RTP_D * RTP_R];
+  __shared__ __align__(16) __nv_bfloat16 sq[RTP_D];
+  pdl_trigger();
+  const int tid = threadIdx.x;
+  if (zp.dq.q && blockIdx.x < (unsigned)(zp.B * zp.Hr)) {
+    const int b = blockIdx.x / zp.Hr, j = blockIdx.x - b * zp.Hr;
+    const uint4* Pg = static_cast<const uint4*>(zp.dq.P) + (size_t)zp.kv[j] * (RTP_D * RTP_R / 8);
+    reinterpret_cast<uint4*>(sP)[tid] = __ldg(Pg + tid);                  // 256 x 16 B = D x R bf16
+    if (tid < RTP_D / 8) {
+      const __nv_bfloat16* qr = static_cast<const __nv_bfloat16*>(zp.dq.q) + (int64_t)b * zp.dq.q_sb +
+                                (int64_t)zp.dq.qhead[j] * zp.dq.q_sh;
+      reinterpret_cast<uint4*>(sq)[tid] = __ldg(reinterpret_cast<const uint4*>(qr) + tid);
+    }
+    __syncthreads();
+    if (tid < RTP_R) {
+      float acc = 0.f;
+#pragma unroll 16
+      for (int d = 0; d < RTP_D; ++d) acc = fmaf(__bfloat162float(sq[d]), __bfloat162float(sP[d * RTP_R + tid]), acc);
+      zp.qt[(size_t)blockIdx.x * RTP_R + tid] = acc;
+    }
+  }
+  for (size_t e = (size_t)blockIdx.x * 256 + tid; e < zp.n16; e += (size_t)gridDim.x * 256)
+    zp.p[e] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+cudaError_t launch_select_decode(const float* qt, const DecodeQuery* dq, float* qt_out, IndexRef index, int B,
+                                 int L, int Hr, int Hkv, const int32_t* kv_of, int topk, int32_t* idx, void* ws,
+                                 cudaStream_t stream) {
   if (topk > kMaxDecodeTopk) return cudaErrorInvalidValue;
   if (Hkv > kMaxGroups) return cudaErrorInvalidValue;
   GroupHeads gh;
@@ -580,13 +625,35 @@ cudaError_t launch_select_decode(const float* qt, IndexRef index, int B, int L, 
     max_nj = c > max_nj ? c : max_nj;
   }
   const DecodeWs w = decode_ws_layout(ws, B, L, Hr);
-  cudaError_t e = cudaMemsetAsync(w.hist, 0, w.zero_bytes, stream);
-  if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
-  e = cudaGetDevice(&dev);
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
+  {
+    ZeroParams zp;
+    zp.p = reinterpret_cast<uint4*>(w.hist);
+    zp.n16 = w.zero_bytes / 16;
+    zp.qt = qt_out;
+    zp.B = B;
+    zp.Hr = Hr;
+    if (dq) {
+      zp.dq = *dq;
+      for (int j = 0; j < Hr; ++j) zp.kv[j] = kv_of[j];
+      qt = qt_out;
+    } else {
+      zp.dq.q = nullptr;
+      zp.dq.P = nullptr;
+      zp.dq.q_sb = zp.dq.q_sh = 0;
+    }
+    size_t gz = (zp.n16 + 255) / 256;
+    if (gz > (size_t)sms) gz = sms;
+    if (dq && gz < (size_t)B * Hr) gz = (size_t)B * Hr;
+    if (gz < 1) gz = 1;
+    decode_zero_kernel<<<(unsigned)gz, 256, 0, stream>>>(zp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   // scan: as many CTAs as fit on the GPU at once, each a contiguous run
   const size_t scan_smem = (size_t)max_nj * kBins * sizeof(uint32_t);
   const int64_t total = (int64_t)B * gh.n_ag * L;
@@ -599,8 +666,8 @@ cudaError_t launch_select_decode(const float* qt, IndexRef index, int B, int L, 
     int64_t grid = (int64_t)(per_sm > 0 ? per_sm : 1) * sms;
     const int64_t min_tokens = kScanThreads * kScanBatch;   // at least one batch of tokens per CTA
     if (grid * min_tokens > total) grid = (total + min_tokens - 1) / min_tokens;
-    kernel<<<(int)grid, kScanThreads, scan_smem, stream>>>(qt, index, B, L, Hr, Hkv, gh, w);
-    return cudaGetLastError();
+    return launch_pdl(kernel, dim3((unsigned)grid), dim3(kScanThreads), scan_smem, stream, qt, index, B, L, Hr, Hkv, gh,
+                      w);
   };
   if (index.k8) {
     if (max_nj <= 1) e = scan(decode_scan_kernel<1, kScanBatch, true>);

@@ -225,12 +225,11 @@ NOMINAL_HBM_GBS = 7700.0
 # kernel is built from: when they have changed since the capture, the entry
 # is stale and the line reports null.
 NCU_TRAFFIC = {
-    # one decode step of the 128K x 8 workload at full size (projection, scan,
-    # filter, attention, merge): profiles/decode_128k_b8.md
-    "decode_step": {"bytes_per_unit": 341084416 / (8 * 131072), "unit": "cached token",
-                    "sources": ["select.cu", "decode_attn.cu", "project.cu", "rtp_common.cuh", "rtp_internal.h",
-                                "api.cu"],
-                    "digest": "94381ed62ffb871f"},
+    # one decode step of the 128K x 8 workload at full size (zero + projection,
+    # scan, filter, attention, merge): profiles/decode_128k_b8.md
+    "decode_step": {"bytes_per_unit": 340969984 / (8 * 131072), "unit": "cached token",
+                    "sources": ["select.cu", "decode_attn.cu", "rtp_common.cuh", "rtp_internal.h", "api.cu"],
+                    "digest": "181cf7b94611a2b7"},
 }
 
 

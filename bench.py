@@ -522,7 +522,9 @@ def run_ours(args, rank, world):
 
 def run_other_configs(args, dev, peaks, stream):
     """The other seeded workloads, each timed on its own (device-resident
-    inputs, CUDA events on the launching stream, median of the timed steps),
+    inputs, the layer or step replayed as one CUDA graph, L2 flushed before
+    every timed step, CUDA events on the launching stream, median of the
+    timed steps),
     with the roofline fraction of its own algorithmic work: prefill layers
     against the sustained bf16 peak (selected work: attended pairs x 4 D plus
     the indexer's 2 r per causal pair), decode steps against the HBM peak
@@ -532,6 +534,7 @@ def run_other_configs(args, dev, peaks, stream):
     import long_context_hybrid_b200 as rtp
     out = {}
     tflops = peaks["bf16_tflops_sustained"]
+    flush = synth.flush_buffer(dev)
     for name in ("prefill_2k_tiny", "prefill_32k", "prefill_128k_all_sparse"):
         cfg = synth.ALL_CONFIGS[name]
         d = synth.make_prefill(cfg, device=dev)
@@ -539,13 +542,17 @@ def run_other_configs(args, dev, peaks, stream):
         layer = rtp.PrefillLayer(cfg.B, cfg.N, cfg.Hq, cfg.Hkv, cfg.ret_heads, cfg.window, cfg.ret_window,
                                  cfg.topk, dev)
         o = torch.empty(cfg.B, cfg.N, cfg.Hq, D, dtype=torch.bfloat16, device=dev)
+        layer(q, k, v, P, o)
+        torch.cuda.synchronize()
+        g = layer.graph(q, k, v, P, o)
         for _ in range(3):
-            layer(q, k, v, P, o)
+            g.replay()
         times = []
         for _ in range(5):
+            flush.zero_()                   # L2 flush between timed steps (not timed)
             s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s0.record(stream)
-            layer(q, k, v, P, o)
+            g.replay()
             s1.record(stream)
             torch.cuda.synchronize()
             times.append(s0.elapsed_time(s1))
@@ -560,8 +567,7 @@ def run_other_configs(args, dev, peaks, stream):
         out[name] = {"value": round(cfg.B * cfg.N / (ms / 1e3), 1), "unit": "tok/s", "ms_per_step": round(ms, 4),
                      "roofline": {"bound": "tensor", "achieved": round(ach, 2), "peak": tflops, "unit": "TFLOP/s",
                                   "frac": round(ach / tflops, 4), "work": "selected work of the layer"}}
-        del d, q, k, v, P, layer, o
-    flush = synth.flush_buffer(dev)
+        del d, q, k, v, P, layer, o, g
     for name, bits in (("decode_64k_b32_all_sparse", 16), ("decode_128k_b8", 8)):
         cfg = synth.ALL_CONFIGS[name]
         d = synth.make_decode(cfg, device=dev)

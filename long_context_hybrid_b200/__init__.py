@@ -470,6 +470,19 @@ class PrefillLayer:
             swa(q, k, v, o, self.swa_heads, self.window, 0, self.scale, ws=self.ws_swa, stream=stream)
         return o
 
+    def graph(self, q, k, v, P, o, index_out: Optional[torch.Tensor] = None) -> "torch.cuda.CUDAGraph":
+        """Captures the layer on these buffers into a CUDA graph.
+
+        ``graph.replay()`` then runs every kernel of the layer with one launch
+        from the host (for short sequences the per-call launches dominate),
+        reading ``q``, ``k``, ``v``, ``P`` as they are at replay and writing
+        ``o``. Run the layer once eagerly before capturing, so that every
+        kernel attribute is set."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self(q, k, v, P, o, index_out=index_out)
+        return g
+
     def device_status(self, stream=None) -> int:
         """Synchronises and returns the worst status word of the attention calls."""
         return max(workspace_status(self.ws_sparse, stream), workspace_status(self.ws_swa, stream),

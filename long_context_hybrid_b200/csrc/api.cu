@@ -454,6 +454,7 @@ rtp_status rtp_decode_step(const void* q, const void* P, const void* kindex, int
   cudaStream_t s = (cudaStream_t)stream;
   char* base = static_cast<char*>(ws);
   char* ws_att = base;
+  int filter_ctas = 0;
   if (Hr > 0) {
     float* qt = reinterpret_cast<float*>(base + align256(decode_attn_ws_bytes(B, L, Hq, topk, wmax)));
     void* ws_sel = reinterpret_cast<char*>(qt) + step_qt_bytes(B, Hr);
@@ -466,15 +467,27 @@ rtp_status rtp_decode_step(const void* q, const void* P, const void* kindex, int
     dq.P = P;
     for (int i = 0; i < Hr; ++i) dq.qhead[i] = ret_heads[i];
     cudaError_t e = launch_select_decode(nullptr, &dq, qt, IndexRef{kindex, kindex8, kscale, kindex_cap}, B, L, Hr,
-                                         Hkv, kv_of, topk, idx, ws_sel, s);
+                                         Hkv, kv_of, topk, idx, ws_sel, s, &filter_ctas);
     if (e != cudaSuccess) return from_cuda(e);
+  }
+  // The attention CTAs start on the SMs the scan leaves while the filter
+  // still runs: where a filter CTA sits, one attention CTA fits beside it.
+  // Launching only as many as fit at once keeps any from starting its whole
+  // run of window chunks after the filter ends.
+  int max_ctas = 0;
+  if (filter_ctas > 0) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess)
+      return RTP_ERR_CUDA;
+    if (filter_ctas < sms) max_ctas = 2 * sms - filter_ctas;
   }
   // The kernel before the attention is the selection's filter (or nothing of
   // this call): it writes only idx, so the attention may read q, K and V early.
   return from_cuda(launch_decode_hybrid(q, (int64_t)Hq * RTP_D, RTP_D, kc, ks.b, ks.n, ks.h, vc, vs.b, vs.n, vs.h,
                                         o, (int64_t)Hq * RTP_D, RTP_D, B, L, L - 1, Hq, Hkv, ret_heads, Hr, idx, topk,
                                         ret_window, sink, swa_heads, n_swa, swa_window, scale, ws_att, s,
-                                        /*early_start=*/Hr > 0));
+                                        /*early_start=*/Hr > 0, max_ctas));
 }
 
 rtp_status rtp_decode_attn_hybrid(const void* q, const void* kc, rtp_strides ks, const void* vc, rtp_strides vs,

@@ -500,7 +500,7 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
                                  const int32_t* ret_heads, int n_ret, const int32_t* idx, int topk,
                                  int ret_window, int sink,
                                  const int32_t* swa_heads, int n_swa, int swa_window,
-                                 float scale, void* ws, cudaStream_t stream, bool early_start) {
+                                 float scale, void* ws, cudaStream_t stream, bool early_start, int max_ctas) {
   DecodeParams p;
   p.early_start = early_start ? 1 : 0;
   p.q = static_cast<const __nv_bfloat16*>(q); p.q_sb = q_sb; p.q_sh = q_sh;
@@ -560,8 +560,11 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
+  // every CTA resident at once: two per SM, or the caller's bound (the CTAs
+  // that fit beside the kernel still running before this one)
   const int most = p.n_win_chunks > p.n_gat_chunks ? p.n_win_chunks : p.n_gat_chunks;
-  const int grid = most < kCtasPerSm * sms ? most : kCtasPerSm * sms;
+  const int cap = max_ctas > 0 && max_ctas < kCtasPerSm * sms ? max_ctas : kCtasPerSm * sms;
+  const int grid = most < cap ? most : cap;
   const size_t smem = sizeof(Smem);
   e = cudaFuncSetAttribute(decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -81,7 +81,7 @@ struct DecodeQuery {
 // formed into `qt_out` by the first kernel.
 cudaError_t launch_select_decode(const float* qt, const DecodeQuery* dq, float* qt_out, IndexRef index, int B,
                                  int L, int Hr, int Hkv, const int32_t* kv_of, int topk, int32_t* idx, void* ws,
-                                 cudaStream_t stream);
+                                 cudaStream_t stream, int* filter_ctas = nullptr);
 
 size_t select_prefill_ws_bytes(int B, int N, int Hr, int topk);
 cudaError_t launch_select_prefill(const void* qt, const void* kt, int64_t kt_cap, int B, int N, int Hr, int Hkv,
@@ -112,7 +112,8 @@ cudaError_t launch_decode_hybrid(const void* q, int64_t q_sb, int64_t q_sh,
                                  const int32_t* ret_heads, int n_ret, const int32_t* idx, int topk,
                                  int ret_window, int sink,
                                  const int32_t* swa_heads, int n_swa, int swa_window,
-                                 float scale, void* ws, cudaStream_t stream, bool early_start = false);
+                                 float scale, void* ws, cudaStream_t stream, bool early_start = false,
+                                 int max_ctas = 0);
 
 // Same as launch_decode_attn for retrieval heads, with the partials in a
 // library-owned static device array of kNoAllocScratchBytes.

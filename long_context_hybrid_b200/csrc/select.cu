@@ -607,7 +607,7 @@ __global__ void __launch_bounds__(256) decode_zero_kernel(const ZeroParams zp) {
 
 cudaError_t launch_select_decode(const float* qt, const DecodeQuery* dq, float* qt_out, IndexRef index, int B,
                                  int L, int Hr, int Hkv, const int32_t* kv_of, int topk, int32_t* idx, void* ws,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, int* filter_ctas) {
   if (topk > kMaxDecodeTopk) return cudaErrorInvalidValue;
   if (Hkv > kMaxGroups) return cudaErrorInvalidValue;
   GroupHeads gh;
@@ -700,6 +700,7 @@ cudaError_t launch_select_decode(const float* qt, const DecodeQuery* dq, float* 
   slice = (slice + 511) / 512 * 512;
   n_split = (L + slice - 1) / slice;
   dim3 g2(n_split, Hr, B);
+  if (filter_ctas) *filter_ctas = n_split * rows;
   return launch_pdl(decode_filter_kernel, g2, dim3(kFiltThreads), sizeof(FiltSmem), stream, w, L, Hr, topk, slice,
                     n_split, idx);
 }

@@ -335,6 +335,30 @@ def _prefill_e2e(cfg, data, qblocks, heads=None, check_kt=True):
     return worst, n_amb_rows
 
 
+def test_prefill_layer_graph_replay_matches_eager():
+    """The layer captured as one CUDA graph reads its inputs at replay: a new
+    query gives the same output as an eager call on that query."""
+    cfg = synth.TINY_PREFILL
+    data = synth.make_prefill(cfg, device=DEV)
+    q, k, v, P = data["q"], data["k"], data["v"], data["P"]
+    B, N = q.shape[0], q.shape[1]
+    layer = rtp.PrefillLayer(B, N, cfg.Hq, cfg.Hkv, cfg.ret_heads, cfg.window, cfg.ret_window, cfg.topk, DEV)
+    o_graph = torch.zeros(B, N, cfg.Hq, 128, dtype=torch.bfloat16, device=DEV)
+    layer(q, k, v, P, o_graph)
+    torch.cuda.synchronize()
+    g = layer.graph(q, k, v, P, o_graph)
+    q2 = synth.make_prefill(cfg, device=DEV, seed=cfg.seed + 99)["q"]
+    q.copy_(q2)
+    o_graph.zero_()
+    g.replay()
+    o_eager = torch.zeros_like(o_graph)
+    layer2 = rtp.PrefillLayer(B, N, cfg.Hq, cfg.Hkv, cfg.ret_heads, cfg.window, cfg.ret_window, cfg.topk, DEV)
+    layer2(q2, k, v, P, o_eager)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert torch.equal(o_graph, o_eager)
+
+
 def test_e2e_tiny_prefill_full_oracle():
     cfg = synth.TINY_PREFILL
     data = synth.make_prefill(cfg, device="cpu")
@@ -396,8 +420,12 @@ def test_e2e_decode_reduced():
 
 def test_decode_step_equals_the_three_calls():
     """rtp_decode_step (projection, selection and attention in one call, the
-    attention starting before the selection ends) gives bit for bit what the
-    three calls give one after another."""
+    attention starting before the selection ends) gives what the three calls
+    give one after another: the same selection bit for bit, and outputs
+    within 2^-10 + 2^-6 |o| (the step runs its attention on as many CTAs as
+    fit beside the filter, so its partials group the keys differently: each
+    partial rounds its probabilities to bf16 against its own running max, and
+    the fp32 sums round differently)."""
     cfg = synth.DECODE_128K
     B, L = 3, 20000
     data = synth.make_decode(cfg, device=DEV, B=B, L=L, seed=cfg.seed + 5)
@@ -416,7 +444,9 @@ def test_decode_step_equals_the_three_calls():
         rtp.decode_attn_hybrid(q, kc, vc, o2, ret, idx2, window, swa_heads, window, 1)
         torch.cuda.synchronize()
         assert torch.equal(idx1, idx2)
-        assert torch.equal(o1, o2)
+        a, b = o1.float(), o2.float()
+        tol = 2.0 ** -10 + torch.maximum(a.abs(), b.abs()) * 2.0 ** -6
+        assert bool(((a - b).abs() <= tol).all()), float((a - b).abs().max())
 
 
 @pytest.mark.parametrize("L,ret_window,swa_window,topk", [(6000, 512, 256, 300), (6000, 256, 1024, 129),

@@ -154,7 +154,16 @@ decode_scan_kernel(const float* __restrict__ qt, const IndexRef index, int B, in
   const int ufull = Q8 ? (L / QGROUP_TOKENS) * QGROUP_TOKENS : 0;   // tokens read from the codes
   const int64_t ngroups = (kcap + QGROUP_TOKENS - 1) / QGROUP_TOKENS;
   pdl_trigger();                                       // the filter may launch and wait for this grid
-  pdl_wait();                                          // q~ and the cleared histograms (previous kernel)
+  // q~ and the cleared histograms come from the previous kernel. With a few
+  // heads per group (MAXJ > 0) the scan waits for it first, so that its small
+  // loads are not queued behind the scan's; with many (MAXJ == 0: long,
+  // compute-heavy runs) the first batch of index loads goes out before the
+  // wait (128K x 8: 96.3 against 92.2 us; 64K x 32: 483 against 551 us).
+  bool waited = false;
+  if constexpr (MAXJ > 0) {
+    pdl_wait();
+    waited = true;
+  }
   extern __shared__ uint32_t shist[];                  // [heads of the group][kBins]
   __shared__ float qs[MAXJ > 0 ? 1 : kMaxHeadsPerGroup][RTP_R];
   const int64_t total = (int64_t)B * gh.n_ag * L;
@@ -177,10 +186,8 @@ decode_scan_kernel(const float* __restrict__ qt, const IndexRef index, int B, in
         for (int c = 0; c < RTP_R; ++c) q[jj][c] = __ldg(qt + ((size_t)b * Hr + j) * RTP_R + c);
         srow[jj] = w.scores + ((size_t)b * Hr + j) * L;
       }
-    } else {
-      for (int e = threadIdx.x; e < n * RTP_R; e += kScanThreads)
-        qs[e / RTP_R][e % RTP_R] = qt[((size_t)b * Hr + gh.j[g][e / RTP_R]) * RTP_R + e % RTP_R];
     }
+    bool q_loaded = MAXJ > 0;                          // MAXJ == 0: q~ rows after the first loads
     for (int e = threadIdx.x; e < n * kBins; e += kScanThreads) shist[e] = 0u;
     __syncthreads();
     const uint4* krow = kindex + ((size_t)b * Hkv + g) * (size_t)kcap * 2;
@@ -201,6 +208,13 @@ decode_scan_kernel(const float* __restrict__ qt, const IndexRef index, int B, in
             hi[t] = __ldcs(krow + (size_t)u * 2 + 1);
           }
         }
+      }
+      if (!q_loaded) {
+        if (!waited) { pdl_wait(); waited = true; }
+        for (int e = threadIdx.x; e < n * RTP_R; e += kScanThreads)
+          qs[e / RTP_R][e % RTP_R] = __ldg(qt + ((size_t)b * Hr + gh.j[g][e / RTP_R]) * RTP_R + e % RTP_R);
+        __syncthreads();
+        q_loaded = true;
       }
 #pragma unroll
       for (int t = 0; t < BATCH; ++t) {

@@ -292,11 +292,19 @@ kc_select_kernel(const ClusterSelParams p, const SelWs w) {
   //    clustered prefix, marked in the token bitmap
   const int32_t* off = p.offsets + (int64_t)bh * (p.C + 1);
   const int32_t* mem = p.members + (int64_t)bh * p.L0;
+  // one warp per probed cluster (every warp's loads in flight together)
   const int n_pr = min(p.n_probe, p.C);
-  for (int e = 0; e < n_pr; ++e) {
-    const int c = __ldcg(probe + e);
-    const int a0 = __ldg(off + c), a1 = __ldg(off + c + 1);
-    for (int x = a0 + tid; x < a1; x += kSelThreads) {
+  const int lane = tid & 31, warp = tid >> 5;
+  for (int e = warp; e < n_pr; e += kSelThreads / 32) {
+    int a0 = 0, a1 = 0;
+    if (lane == 0) {
+      const int c = __ldcg(probe + e);
+      a0 = __ldg(off + c);
+      a1 = __ldg(off + c + 1);
+    }
+    a0 = __shfl_sync(0xffffffffu, a0, 0);
+    a1 = __shfl_sync(0xffffffffu, a1, 0);
+    for (int x = a0 + lane; x < a1; x += 32) {
       const int u = __ldg(mem + x);
       atomicOr(&sm.bits[u >> 5], 1u << (u & 31));
     }
@@ -321,15 +329,37 @@ kc_select_kernel(const ClusterSelParams p, const SelWs w) {
     while (v) {
       const int bit = __ffs(v) - 1;
       v &= v - 1;
-      const int u = wi * 32 + bit;
-      float x[16];
-      load_row16(p.kindex + ((int64_t)bh * p.cap + u) * 2, x);
+      ct[pos++] = wi * 32 + bit;
+    }
+  }
+  __syncthreads();
+  // the candidates' scores, two rows of a thread in flight together
+  for (int i0 = 0; i0 < n_cand; i0 += 2 * kSelThreads) {
+    int us[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int i = i0 + t * kSelThreads + tid;
+      us[t] = i < n_cand ? __ldcg(ct + i) : -1;
+    }
+    uint4 lo[2], hi[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+      if (us[t] >= 0) {
+        const uint4* r = p.kindex + ((int64_t)bh * p.cap + us[t]) * 2;
+        lo[t] = __ldg(r);
+        hi[t] = __ldg(r + 1);
+      }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if (us[t] < 0) continue;
+      const uint32_t v8[8] = {lo[t].x, lo[t].y, lo[t].z, lo[t].w, hi[t].x, hi[t].y, hi[t].z, hi[t].w};
       float acc = 0.f;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) acc = fmaf(q[c], x[c], acc);
-      ct[pos] = u;
-      sk[pos] = f2key(acc);
-      ++pos;
+      for (int c = 0; c < 8; ++c) {
+        acc = fmaf(q[2 * c], bf16_lo(v8[c]), acc);
+        acc = fmaf(q[2 * c + 1], bf16_hi(v8[c]), acc);
+      }
+      sk[i0 + t * kSelThreads + tid] = f2key(acc);
     }
   }
   __syncthreads();

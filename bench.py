@@ -637,8 +637,8 @@ def _time_graph(fn, stream, flush, reps=10):
 
 def run_preset_configs(dev, peaks, stream, flush):
     """The rows beyond the hot path, each on the workload shape it belongs to:
-    the 128K decode over a clustered key index (two-level selection, then the
-    attention), Orthros' decode (SWA plus a full cross-attention over the
+    the 128K decode over a clustered key index (one rtp_decode_step_clustered
+    call: projection, two-level selection, attention), Orthros' decode (SWA plus a full cross-attention over the
     128K cache, every head), and the triangle-mask prefill on the 128K
     all-sparse shape (sink block, 2048-token band, last 2048 queries dense)."""
     import long_context_hybrid_b200 as rtp
@@ -659,16 +659,14 @@ def run_preset_configs(dev, peaks, stream, flush):
     qt = torch.empty(B, len(ret), R, dtype=torch.float32, device=dev)
     idx = torch.empty(B, len(ret), cfg.topk, dtype=torch.int32, device=dev)
     od = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
-    ws_sel = torch.empty(rtp.lib().rtp_workspace_size_select_decode_clustered(B, len(ret), cl.C, n_probe, L),
-                         dtype=torch.uint8, device=dev)
-    ws_att = torch.empty(rtp.lib().rtp_workspace_size_decode_attn_hybrid(B, L, Hq, cfg.topk, cfg.window),
-                         dtype=torch.uint8, device=dev)
+    ws_step = torch.empty(rtp.lib().rtp_workspace_size_decode_step_clustered(B, L, Hq, len(ret), cl.C, n_probe,
+                                                                             cfg.topk, cfg.window),
+                          dtype=torch.uint8, device=dev)
+    rtp.index_project(qd.unsqueeze(1), P, ret, kv_ret, out=qt.view(B, len(ret), 1, R))   # for the byte count
 
     def clustered_step():
-        rtp.index_project(qd.unsqueeze(1), P, ret, kv_ret, out=qt.view(B, len(ret), 1, R))
-        rtp.select_decode_clustered(qt, kindex, cl, kv_ret, n_probe, cfg.topk, idx=idx, ws=ws_sel)
-        rtp.decode_attn_hybrid(qd, kc, vc, od, ret, idx, cfg.ret_window, swa_heads, cfg.window, cfg.sink, None,
-                               ws_att)
+        rtp.decode_step_clustered(qd, P, kindex, cl, kc, vc, od, ret, idx, cfg.ret_window, swa_heads, cfg.window,
+                                  cfg.topk, n_probe, sink=cfg.sink, ws=ws_step)
     ms = _time_graph(clustered_step, stream, flush)
     counts = torch.diff(cl.offsets.long(), dim=-1)                         # [B, Hkv, C]
     probed = 0
@@ -694,7 +692,7 @@ def run_preset_configs(dev, peaks, stream, flush):
         "value": round(B / (ms / 1e3), 1), "unit": "tok/s", "ms_per_step": round(ms, 4),
         "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
                      "bytes_per_step": total}}
-    del d, qd, kc, vc, P, kindex, cl, qt, idx, od, ws_sel, ws_att, orth, o_ca
+    del d, qd, kc, vc, P, kindex, cl, qt, idx, od, ws_step, orth, o_ca
     # triangle mask on the 128K all-sparse shape
     pc = synth.PREFILL_128K_ALL
     dp = synth.make_prefill(pc, device=dev)

@@ -442,6 +442,39 @@ RTP_API rtp_status rtp_decode_step(const void* q, const void* P, const void* kin
                                    void* ws, size_t ws_bytes, rtp_stream_t stream);
 
 /*
+ * rtp_decode_step_clustered - one decode step as rtp_decode_step, with the
+ * retrieval heads' tokens chosen by the two-level selection over a clustered
+ * key index (as rtp_select_decode_clustered) instead of the scan of the whole
+ * index.
+ *   Sources: RTPurboV2 article (th-motor.com), the sequence-dimension
+ *   compression paragraph and the Qwen3-Coder-30B-A3B recipe (clustered K
+ *   cache for the retrieval heads); the 128K decode workload statement for
+ *   the union with the window and token 0. As for rtp_decode_step, the
+ *   grouping lets the attention stream its window while the selection runs
+ *   (the clustered selection occupies one SM per (sequence, retrieval head)).
+ *   Arguments as rtp_decode_step, plus:
+ *   centroids, offsets, members  from rtp_kcluster_build over the first L0
+ *            rows of kindex (C clusters); rows L0 .. L-1 (appended after the
+ *            build) are always candidates.
+ *   n_probe  clusters probed per (sequence, retrieval head), >= 1.
+ *   ws       rtp_workspace_size_decode_step_clustered(B, L, Hq, Hr, C, n_probe,
+ *            topk, max(ret_window, swa_window)) bytes, 256-byte aligned; its
+ *            first word is the status word read by rtp_get_device_status.
+ *   Hr >= 1; 1 <= L0 <= L <= 262144 (RTP_ERR_UNSUPPORTED beyond); other
+ *   limits as in the calls it combines. Asynchronous on `stream`.
+ */
+RTP_API size_t rtp_workspace_size_decode_step_clustered(int B, int L, int Hq, int Hr, int C, int n_probe, int topk,
+                                                        int window);
+RTP_API rtp_status rtp_decode_step_clustered(const void* q, const void* P, const void* kindex, int64_t kindex_cap,
+                                             const float* centroids, const int32_t* offsets,
+                                             const int32_t* members, int L0, int C, int n_probe, const void* kc,
+                                             rtp_strides ks, const void* vc, rtp_strides vs, void* o, int B, int L,
+                                             int Hq, int Hkv, const int32_t* ret_heads, int Hr, int topk,
+                                             int ret_window, int sink, const int32_t* swa_heads, int n_swa,
+                                             int swa_window, float scale, int32_t* idx, void* ws, size_t ws_bytes,
+                                             rtp_stream_t stream);
+
+/*
  * rtp_sparse_attn_decode_noalloc - rtp_sparse_attn_decode without a workspace
  * argument and without allocating anything.
  *   The method's sources have no counterpart of this call: it exists for

@@ -72,6 +72,9 @@ _SIGNATURES = {
     "rtp_decode_step": (_I, [_P, _P, _P, _L, _P, _P, _P, Strides, _P, Strides, _P, _I, _I, _I, _I, _c_i32p, _I, _I,
                              _I, _I,
                              _c_i32p, _I, _I, _F, _P, _P, _SZ, _P]),
+    "rtp_workspace_size_decode_step_clustered": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "rtp_decode_step_clustered": (_I, [_P, _P, _P, _L, _P, _P, _P, _I, _I, _I, _P, Strides, _P, Strides, _P, _I, _I,
+                                       _I, _I, _c_i32p, _I, _I, _I, _I, _c_i32p, _I, _I, _F, _P, _P, _SZ, _P]),
     "rtp_workspace_size_swa": (_SZ, [_I, _I, _I, _I, _I]),
     "rtp_swa": (_I, [_P, Strides, _P, Strides, _P, Strides, _P, Strides, _I, _I, _I, _I, _I, _I,
                      _c_i32p, _I, _I, _F, _P, _SZ, _P]),
@@ -398,6 +401,33 @@ def decode_step(q, P, kindex, kc, vc, o, ret_heads: Sequence[int], idx, ret_wind
     return o
 
 
+def decode_step_clustered(q, P, kindex, clusters: "KeyClusters", kc, vc, o, ret_heads: Sequence[int], idx,
+                          ret_window: int, swa_heads: Sequence[int], swa_window: int, topk: int, n_probe: int,
+                          sink: int = 1, scale: Optional[float] = None, ws: Optional[torch.Tensor] = None,
+                          stream=None, L: Optional[int] = None):
+    """One decode step in one call with the two-level clustered selection:
+    q~ projection, the n_probe best clusters then the top-k tokens among
+    their members and the rows appended after the build (into idx), and the
+    attention of retrieval and streaming heads. Shapes as decode_step;
+    clusters from kcluster_build over the first clusters.L0 rows."""
+    B, Hq, D = q.shape
+    Hkv = kc.shape[2]
+    L = kc.shape[1] if L is None else L
+    assert kindex.is_contiguous() and kindex.shape[2] >= L
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    wmax = max(ret_window, swa_window if swa_heads else 0)
+    need = lib().rtp_workspace_size_decode_step_clustered(B, L, Hq, len(ret_heads), clusters.C, n_probe, topk, wmax)
+    buf, nbytes = _ws(need, q.device, ws)
+    _check(lib().rtp_decode_step_clustered(q.data_ptr(), P.data_ptr(), kindex.data_ptr(), kindex.shape[2],
+                                           clusters.centroids.data_ptr(), clusters.offsets.data_ptr(),
+                                           clusters.members.data_ptr(), clusters.L0, clusters.C, n_probe,
+                                           kc.data_ptr(), _strides4(kc), vc.data_ptr(), _strides4(vc), o.data_ptr(),
+                                           B, L, Hq, Hkv, _i32(ret_heads), len(ret_heads), topk, ret_window, sink,
+                                           _i32(swa_heads), len(swa_heads), swa_window, scale, idx.data_ptr(),
+                                           _wsptr(buf), nbytes, _stream(stream)), "rtp_decode_step_clustered")
+    return o
+
+
 def swa(q, k, v, o, heads: Sequence[int], window: int, q_pos0: int = 0,
         scale: Optional[float] = None, ws: Optional[torch.Tensor] = None, stream=None):
     """Streaming-head sliding-window attention. q/o [B,Nq,Hq,D], k/v [B,Nk,Hkv,D]."""
@@ -576,5 +606,6 @@ class DecodeStep:
 __all__ = ["lib", "RtpError", "index_project", "index_append", "index_quantize", "select_prefill", "select_decode",
            "select_decode_q8", "KeyClusters", "kcluster_build", "select_decode_clustered",
            "sparse_attn_prefill", "triangle_prefill", "sparse_attn_decode", "swa", "decode_attn_hybrid",
+           "decode_step", "decode_step_clustered",
            "PrefillLayer", "DecodeStep", "OrthrosStep",
            "kv_of", "LIB_PATH"]

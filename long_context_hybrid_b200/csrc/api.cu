@@ -490,6 +490,72 @@ rtp_status rtp_decode_step(const void* q, const void* P, const void* kindex, int
                                         /*early_start=*/Hr > 0, max_ctas));
 }
 
+size_t rtp_workspace_size_decode_step_clustered(int B, int L, int Hq, int Hr, int C, int n_probe, int topk,
+                                                int window) {
+  if (B < 1 || L < 1 || Hq < 1 || Hr < 1 || C < 1 || n_probe < 1 || topk < 1 || window < 1) return 0;
+  return align256(decode_attn_ws_bytes(B, L, Hq, topk, window)) + step_qt_bytes(B, Hr) +
+         align256(kcluster_select_ws_bytes(B, Hr, C, n_probe, L));
+}
+
+rtp_status rtp_decode_step_clustered(const void* q, const void* P, const void* kindex, int64_t kindex_cap,
+                                     const float* centroids, const int32_t* offsets, const int32_t* members, int L0,
+                                     int C, int n_probe, const void* kc, rtp_strides ks, const void* vc,
+                                     rtp_strides vs, void* o, int B, int L, int Hq, int Hkv,
+                                     const int32_t* ret_heads, int Hr, int topk, int ret_window, int sink,
+                                     const int32_t* swa_heads, int n_swa, int swa_window, float scale, int32_t* idx,
+                                     void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  if (!q || !P || !kindex || !centroids || !offsets || !members || !kc || !vc || !o || !idx || !ret_heads)
+    return RTP_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return RTP_ERR_INVALID_ARG;
+  if (Hr < 1 || n_swa < 0 || Hr + n_swa > kMaxHeads) return RTP_ERR_INVALID_ARG;
+  if (Hq / Hkv > 16 || Hkv > 16) return RTP_ERR_UNSUPPORTED;
+  if (C < 1 || n_probe < 1 || topk < 1 || ret_window < 1) return RTP_ERR_INVALID_ARG;
+  if (L0 < 1 || L < L0 || kindex_cap < L) return RTP_ERR_INVALID_ARG;
+  if (L > kClusterSelectMaxTokens || topk > kMaxDecodeTopk) return RTP_ERR_UNSUPPORTED;
+  if (n_swa > 0 && swa_window < 1) return RTP_ERR_INVALID_ARG;
+  if (sink < 0 || sink > kMaxSink || !(scale > 0.f)) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(o) || !aligned16(P) || !aligned16(kindex) ||
+      !aligned16(idx))
+    return RTP_ERR_INVALID_ARG;
+  if (!stride_ok(ks) || !stride_ok(vs)) return RTP_ERR_INVALID_ARG;
+  int32_t all[kMaxHeads];
+  for (int i = 0; i < Hr; ++i) all[i] = ret_heads[i];
+  for (int i = 0; i < n_swa; ++i) all[Hr + i] = swa_heads ? swa_heads[i] : -1;
+  rtp_status st = check_heads(all, Hr + n_swa, Hq);
+  if (st != RTP_OK) return st;
+  const int G = Hq / Hkv;
+  int32_t kv_of[kMaxHeads];
+  for (int i = 0; i < Hr; ++i) kv_of[i] = ret_heads[i] / G;
+  const int wmax = ret_window > swa_window || n_swa == 0 ? ret_window : swa_window;
+  const size_t need = rtp_workspace_size_decode_step_clustered(B, L, Hq, Hr, C, n_probe, topk, wmax);
+  if (!ws || ws_bytes < need || !aligned256(ws)) return RTP_ERR_WORKSPACE;
+  if ((st = check_device()) != RTP_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* base = static_cast<char*>(ws);
+  float* qt = reinterpret_cast<float*>(base + align256(decode_attn_ws_bytes(B, L, Hq, topk, wmax)));
+  void* ws_sel = reinterpret_cast<char*>(qt) + step_qt_bytes(B, Hr);
+  // q~ = q . P for the retrieval heads (fp32, unrounded), then the two-level top-k
+  cudaError_t e = launch_project(q, (int64_t)Hq * RTP_D, (int64_t)Hq * RTP_D, RTP_D, B, 1, P, ret_heads, kv_of, Hr,
+                                 qt, 1, s);
+  if (e != cudaSuccess) return from_cuda(e);
+  e = launch_kcluster_select(qt, kindex, kindex_cap, centroids, offsets, members, B, L0, L, Hr, Hkv, C, kv_of,
+                             n_probe, topk, idx, ws_sel, s);
+  if (e != cudaSuccess) return from_cuda(e);
+  // The selection holds one SM per (sequence, retrieval head) and no
+  // attention CTA fits beside it: launch as many as fit on the others (two
+  // per SM), all streaming their window while the selection runs.
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                cudaSuccess)
+    return RTP_ERR_CUDA;
+  const int n_sel = B * Hr;
+  const int max_ctas = n_sel < sms ? 2 * (sms - n_sel) : 0;
+  return from_cuda(launch_decode_hybrid(q, (int64_t)Hq * RTP_D, RTP_D, kc, ks.b, ks.n, ks.h, vc, vs.b, vs.n, vs.h,
+                                        o, (int64_t)Hq * RTP_D, RTP_D, B, L, L - 1, Hq, Hkv, ret_heads, Hr, idx, topk,
+                                        ret_window, sink, swa_heads, n_swa, swa_window, scale, base, s,
+                                        /*early_start=*/true, max_ctas));
+}
+
 rtp_status rtp_decode_attn_hybrid(const void* q, const void* kc, rtp_strides ks, const void* vc, rtp_strides vs,
                                   void* o, int B, int L, int Hq, int Hkv,
                                   const int32_t* ret_heads, int Hr, const int32_t* idx, int topk, int ret_window,

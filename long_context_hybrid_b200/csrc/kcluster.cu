@@ -265,6 +265,7 @@ __global__ void __launch_bounds__(kSelThreads)
 kc_select_kernel(const ClusterSelParams p, const SelWs w) {
   extern __shared__ __align__(16) unsigned char kc_smem[];
   SelSmem& sm = *reinterpret_cast<SelSmem*>(kc_smem);
+  pdl_trigger();         // a decode step's attention may launch; it waits for this grid before reading idx
   const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int row = b * p.Hr + j;
   const int bh = b * p.Hkv + p.kv[j];

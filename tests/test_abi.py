@@ -139,6 +139,20 @@ def test_rejects_bad_arguments_without_launching(L):
                              _heads([1]), 1, 64, f, fake, fake, 1 << 24, None) == INVALID
     assert L.rtp_decode_step(fake, fake, fake, 640, None, None, fake, ks, fake, ks, fake, 1, 640, 8, 2, _heads([0]), 1, (1 << 22) + 1, 64, 1,
                              _heads([1]), 1, 64, f, fake, fake, 1 << 30, None) == UNSUP
+    # clustered decode step: clusters required, L0 within L, the clustered
+    # selection's token limit, workspace checked
+    def step_cl(centroids=fake, L0=100, n=640, cap=640, ws=fake, ws_bytes=1 << 24):
+        return L.rtp_decode_step_clustered(fake, fake, fake, cap, centroids, fake, fake, L0, 4, 2, fake, ks, fake, ks,
+                                           fake, 1, n, 8, 2, _heads([0]), 1, 16, 64, 1, _heads([1]), 1, 64, f, fake,
+                                           ws, ws_bytes, None)
+    assert step_cl(centroids=None) == INVALID
+    assert step_cl(L0=700) == INVALID
+    assert step_cl(cap=600) == INVALID
+    assert step_cl(n=300000, cap=300000) == UNSUP
+    assert step_cl(ws=None, ws_bytes=0) == WS
+    whole = L.rtp_workspace_size_decode_step_clustered(4, 20000, 32, 5, 313, 32, 2048, 4096)
+    assert whole >= (L.rtp_workspace_size_decode_attn_hybrid(4, 20000, 32, 2048, 4096)
+                     + L.rtp_workspace_size_select_decode_clustered(4, 5, 313, 32, 20000) + 4 * 5 * 16 * 4)
     # its workspace holds the three calls' workspaces
     B, Lc, Hq, Hr, k, w = 4, 20000, 32, 5, 2048, 4096
     whole = L.rtp_workspace_size_decode_step(B, Lc, Hq, Hr, k, w)

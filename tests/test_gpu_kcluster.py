@@ -133,3 +133,49 @@ def test_clustered_decode_step_attention_matches_oracle():
             recall.append(len(np.intersect1d(sel, flat[b, j])) / cfg.topk)
     assert_attn_close(np.stack(outs), np.stack(refs), "clustered decode attention")
     print(f"recall of the flat top-{cfg.topk} by 32 probed clusters of 64: mean {np.mean(recall):.3f}")
+
+
+def test_clustered_decode_step_call_matches_the_calls_and_the_oracle():
+    """rtp_decode_step_clustered (projection, two-level selection and the
+    attention streaming its window while the selection runs) selects exactly
+    what the separate calls select; its outputs agree with theirs within
+    2^-10 + 2^-6 |o| (its attention runs on fewer CTAs, so its partials group
+    the keys differently) and with the oracle over its selection."""
+    cfg = synth.DECODE_128K
+    B, L, L0 = 2, 16384, 16000
+    d = synth.make_decode(cfg, device=DEV, B=B, L=L, seed=cfg.seed + 23)
+    q, kc, vc, P = d["q"], d["kc"], d["vc"], d["P"]
+    kindex = rtp.index_project(kc, P, list(range(cfg.Hkv)), list(range(cfg.Hkv)))
+    cl = rtp.kcluster_build(kindex, L0, 64, 2)
+    ret = list(cfg.ret_heads)
+    kv_ret = [h // 8 for h in ret]
+    swa_heads = [h for h in range(cfg.Hq) if h not in ret]
+    n_probe = 16
+    o1 = torch.zeros(B, cfg.Hq, 128, dtype=torch.bfloat16, device=DEV)
+    idx1 = torch.empty(B, len(ret), cfg.topk, dtype=torch.int32, device=DEV)
+    rtp.decode_step_clustered(q, P, kindex, cl, kc, vc, o1, ret, idx1, cfg.ret_window, swa_heads, cfg.window,
+                              cfg.topk, n_probe, sink=1)
+    qt = rtp.index_project(q.unsqueeze(1), P, ret, kv_ret, out_dtype=torch.float32).view(B, len(ret), 16)
+    idx2 = rtp.select_decode_clustered(qt, kindex, cl, kv_ret, n_probe, cfg.topk, L=L)
+    o2 = torch.zeros_like(o1)
+    rtp.decode_attn_hybrid(q, kc, vc, o2, ret, idx2, cfg.ret_window, swa_heads, cfg.window, 1)
+    torch.cuda.synchronize()
+    assert torch.equal(idx1, idx2)
+    a, b = o1.float(), o2.float()
+    tol = 2.0 ** -10 + torch.maximum(a.abs(), b.abs()) * 2.0 ** -6
+    assert bool(((a - b).abs() <= tol).all()), float((a - b).abs().max())
+    idx1 = idx1.cpu().numpy()
+    scale = 1 / math.sqrt(128)
+    outs, refs = [], []
+    for bb in range(B):
+        for j, h in enumerate(ret):
+            g = kv_ret[j]
+            att = O.decode_attended(idx1[bb, j][idx1[bb, j] >= 0], L, cfg.ret_window, 1)
+            refs.append(O.attend_decode(q[bb, h].cpu(), kc[bb, :, g].cpu(), vc[bb, :, g].cpu(), att, scale))
+            outs.append(o1[bb, h].float().cpu().numpy())
+        for h in swa_heads[:4]:
+            g = h // 8
+            att = np.arange(max(0, L - cfg.window), L)
+            refs.append(O.attend_decode(q[bb, h].cpu(), kc[bb, :, g].cpu(), vc[bb, :, g].cpu(), att, scale))
+            outs.append(o1[bb, h].float().cpu().numpy())
+    assert_attn_close(np.stack(outs), np.stack(refs), "clustered decode step")

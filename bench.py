@@ -227,9 +227,9 @@ NOMINAL_HBM_GBS = 7700.0
 NCU_TRAFFIC = {
     # one decode step of the 128K x 8 workload at full size (zero + projection,
     # scan, filter, attention, merge): profiles/decode_128k_b8.md
-    "decode_step": {"bytes_per_unit": 338594816 / (8 * 131072), "unit": "cached token",
+    "decode_step": {"bytes_per_unit": 338815232 / (8 * 131072), "unit": "cached token",
                     "sources": ["select.cu", "decode_attn.cu", "rtp_common.cuh", "rtp_internal.h", "api.cu"],
-                    "digest": "169706ae0555f20b"},
+                    "digest": "9501a8709f25eabd"},
 }
 
 

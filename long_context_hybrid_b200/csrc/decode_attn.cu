@@ -478,7 +478,6 @@ decode_merge_kernel(const DecodeParams p, int n_ctas, int* status) {
 
 namespace {
 int n_gathered_chunks(int topk, int sink) { return (topk + sink + kChunk - 1) / kChunk; }
-size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 }  // namespace
 
 size_t decode_attn_ws_bytes(int B, int L, int n_heads, int topk, int window) {

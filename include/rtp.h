@@ -432,6 +432,10 @@ RTP_API rtp_status rtp_decode_attn_hybrid(const void* q, const void* kc, rtp_str
  *            max(ret_window, swa_window)) bytes, 256-byte aligned; its first
  *            word is the status word read by rtp_get_device_status.
  *   Limits as in the three calls it combines. Asynchronous on `stream`.
+ *   idx equals what rtp_select_decode writes; the attention runs on as many
+ *   thread blocks as fit beside the selection's last kernel, so its split of
+ *   the keys (and hence the fp32 rounding of o) can differ from a separate
+ *   rtp_decode_attn_hybrid call's.
  */
 RTP_API size_t rtp_workspace_size_decode_step(int B, int L, int Hq, int Hr, int topk, int window);
 RTP_API rtp_status rtp_decode_step(const void* q, const void* P, const void* kindex, int64_t kindex_cap,

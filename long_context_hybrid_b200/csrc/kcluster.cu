@@ -241,9 +241,12 @@ SelWs sel_ws(void* base, int rows, int C, int n_probe, int L) {
   return w;
 }
 
+constexpr int kSelKeys = 8192;      // centroid or candidate keys (and tokens) kept in shared memory
 struct SelSmem {
   TopkSmem<kSelThreads> tk;
   uint32_t bits[kSelWords];
+  uint32_t keys[kSelKeys];            // centroid keys, then candidate keys
+  int32_t toks[kSelKeys];             // candidate tokens in token order
   float q[16];
   int n_cand;
 };
@@ -277,17 +280,21 @@ kc_select_kernel(const ClusterSelParams p, const SelWs w) {
 #pragma unroll
   for (int c = 0; c < 16; ++c) q[c] = sm.q[c];
   // 1. centroid scores, exact top-n_probe of them (ascending cluster ids)
+  //    (keys in shared memory when they fit, else in the workspace)
   uint32_t* ck = w.ckey + (int64_t)row * p.C;
+  const bool ck_sm = p.C <= kSelKeys;
   const float* mu = p.mu + (int64_t)bh * p.C * 16;
   for (int i = tid; i < p.C; i += kSelThreads) {
     float acc = 0.f;
 #pragma unroll
     for (int c = 0; c < 16; ++c) acc = fmaf(q[c], __ldg(mu + (int64_t)i * 16 + c), acc);
-    ck[i] = f2key(acc);
+    if (ck_sm) sm.keys[i] = f2key(acc);
+    else ck[i] = f2key(acc);
   }
   __syncthreads();
   int32_t* probe = w.probe + (int64_t)row * p.n_probe;
-  block_topk_ascending<kSelThreads>([&](int i) { return __ldcg(ck + i); }, p.C, p.n_probe, probe, sm.tk);
+  block_topk_ascending<kSelThreads>([&](int i) { return ck_sm ? sm.keys[i] : __ldcg(ck + i); }, p.C, p.n_probe,
+                                    probe, sm.tk);
   __syncthreads();
   // 2. candidates: the probed clusters' members and the tokens past the
   //    clustered prefix, marked in the token bitmap
@@ -323,6 +330,7 @@ kc_select_kernel(const ClusterSelParams p, const SelWs w) {
   }
   int n_cand;
   int pos = block_exclusive_scan<kSelThreads>(cnt, n_cand, sm.tk.scan);
+  const bool c_sm = n_cand <= kSelKeys;           // candidates (tokens, keys) in shared memory
   for (int qq = 0; qq < per; ++qq) {
     const int wi = tid * per + qq;
     if (wi >= W) break;
@@ -330,7 +338,8 @@ kc_select_kernel(const ClusterSelParams p, const SelWs w) {
     while (v) {
       const int bit = __ffs(v) - 1;
       v &= v - 1;
-      ct[pos++] = wi * 32 + bit;
+      if (c_sm) sm.toks[pos++] = wi * 32 + bit;
+      else ct[pos++] = wi * 32 + bit;
     }
   }
   __syncthreads();
@@ -340,7 +349,7 @@ kc_select_kernel(const ClusterSelParams p, const SelWs w) {
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       const int i = i0 + t * kSelThreads + tid;
-      us[t] = i < n_cand ? __ldcg(ct + i) : -1;
+      us[t] = i < n_cand ? (c_sm ? sm.toks[i] : __ldcg(ct + i)) : -1;
     }
     uint4 lo[2], hi[2];
 #pragma unroll
@@ -360,17 +369,19 @@ kc_select_kernel(const ClusterSelParams p, const SelWs w) {
         acc = fmaf(q[2 * c], bf16_lo(v8[c]), acc);
         acc = fmaf(q[2 * c + 1], bf16_hi(v8[c]), acc);
       }
-      sk[i0 + t * kSelThreads + tid] = f2key(acc);
+      if (c_sm) sm.keys[i0 + t * kSelThreads + tid] = f2key(acc);
+      else sk[i0 + t * kSelThreads + tid] = f2key(acc);
     }
   }
   __syncthreads();
   // 4. top-k by (score, token): candidate positions are in token order
   int32_t* out = p.idx + (int64_t)row * p.topk;
-  block_topk_ascending<kSelThreads>([&](int i) { return __ldcg(sk + i); }, n_cand, p.topk, out, sm.tk);
+  block_topk_ascending<kSelThreads>([&](int i) { return c_sm ? sm.keys[i] : __ldcg(sk + i); }, n_cand, p.topk, out,
+                                    sm.tk);
   __syncthreads();
   for (int i = tid; i < p.topk; i += kSelThreads) {
-    const int x = out[i];
-    if (x >= 0) out[i] = __ldcg(ct + x);
+    const int x = __ldcg(out + i);
+    if (x >= 0) out[i] = c_sm ? sm.toks[x] : __ldcg(ct + x);
   }
 }
 

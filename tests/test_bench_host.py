@@ -91,3 +91,38 @@ def test_triangle_pairs_match_oracle_key_sets():
     for N, sink, wb, last in [(1024, 1, 2, 256), (640, 0, 3, 0), (512, 2, 1, 512), (1536, 1, 4, 320), (960, 3, 2, 64)]:
         want = sum(len(O.triangle_keys(t, N, sink, wb, last)) for t in range(N))
         assert bench.triangle_pairs(N, sink, wb, last) == want, (N, sink, wb, last)
+
+
+def test_decode_bytes_counts_every_row_the_step_needs_once():
+    """The decode roofline's bytes: per (sequence, KV group) every row the
+    attention needs (the window of every KV group, and for the groups of
+    retrieval heads the sink and the selected rows outside the window, each
+    row once however many heads select it), plus the key index of the
+    retrieval groups and q / o; checked against explicit sets built from the
+    oracle's attended sets."""
+    from types import SimpleNamespace
+    cfg = SimpleNamespace(Hq=8, Hkv=4, ret_heads=[0, 1, 5], window=40, ret_window=40, sink=1)
+    B, L, k = 3, 300, 25
+    rs = np.random.default_rng(3)
+    idx = torch.full((B, len(cfg.ret_heads), k), -1, dtype=torch.int32)
+    for b in range(B):
+        for j in range(len(cfg.ret_heads)):
+            sel = np.sort(rs.choice(L, size=k - 3, replace=False))
+            idx[b, j, :len(sel)] = torch.from_numpy(sel.astype(np.int32))
+    got = bench.decode_bytes(cfg, idx, L, B)
+    G = cfg.Hq // cfg.Hkv
+    rows = 0
+    for b in range(B):
+        for g in range(cfg.Hkv):
+            need = set(range(L - cfg.window, L))
+            for j, h in enumerate(cfg.ret_heads):
+                if h // G == g:
+                    sel = idx[b, j].numpy()
+                    need |= set(O.decode_attended(sel[sel >= 0], L, cfg.ret_window, cfg.sink).tolist())
+            rows += len(need)
+    kv_ret = {h // G for h in cfg.ret_heads}
+    want_scan = B * len(kv_ret) * L * 16 * 2
+    assert got["scan"] == want_scan
+    assert got["window"] + got["gathered"] == rows * 128 * 2 * 2
+    assert got["qo"] == B * cfg.Hq * 128 * 2 * 2
+    assert got["total"] == want_scan + rows * 128 * 2 * 2 + got["qo"]
